@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE decode hot path on B200.
+
+Default workload (one "step"): one decode token through 30 MoE layers back to
+back, each layer = 8-bit router GEMV -> softmax -> top-8 of 128 experts ->
+8 gathered routed SwiGLU experts + the resident shared expert (affine 4-bit,
+group 64, hidden 2816, intermediate 704) -> weighted combine.  Every layer has
+its own seeded weights (12.96 GB in total, far larger than the 126 MB L2, so
+each step streams its 915 MB of weights from HBM) and its own seeded input.
+
+Metric: MoE decode layers/s (whole job, all ranks).  The JSON line also gives
+the weight-stream GB/s of the dominant kernel against the measured HBM peak
+(`roofline`), the same metric end to end through host buffers (`e2e`), and the
+CPU oracle timed on a bounded sample (`cpu_baseline`).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload moe_decode|qgemv|router|prefill]
+
+Under torchrun every rank runs an independent replica (weak scaling); the
+timed region is bracketed by a barrier and device synchronisation, and the
+slowest rank's time is reported.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+E, H, I, TOPK, LAYERS = 128, 2816, 704, 8, 30
+# algorithmic bytes (packed codes + fp16 scales + fp16 biases)
+MAT_BYTES = I * H // 2 + 2 * I * (H // 64) * 2            # one 704x2816 4-bit matrix
+EXPERT_BYTES = 3 * MAT_BYTES                                # gate + up + down
+ROUTER_BYTES = E * H + 2 * E * (H // 64) * 2                # 128x2816 8-bit
+LAYER_BYTES = ROUTER_BYTES + (TOPK + 1) * EXPERT_BYTES      # 30,491,648
+GATEUP_BYTES = (TOPK + 1) * 2 * MAT_BYTES + H * 2 + (TOPK + 1) * I * 4
+DOWN_BYTES = (TOPK + 1) * MAT_BYTES + (TOPK + 1) * I * 4 + H * 2
+ROUTER_CALL_BYTES = ROUTER_BYTES + H * 2 + TOPK * 8
+
+# DRAM traffic per launch of the dominant kernel from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
+# source it was taken on (sha256 of csrc/expert.cu); otherwise reported null.
+NCU_TRAFFIC = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["moe_decode", "qgemv", "router", "prefill"],
+                    default="moe_decode")
+    ap.add_argument("--layers", type=int, default=LAYERS)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="time budget of the CPU-oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------- helpers --
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+def source_sha(name):
+    with open(os.path.join(ROOT, "moe_expert_gemv_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.device_index = device_index
+
+    def start(self):
+        try:
+            import torch
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(self.device_index).uuid)
+            cmd = ["nvidia-smi", "-i", uuid, "--query-gpu=" + self.FIELDS,
+                   "--format=csv,noheader,nounits", "-lms", "100"]
+            self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, AttributeError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(", ") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+class Dist:
+    def __init__(self, want_gpu=True):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+        if self.world > 1:
+            import datetime
+            import torch
+            import torch.distributed as dist
+            backend = "nccl" if (want_gpu and torch.cuda.is_available()) else "gloo"
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, v):
+        if not self.pg:
+            return v
+        import torch
+        import torch.distributed as dist
+        dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([float(v)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def timed_replays(fn, iters, dist=None):
+    """Device time (ms) of `iters` calls of fn on the current stream."""
+    import torch
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(iters):
+        fn()
+    e.record()
+    e.synchronize()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e)
+
+
+# ---------------------------------------------------- CPU oracle baseline --
+def oracle_decode_layers(seconds, seed, max_layers=None, m=None):
+    """Run the CPU oracle on decode layers (router + shared + 8 routed experts)
+    of one layer's weights with fresh seeded tokens until `seconds` elapse.
+    Returns (layers done, elapsed s)."""
+    import oracle
+    from moe_expert_gemv_b200 import synth
+    if m is None:
+        m = synth.moe_layer(seed, 0)
+    L = oracle.Layer(m, E, H, I)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        x16 = synth.activations(seed + 1000 + done, 1, H)
+        _, idx, wt = oracle.router(*m["router"], E, H, 8, x16, TOPK)
+        L.moe(x16, idx, wt)
+        done += 1
+        el = time.perf_counter() - t0
+        if (el >= seconds and done >= 3) or (max_layers and done >= max_layers):
+            return done, el
+
+
+# --------------------------------------------------------- MoE decode run --
+def build_decode(args, dev):
+    import concurrent.futures as cf
+    import torch
+    from moe_expert_gemv_b200 import qmoe, synth
+
+    def gen(l):
+        m = synth.moe_layer(args.seed, l)
+        G = qmoe.MoELayer.from_numpy(m, E, H, I, device=dev)
+        return G, (m if l == 0 else None)
+
+    with cf.ThreadPoolExecutor(8) as ex:
+        res = list(ex.map(gen, range(args.layers)))
+    layers = [r[0] for r in res]
+    m0 = res[0][1]
+    xs = np.stack([synth.activations(args.seed, 1, H, layer=l)[0] for l in range(args.layers)])
+    x = torch.from_numpy(xs.view(np.float16).copy()).to(dev)
+    idx = torch.zeros(args.layers, TOPK, dtype=torch.int32, device=dev)
+    wt = torch.zeros(args.layers, TOPK, dtype=torch.float32, device=dev)
+    y = torch.zeros(args.layers, H, dtype=torch.float16, device=dev)
+    ws = [qmoe.expert_workspace(layers[0], TOPK, dev) for _ in range(args.layers)]
+    torch.cuda.synchronize()
+    return layers, m0, x, idx, wt, y, ws
+
+
+def run_decode(args, dist):
+    import torch
+    from moe_expert_gemv_b200 import qmoe
+
+    dev = torch.device("cuda", dist.local if dist.world > 1 else 0)
+    torch.cuda.set_device(dev)
+    layers, m0, x, idx, wt, y, ws = build_decode(args, dev)
+    nl = args.layers
+
+    def step():
+        for l in range(nl):
+            qmoe.moe_router_topk(layers[l].router, x[l:l + 1], TOPK, idx[l:l + 1], wt[l:l + 1])
+            qmoe.moe_expert_qmlp(layers[l], x[l], idx[l], wt[l], y[l], ws[l])
+
+    def gateup_only():
+        for l in range(nl):
+            qmoe.moe_expert_gateup(layers[l], x[l], idx[l], ws[l])
+
+    def down_only():
+        for l in range(nl):
+            qmoe.moe_expert_down(layers[l], idx[l], wt[l], y[l], ws[l])
+
+    def router_only():
+        for l in range(nl):
+            qmoe.moe_router_topk(layers[l].router, x[l:l + 1], TOPK, idx[l:l + 1], wt[l:l + 1])
+
+    stream = torch.cuda.Stream()
+    graphs = {}
+    with torch.cuda.stream(stream):
+        step()   # eager warm-up (first-use set-up happens outside capture)
+        gateup_only()
+        down_only()
+        torch.cuda.synchronize()
+        assert qmoe.qmoe_check_status() == 0
+        for name, fn in (("step", step), ("gateup", gateup_only), ("down", down_only),
+                         ("router", router_only)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            graphs[name] = g
+        torch.cuda.synchronize()
+
+        for _ in range(args.warmup):
+            graphs["step"].replay()
+        torch.cuda.synchronize()
+        clocks = ClockSampler(dev.index) if dist.rank == 0 else None
+        if clocks:
+            clocks.start()
+        ms = timed_replays(graphs["step"].replay, args.steps, dist)
+        clk = clocks.stop() if clocks else None
+        ms = dist.max(ms)
+        flags = qmoe.qmoe_check_status()
+
+        # per-kernel averages (each graph chains the kernel over the 30 layers)
+        reps = max(20, args.steps // 10)
+        kern = {}
+        for name in ("gateup", "down", "router"):
+            for _ in range(3):
+                graphs[name].replay()
+            kern[name] = timed_replays(graphs[name].replay, reps) / (reps * nl)
+
+        # end to end through host buffers: H2D of every layer's input token,
+        # the step, D2H of every layer's output, each step
+        x_host = x.cpu().pin_memory()
+        y_host = torch.empty_like(y, device="cpu").pin_memory()
+
+        def e2e_step():
+            x.copy_(x_host, non_blocking=True)
+            graphs["step"].replay()
+            y_host.copy_(y, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        e2e_steps = max(10, args.steps // 4)
+        e2e_ms = dist.max(timed_replays(e2e_step, e2e_steps, dist))
+    graphs.clear()
+    return dict(ms=ms, kern=kern, clk=clk, flags=flags, e2e_ms=e2e_ms, e2e_steps=e2e_steps,
+                m0=m0, h2d=x.numel() * 2, d2h=y.numel() * 2)
+
+
+def main_decode(args):
+    dist = Dist()
+    r = run_decode(args, dist)
+    if dist.rank != 0:
+        dist.close()
+        return
+    hbm, _, peak_kind = peaks()
+    nl, K, N = args.layers, args.steps, dist.world
+    value = nl * K * N / (r["ms"] / 1e3)
+    gu_ms = r["kern"]["gateup"]
+    gu_gbs = GATEUP_BYTES / (gu_ms / 1e3) / 1e9
+    trf = NCU_TRAFFIC.get("expert_gateup_kernel")
+    traffic = trf["bytes"] if trf and trf["sha"] == source_sha("expert.cu") else None
+    line = {
+        "metric": "qGEMV/MoE-layer weight-stream GB/s vs HBM peak; MoE decode layers/s",
+        "value": round(value, 1),
+        "unit": "layers/s",
+        "n_gpus": N,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(r["ms"] / K, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16xf16->f32 (affine int4 weights)",
+        "data": "synthetic (seeded; value distributions of the pages' workloads)",
+        "config": {
+            "workload": "moe_decode: 1 token x %d MoE layers (router 8-bit 128x%d, top-%d of %d "
+                        "SwiGLU experts %dx%d 4-bit g64 + shared expert)" % (nl, H, TOPK, E, I, H),
+            "layers": nl, "experts": E, "hidden": H, "inter": I, "top_k": TOPK,
+            "bytes_per_layer": LAYER_BYTES,
+            "weight_stream_gbs": round(LAYER_BYTES * nl * K / (r["ms"] / 1e3) / 1e9, 1),
+            "l2": "inputs larger than L2: 12.96 GB of weights, each step streams 915 MB",
+            "graph": "CUDA graph of the 30-layer step, kernels chained by programmatic "
+                     "dependent launch",
+            "parallelism": "replicas" if N > 1 else "single GPU",
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": "expert_gateup_kernel",
+            "achieved": round(gu_gbs, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+            "frac": round(gu_gbs / hbm, 4), "traffic": traffic,
+            "algorithmic_bytes_per_launch": GATEUP_BYTES,
+            "launch_us": round(gu_ms * 1e3, 3),
+        },
+        "kernels_us": {k: round(v * 1e3, 3) for k, v in r["kern"].items()},
+        "kernels_gbs": {
+            "gateup": round(GATEUP_BYTES / (r["kern"]["gateup"] / 1e3) / 1e9, 1),
+            "down": round(DOWN_BYTES / (r["kern"]["down"] / 1e3) / 1e9, 1),
+            "router": round(ROUTER_CALL_BYTES / (r["kern"]["router"] / 1e3) / 1e9, 1),
+        },
+        "e2e": {"value": round(nl * r["e2e_steps"] * N / (r["e2e_ms"] / 1e3), 1),
+                "unit": "layers/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": 3 * nl * K,
+        "device_flags": r["flags"],
+    }
+    if r["clk"]:
+        line["clocks"] = r["clk"]
+    if N == 1 and not args.no_cpu_baseline:
+        done, el = oracle_decode_layers(args.cpu_seconds, args.seed, m=r["m0"])
+        line["cpu_baseline"] = {"value": round(done / el, 3), "unit": "layers/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": "%d decode layers (router + shared + 8 routed experts) "
+                                          "of layer 0's weights, fresh seeded tokens, %.1f s, "
+                                          "single thread" % (done, el)}
+    print(json.dumps(line), flush=True)
+    dist.close()
+
+
+# ----------------------------------------------------- reference (oracle) --
+def main_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    budget = 150.0
+    per_layer = 0.25
+    steps = max(3, min(args.steps, int(budget / per_layer)))
+    warm = min(args.warmup, 2)
+    from moe_expert_gemv_b200 import synth
+    m = synth.moe_layer(args.seed, 0)
+    oracle_decode_layers(0.0, args.seed, max_layers=max(1, warm), m=m)
+    done, el = oracle_decode_layers(1e9, args.seed, max_layers=steps, m=m)
+    value = done / el
+    line = {
+        "impl": "reference",
+        "metric": "qGEMV/MoE-layer weight-stream GB/s vs HBM peak; MoE decode layers/s",
+        "value": round(value, 3), "unit": "layers/s", "n_gpus": 1, "steps": done,
+        "warmup": warm, "ms_per_step": round(el / done * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "moe_decode (CPU oracle, one layer per step)", "layers": 1,
+                   "experts": E, "hidden": H, "inter": I, "top_k": TOPK},
+        "cpu_baseline": {"value": round(value, 3), "unit": "layers/s", "cores": 1,
+                         "kind": "oracle",
+                         "sample": "%d decode layers of layer 0's weights, single thread" % done},
+        "e2e": {"value": round(value, 3), "unit": "layers/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------- secondary workloads --
+def main_other(args):
+    """Single-kernel workloads used for the per-kernel roofline notes."""
+    import torch
+    from moe_expert_gemv_b200 import qmoe, synth
+    dev = torch.device("cuda", 0)
+    hbm, _, peak_kind = peaks()
+    out = {"workload": args.workload, "peak_gbs": hbm, "peak_kind": peak_kind, "results": []}
+    if args.workload == "qgemv":
+        for N in (14336, 4096):
+            K = 4096
+            copies = max(2, int(4 * 126e6 // (N * K * 9 // 16)) + 1)
+            Ws = []
+            for c in range(copies):
+                P, S, B = synth.dense(c, N, K)
+                Ws.append(qmoe.QMatrix.from_numpy(P, S, B, N, K, 4, dev))
+            nbytes = N * K // 2 + 2 * N * (K // 64) * 2
+            for Bt in (1, 4, 8):
+                x = torch.from_numpy(synth.activations(Bt, Bt, K).view(np.float16).copy()).to(dev)
+                y = torch.empty(Bt, N, dtype=torch.float16, device=dev)
+
+                def run():
+                    for W in Ws:
+                        qmoe.qgemv_affine(W, x, y)
+                run()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    run()
+                for _ in range(3):
+                    g.replay()
+                reps = max(10, args.steps // 10)
+                ms = timed_replays(g.replay, reps) / (reps * copies)
+                gbs = (nbytes + Bt * K * 2 + Bt * N * 2) / (ms / 1e3) / 1e9
+                out["results"].append({"N": N, "K": K, "B": Bt, "us": round(ms * 1e3, 3),
+                                       "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
+                                       "rotated_copies": copies})
+    elif args.workload == "router":
+        P, S, B = synth.router(args.seed)
+        R = qmoe.QMatrix.from_numpy(P, S, B, E, H, 8, dev)
+        for T in (1, 2, 4, 8, 16, 32, 64, 128):
+            x = torch.from_numpy(synth.activations(T, T, H).view(np.float16).copy()).to(dev)
+            idx = torch.empty(T, TOPK, dtype=torch.int32, device=dev)
+            wt = torch.empty(T, TOPK, dtype=torch.float32, device=dev)
+
+            def run():
+                qmoe.moe_router_topk(R, x, TOPK, idx, wt)
+            run()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for _ in range(20):
+                    run()
+            g.replay()
+            reps = 50
+            ms = timed_replays(g.replay, reps) / (reps * 20)
+            out["results"].append({"T": T, "us": round(ms * 1e3, 3),
+                                   "tokens_per_s": round(T / (ms / 1e3), 1)})
+    else:
+        out["error"] = "workload not available"
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        main_reference(args)
+    elif args.workload == "moe_decode":
+        main_decode(args)
+    else:
+        main_other(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,229 @@
+/*
+ * qmoe.h -- C ABI of libqmoe.so: affine-quantized GEMV and Mixture-of-Experts
+ * decode / prefill kernels for NVIDIA B200 (sm_100a).
+ *
+ * What is computed, and where the pages say so:
+ *   - Weights are "MLX affine 4-bit, group 64"; the router is 8-bit; the
+ *     routed and shared experts are 4-bit (TurboFieldfare article, jeff.news,
+ *     section "성능과 제약" -- performance and constraints).
+ *     Reading of the format: element (n, k) of a row-major [rows][cols] matrix
+ *     is  w = scale[n][k/64] * q + bias[n][k/64]  with q the unsigned code in
+ *     bits [bits*(k%p), bits*(k%p)+bits) of word k/p of row n, p = 32/bits
+ *     (least-significant field first); scale and bias are fp16.
+ *   - Each layer's router runs on resident weights, picks the top-8 experts,
+ *     and the routed experts' output is added to a resident shared expert's
+ *     output; prefill runs in chunks of at most 128 tokens so one fetched
+ *     expert serves many rows (same article, section "내부 구조가 진짜 흥미로운
+ *     부분" -- internal structure).  Router weights are fp32-softmaxed and the
+ *     top_k largest logits are kept (ties: lower expert index first), listed
+ *     in descending order, renormalised to sum to one.  Experts are SwiGLU:
+ *     r = down( silu(gate x) * (up x) ),  silu(z) = z / (1 + e^-z).
+ *   - Quantized GEMV is one of the operations such a runtime hand-controls
+ *     (same article, section "기술 맥락" -- technical context).
+ *
+ * Conventions for every entry point:
+ *   - fp16 tensors are passed as uint16_t bit patterns; all tensor pointers
+ *     are DEVICE pointers owned by the caller, row-major and densely packed.
+ *     The three arrays of a qmoe_qmatrix must be 16-byte aligned; other
+ *     fp16/fp32/int32 arrays naturally aligned (2/4/4 bytes).  Violations
+ *     return QMOE_ERR_ALIGNMENT.
+ *   - Weight operands (qmoe_qmatrix, qmoe_moe_layer) are read-only model
+ *     parameters.  Kernels start streaming them before the previous kernel on
+ *     the stream has finished (programmatic dependent launch), so a weight
+ *     buffer must not be written by the kernel enqueued immediately before a
+ *     call on the same stream: synchronise after writing weights, or turn the
+ *     overlap off with qmoe_set_dependent_launch(0).  Activations, routing
+ *     inputs and outputs are ordered as usual.
+ *   - `stream` is a cudaStream_t (NULL: the legacy default stream).  Calls are
+ *     asynchronous: they validate on the host, enqueue kernels and return.
+ *     The library never allocates, frees or synchronises inside a compute
+ *     call.  The current CUDA device must be the one that owns the pointers.
+ *   - `status_dev` (optional, may be NULL) is a device int32 word that kernels
+ *     OR device-detected problems into (QMOE_DEV_* flags).  With NULL the
+ *     library's own per-device word is used.  qmoe_check_status() reads and
+ *     clears it.  Kernels never trap: a bad expert id is skipped (its
+ *     contribution is zero) and flagged; a pipeline wait that exceeds its
+ *     time limit abandons the work and flags QMOE_DEV_TIMEOUT.
+ *   - Host-side validation happens before any launch; on error nothing is
+ *     enqueued.  A CUDA launch failure returns QMOE_ERR_CUDA.
+ */
+#ifndef QMOE_H
+#define QMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qmoe_status {
+    QMOE_OK = 0,
+    QMOE_ERR_INVALID_ARG = -1,   /* NULL pointer, size out of range, shape mismatch */
+    QMOE_ERR_ALIGNMENT = -2,     /* pointer not aligned as stated above */
+    QMOE_ERR_UNSUPPORTED = -3,   /* valid request outside what the kernels implement */
+    QMOE_ERR_CUDA = -4,          /* a CUDA runtime call failed */
+    QMOE_ERR_DEVICE_STATUS = -5, /* qmoe_check_status: a kernel flagged bad input */
+    QMOE_ERR_TIMEOUT = -6,       /* qmoe_check_status: a kernel wait timed out */
+    QMOE_ERR_WORKSPACE = -7      /* workspace missing or smaller than required */
+} qmoe_status;
+
+/* flags OR-ed into the device status word */
+#define QMOE_DEV_BAD_EXPERT 0x1  /* an expert id outside [0, num_experts) was skipped */
+#define QMOE_DEV_TIMEOUT 0x2     /* a pipeline wait gave up; outputs are invalid */
+
+/* One affine-quantized matrix (or a stack of equally-shaped matrices).
+ *   packed: uint32 [rows][cols*bits/32]   (16-byte aligned)
+ *   scales: fp16   [rows][cols/group]
+ *   biases: fp16   [rows][cols/group]
+ * bits is 4 or 8, group must be 64, cols a multiple of 64, rows a multiple
+ * of 8.  For a stack (the routed experts) the matrices follow each other
+ * with no gap: matrix e starts at packed + e*rows*cols*bits/32 and at
+ * scales/biases + e*rows*cols/64. */
+typedef struct qmoe_qmatrix {
+    const uint32_t *packed;
+    const uint16_t *scales;
+    const uint16_t *biases;
+    int32_t rows;
+    int32_t cols;
+    int32_t bits;
+    int32_t group;
+} qmoe_qmatrix;
+
+/* One MoE layer: num_experts routed SwiGLU experts stacked in gate/up/down
+ * (gate, up: rows = inter, cols = hidden; down: rows = hidden, cols = inter;
+ * 4-bit), plus the always-resident shared expert of the same shapes.
+ * The router is a separate qmoe_qmatrix (rows = num_experts, cols = hidden,
+ * 8-bit) handed to moe_router_topk. */
+typedef struct qmoe_moe_layer {
+    qmoe_qmatrix gate, up, down;          /* routed experts, stacked */
+    qmoe_qmatrix sh_gate, sh_up, sh_down; /* shared expert */
+    int32_t num_experts;
+    int32_t hidden;
+    int32_t inter;
+} qmoe_moe_layer;
+
+/* ---------------------------------------------------------------------------
+ * Dense affine qGEMV, batch 1..8 (decode projection; quantized GEMV of the
+ * "기술 맥락" section, format of the "성능과 제약" section).
+ *   y[b][n] = sum_k w[n][k] * x[b][k]     fp32 accumulate, fp16 output
+ *   W: bits 4 or 8; x: fp16 [batch][W->cols]; y: fp16 [batch][W->rows].
+ * Errors: INVALID_ARG (NULL, batch outside 1..8, shape), ALIGNMENT,
+ * UNSUPPORTED (group != 64, cols % 64, rows % 8), CUDA.
+ * ------------------------------------------------------------------------- */
+qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch,
+                         uint16_t *y, int32_t *status_dev, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Router + softmax + top-k + renormalisation ("내부 구조" section: the router
+ * runs on resident weights and picks the top-8 experts).
+ *   logits[t][e] = sum_k w_router[e][k] x[t][k]    (fp32)
+ *   idx[t][0..top_k): the top_k largest logits, descending, ties -> lower e
+ *   weights[t][j] = softmax(logits[t])[idx[t][j]] / sum_j' softmax(...)[idx[t][j']]
+ * router: rows = num_experts (a multiple of 8, at most 128), bits 4 or 8.
+ * x: fp16 [tokens][router->cols], tokens 1..65536; top_k 1..min(16, rows).
+ * idx: int32 [tokens][top_k]; weights: fp32 [tokens][top_k];
+ * logits: fp32 [tokens][rows] or NULL.
+ * Selection uses exactly the fp32 logits written to `logits`.
+ * ------------------------------------------------------------------------- */
+qmoe_status moe_router_topk(const qmoe_qmatrix *router, const uint16_t *x, int32_t tokens,
+                            int32_t top_k, int32_t *idx, float *weights, float *logits,
+                            int32_t *status_dev, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Decode MoE layer for one token ("내부 구조" section: routed experts computed
+ * from the router's top-8 ids, added to the shared expert's output):
+ *   y = shared(x) + sum_j weights[j] * expert_{idx[j]}(x)
+ *   expert(x) = down( silu(gate x) * (up x) ), all intermediates fp32.
+ * x: fp16 [hidden]; idx: int32 [top_k] (device memory, e.g. written by
+ * moe_router_topk); weights: fp32 [top_k]; y: fp16 [hidden]; top_k 1..16.
+ * Shapes: hidden and inter multiples of 64; hidden a multiple of 16.
+ * workspace: device memory of moe_expert_workspace_bytes() bytes, 16-byte
+ * aligned, ZERO-FILLED before its first use (e.g. cudaMemsetAsync).  Every
+ * successful call leaves it zero-filled again, so it can be reused by later
+ * calls on the same stream (also inside CUDA graphs); calls that overlap in
+ * time need separate workspaces.  After a QMOE_DEV_TIMEOUT re-zero it.
+ * An idx entry outside [0, num_experts) contributes zero and raises
+ * QMOE_DEV_BAD_EXPERT.
+ * moe_expert_qmlp == moe_expert_gateup followed by moe_expert_down on the
+ * same workspace; the two halves are exported for measurement.
+ * ------------------------------------------------------------------------- */
+size_t moe_expert_workspace_bytes(const qmoe_moe_layer *L, int32_t top_k);
+
+qmoe_status moe_expert_qmlp(const qmoe_moe_layer *L, const uint16_t *x, const int32_t *idx,
+                            const float *weights, int32_t top_k, uint16_t *y, void *workspace,
+                            size_t workspace_bytes, int32_t *status_dev, void *stream);
+
+/* h_j = silu(gate_e x) * (up_e x) for the top_k routed experts e = idx[j] and
+ * the shared expert (slot top_k), fp32, kept in the workspace. */
+qmoe_status moe_expert_gateup(const qmoe_moe_layer *L, const uint16_t *x, const int32_t *idx,
+                              int32_t top_k, void *workspace, size_t workspace_bytes,
+                              int32_t *status_dev, void *stream);
+
+/* y = down_shared h_shared + sum_j weights[j] * down_{idx[j]} h_j, fp16, from
+ * the h left in the workspace by moe_expert_gateup. */
+qmoe_status moe_expert_down(const qmoe_moe_layer *L, const int32_t *idx, const float *weights,
+                            int32_t top_k, uint16_t *y, void *workspace, size_t workspace_bytes,
+                            int32_t *status_dev, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Prefill grouping ("내부 구조" section: a chunk's tokens are gathered per
+ * expert so one fetched expert serves many rows).
+ *   counts[e]  = number of (token, slot) pairs with idx == e
+ *   offsets[0..num_experts] = exclusive prefix sum of counts
+ *   pairs[offsets[e] .. offsets[e+1]) = flat indices t*top_k + j with
+ *                                       idx[t][j] == e, ascending
+ * idx: int32 [tokens][top_k], tokens 1..128, top_k 1..16, num_experts 1..256.
+ * An id outside [0, num_experts) raises QMOE_DEV_BAD_EXPERT and is dropped.
+ * ------------------------------------------------------------------------- */
+qmoe_status moe_group_tokens(const int32_t *idx, int32_t tokens, int32_t top_k,
+                             int32_t num_experts, int32_t *counts, int32_t *offsets,
+                             int32_t *pairs, int32_t *status_dev, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Prefill chunk through the MoE layer as a grouped qGEMM (same formula as
+ * moe_expert_qmlp, row by row):
+ *   y[t] = shared(x[t]) + sum_j weights[t][j] * expert_{idx[t][j]}(x[t])
+ * x: fp16 [tokens][hidden], tokens 1..128; idx: int32 [tokens][top_k];
+ * weights: fp32 [tokens][top_k]; y: fp16 [tokens][hidden].
+ * workspace: moe_prefill_workspace_bytes() bytes, 16-byte aligned; no
+ * initial contents are required.
+ * ------------------------------------------------------------------------- */
+size_t moe_prefill_workspace_bytes(const qmoe_moe_layer *L, int32_t tokens, int32_t top_k);
+
+qmoe_status moe_prefill_qgemm(const qmoe_moe_layer *L, const uint16_t *x, int32_t tokens,
+                              const int32_t *idx, const float *weights, int32_t top_k,
+                              uint16_t *y, void *workspace, size_t workspace_bytes,
+                              int32_t *status_dev, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Format helpers (the packing reading of the "성능과 제약" section).
+ * codes: uint8 [rows][cols] (values >= 2^bits are masked); packed: uint32
+ * [rows][cols*bits/32].  cols must be a multiple of 32/bits.
+ * ------------------------------------------------------------------------- */
+qmoe_status qmoe_pack_codes(const uint8_t *codes, int32_t rows, int32_t cols, int32_t bits,
+                            uint32_t *packed, void *stream);
+qmoe_status qmoe_unpack_codes(const uint32_t *packed, int32_t rows, int32_t cols, int32_t bits,
+                              uint8_t *codes, void *stream);
+
+/* Synchronises `stream`, reads and clears the status word (NULL: the
+ * library's word on the current device).  Returns QMOE_OK, QMOE_ERR_TIMEOUT
+ * (if QMOE_DEV_TIMEOUT was set), QMOE_ERR_DEVICE_STATUS (other flags) or
+ * QMOE_ERR_CUDA.  If flags_out is not NULL it receives the raw flags. */
+qmoe_status qmoe_check_status(int32_t *status_dev, void *stream, int32_t *flags_out);
+
+/* Static, human-readable name of a status code. */
+const char *qmoe_status_string(qmoe_status s);
+
+/* Enable (1, the default) or disable (0) programmatic dependent launch for
+ * all later calls in this process.  Returns the previous setting. */
+int32_t qmoe_set_dependent_launch(int32_t enable);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t qmoe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QMOE_H */

@@ -1,0 +1,473 @@
+// api.cu -- the C ABI of libqmoe.so (declared in include/qmoe.h): host-side
+// validation, per-device state, workspace layout and kernel launches.
+//
+// The operations and where the pages define them are listed in qmoe.h.  This
+// layer allocates nothing and never synchronises inside a compute call; the
+// one per-device object it owns is a status word in a __device__ variable.
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qmoe {
+
+__device__ int32_t g_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DevState {
+    bool init = false;
+    int num_sms = 0;
+    int cc_major = 0;
+    int32_t *status = nullptr;
+};
+
+DevState g_dev[kMaxDevices];
+std::mutex g_mu;
+std::atomic<int32_t> g_pdl_enabled{1};
+
+qmoe_status device_state(DevState **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return QMOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DevState &d = g_dev[dev];
+    if (!d.init) {
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return QMOE_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) !=
+            cudaSuccess)
+            return QMOE_ERR_CUDA;
+        if (cudaGetSymbolAddress(reinterpret_cast<void **>(&d.status), g_status_word) !=
+            cudaSuccess)
+            return QMOE_ERR_CUDA;
+        d.init = true;
+    }
+    if (d.cc_major != 10)
+        return QMOE_ERR_UNSUPPORTED;   // built for sm_100a only
+    *out = &d;
+    return QMOE_OK;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Validate one (possibly stacked) quantized matrix of `rows` x `cols`.
+qmoe_status check_qmatrix(const qmoe_qmatrix *W, int rows, int cols, int bits_required)
+{
+    if (!W || !W->packed || !W->scales || !W->biases)
+        return QMOE_ERR_INVALID_ARG;
+    if (W->rows != rows || W->cols != cols || rows <= 0 || cols <= 0)
+        return QMOE_ERR_INVALID_ARG;
+    if (W->bits != 4 && W->bits != 8)
+        return QMOE_ERR_INVALID_ARG;
+    if (bits_required && W->bits != bits_required)
+        return QMOE_ERR_UNSUPPORTED;
+    if (W->group != kGroup || cols % kGroup != 0 || rows % 8 != 0)
+        return QMOE_ERR_UNSUPPORTED;
+    if (!aligned(W->packed, 16) || !aligned(W->scales, 16) || !aligned(W->biases, 16))
+        return QMOE_ERR_ALIGNMENT;
+    return QMOE_OK;
+}
+
+qmoe_status cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess)
+        return QMOE_OK;
+    if (e == cudaErrorInvalidValue)
+        return QMOE_ERR_UNSUPPORTED;   // a shape whose tiles do not fit on chip
+    return QMOE_ERR_CUDA;
+}
+
+QMat qmat(const qmoe_qmatrix &m)
+{
+    QMat q;
+    q.packed = m.packed;
+    q.scales = reinterpret_cast<const __half *>(m.scales);
+    q.biases = reinterpret_cast<const __half *>(m.biases);
+    return q;
+}
+
+qmoe_status check_layer(const qmoe_moe_layer *L)
+{
+    if (!L)
+        return QMOE_ERR_INVALID_ARG;
+    const int E = L->num_experts, H = L->hidden, I = L->inter;
+    if (E < 1 || E > 256 || H < 64 || I < 64)
+        return QMOE_ERR_INVALID_ARG;
+    if (H % 64 || I % 64)
+        return QMOE_ERR_UNSUPPORTED;
+    qmoe_status s;
+    if ((s = check_qmatrix(&L->gate, I, H, 4)) != QMOE_OK ||
+        (s = check_qmatrix(&L->up, I, H, 4)) != QMOE_OK ||
+        (s = check_qmatrix(&L->down, H, I, 4)) != QMOE_OK ||
+        (s = check_qmatrix(&L->sh_gate, I, H, 4)) != QMOE_OK ||
+        (s = check_qmatrix(&L->sh_up, I, H, 4)) != QMOE_OK ||
+        (s = check_qmatrix(&L->sh_down, H, I, 4)) != QMOE_OK)
+        return s;
+    return QMOE_OK;
+}
+
+LaunchCfg launch_cfg(const DevState *d, void *stream)
+{
+    LaunchCfg c;
+    c.stream = static_cast<cudaStream_t>(stream);
+    c.num_sms = d->num_sms;
+    c.pdl = g_pdl_enabled.load() != 0;
+    return c;
+}
+
+qmoe_status expert_args(const qmoe_moe_layer *L, const uint16_t *x, const int32_t *idx,
+                        const float *weights, int32_t top_k, uint16_t *y, void *workspace,
+                        size_t ws_bytes, int32_t *status, ExpertArgs *a)
+{
+    a->gate = qmat(L->gate);
+    a->up = qmat(L->up);
+    a->down = qmat(L->down);
+    a->sh_gate = qmat(L->sh_gate);
+    a->sh_up = qmat(L->sh_up);
+    a->sh_down = qmat(L->sh_down);
+    a->E = L->num_experts;
+    a->H = L->hidden;
+    a->I = L->inter;
+    a->top_k = top_k;
+    a->x = reinterpret_cast<const __half *>(x);
+    a->idx = idx;
+    a->weights = weights;
+    a->y = reinterpret_cast<__half *>(y);
+    a->status = status;
+    if (!workspace)
+        return QMOE_ERR_WORKSPACE;
+    if (!aligned(workspace, 16))
+        return QMOE_ERR_ALIGNMENT;
+    if (ws_bytes < expert_workspace_layout(a->H, a->I, top_k, nullptr, nullptr))
+        return QMOE_ERR_WORKSPACE;
+    expert_workspace_layout(a->H, a->I, top_k, workspace, &a->ws);
+    return QMOE_OK;
+}
+
+qmoe_status check_expert_common(const qmoe_moe_layer *L, int32_t top_k)
+{
+    qmoe_status s = check_layer(L);
+    if (s != QMOE_OK)
+        return s;
+    if (top_k < 1 || top_k > 16 || top_k > L->num_experts)
+        return QMOE_ERR_INVALID_ARG;
+    if (L->hidden % 16)
+        return QMOE_ERR_UNSUPPORTED;
+    return QMOE_OK;
+}
+
+}  // namespace
+}  // namespace qmoe
+
+using namespace qmoe;
+
+extern "C" {
+
+qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch, uint16_t *y,
+                         int32_t *status_dev, void *stream)
+{
+    if (!W || !x || !y)
+        return QMOE_ERR_INVALID_ARG;
+    if (batch < 1 || batch > 8)
+        return QMOE_ERR_INVALID_ARG;
+    qmoe_status s = check_qmatrix(W, W->rows, W->cols, 0);
+    if (s != QMOE_OK)
+        return s;
+    if (!aligned(x, 2) || !aligned(y, 2) || (status_dev && !aligned(status_dev, 4)))
+        return QMOE_ERR_ALIGNMENT;
+    DevState *d;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    QgemvArgs a;
+    a.packed = W->packed;
+    a.scales = reinterpret_cast<const __half *>(W->scales);
+    a.biases = reinterpret_cast<const __half *>(W->biases);
+    a.N = W->rows;
+    a.K = W->cols;
+    a.bits = W->bits;
+    a.x = reinterpret_cast<const __half *>(x);
+    a.B = batch;
+    a.y = reinterpret_cast<__half *>(y);
+    a.status = status_dev ? status_dev : d->status;
+    return cuda_status(launch_qgemv(a, launch_cfg(d, stream)));
+}
+
+qmoe_status moe_router_topk(const qmoe_qmatrix *router, const uint16_t *x, int32_t tokens,
+                            int32_t top_k, int32_t *idx, float *weights, float *logits,
+                            int32_t *status_dev, void *stream)
+{
+    if (!router || !x || !idx || !weights)
+        return QMOE_ERR_INVALID_ARG;
+    if (tokens < 1 || tokens > 65536)
+        return QMOE_ERR_INVALID_ARG;
+    qmoe_status s = check_qmatrix(router, router->rows, router->cols, 0);
+    if (s != QMOE_OK)
+        return s;
+    if (router->rows > 128)
+        return QMOE_ERR_UNSUPPORTED;
+    if (top_k < 1 || top_k > 16 || top_k > router->rows)
+        return QMOE_ERR_INVALID_ARG;
+    if (!aligned(x, 2) || !aligned(idx, 4) || !aligned(weights, 4) ||
+        (logits && !aligned(logits, 4)) || (status_dev && !aligned(status_dev, 4)))
+        return QMOE_ERR_ALIGNMENT;
+    DevState *d;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    RouterArgs a;
+    a.packed = router->packed;
+    a.scales = reinterpret_cast<const __half *>(router->scales);
+    a.biases = reinterpret_cast<const __half *>(router->biases);
+    a.E = router->rows;
+    a.K = router->cols;
+    a.bits = router->bits;
+    a.x = reinterpret_cast<const __half *>(x);
+    a.T = tokens;
+    a.top_k = top_k;
+    a.idx = idx;
+    a.weights = weights;
+    a.logits = logits;
+    a.status = status_dev ? status_dev : d->status;
+    return cuda_status(launch_router(a, launch_cfg(d, stream)));
+}
+
+size_t moe_expert_workspace_bytes(const qmoe_moe_layer *L, int32_t top_k)
+{
+    if (!L || L->hidden <= 0 || L->inter <= 0 || top_k < 1)
+        return 0;
+    return expert_workspace_layout(L->hidden, L->inter, top_k, nullptr, nullptr);
+}
+
+qmoe_status moe_expert_gateup(const qmoe_moe_layer *L, const uint16_t *x, const int32_t *idx,
+                              int32_t top_k, void *workspace, size_t workspace_bytes,
+                              int32_t *status_dev, void *stream)
+{
+    qmoe_status s = check_expert_common(L, top_k);
+    if (s != QMOE_OK)
+        return s;
+    if (!x || !idx)
+        return QMOE_ERR_INVALID_ARG;
+    if (!aligned(x, 2) || !aligned(idx, 4) || (status_dev && !aligned(status_dev, 4)))
+        return QMOE_ERR_ALIGNMENT;
+    DevState *d;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    ExpertArgs a;
+    if ((s = expert_args(L, x, idx, nullptr, top_k, nullptr, workspace, workspace_bytes,
+                         status_dev ? status_dev : d->status, &a)) != QMOE_OK)
+        return s;
+    return cuda_status(launch_expert_gateup(a, launch_cfg(d, stream)));
+}
+
+qmoe_status moe_expert_down(const qmoe_moe_layer *L, const int32_t *idx, const float *weights,
+                            int32_t top_k, uint16_t *y, void *workspace, size_t workspace_bytes,
+                            int32_t *status_dev, void *stream)
+{
+    qmoe_status s = check_expert_common(L, top_k);
+    if (s != QMOE_OK)
+        return s;
+    if (!idx || !weights || !y)
+        return QMOE_ERR_INVALID_ARG;
+    if (!aligned(idx, 4) || !aligned(weights, 4) || !aligned(y, 2) ||
+        (status_dev && !aligned(status_dev, 4)))
+        return QMOE_ERR_ALIGNMENT;
+    DevState *d;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    ExpertArgs a;
+    if ((s = expert_args(L, nullptr, idx, weights, top_k, y, workspace, workspace_bytes,
+                         status_dev ? status_dev : d->status, &a)) != QMOE_OK)
+        return s;
+    return cuda_status(launch_expert_down(a, launch_cfg(d, stream)));
+}
+
+qmoe_status moe_expert_qmlp(const qmoe_moe_layer *L, const uint16_t *x, const int32_t *idx,
+                            const float *weights, int32_t top_k, uint16_t *y, void *workspace,
+                            size_t workspace_bytes, int32_t *status_dev, void *stream)
+{
+    qmoe_status s = check_expert_common(L, top_k);
+    if (s != QMOE_OK)
+        return s;
+    if (!x || !idx || !weights || !y)
+        return QMOE_ERR_INVALID_ARG;
+    if (!aligned(x, 2) || !aligned(idx, 4) || !aligned(weights, 4) || !aligned(y, 2) ||
+        (status_dev && !aligned(status_dev, 4)))
+        return QMOE_ERR_ALIGNMENT;
+    DevState *d;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    ExpertArgs a;
+    if ((s = expert_args(L, x, idx, weights, top_k, y, workspace, workspace_bytes,
+                         status_dev ? status_dev : d->status, &a)) != QMOE_OK)
+        return s;
+    const LaunchCfg c = launch_cfg(d, stream);
+    if ((s = cuda_status(launch_expert_gateup(a, c))) != QMOE_OK)
+        return s;
+    return cuda_status(launch_expert_down(a, c));
+}
+
+qmoe_status moe_group_tokens(const int32_t *idx, int32_t tokens, int32_t top_k,
+                             int32_t num_experts, int32_t *counts, int32_t *offsets,
+                             int32_t *pairs, int32_t *status_dev, void *stream)
+{
+    if (!idx || !counts || !offsets || !pairs)
+        return QMOE_ERR_INVALID_ARG;
+    if (tokens < 1 || tokens > 128 || top_k < 1 || top_k > 16 || num_experts < 1 ||
+        num_experts > 256)
+        return QMOE_ERR_INVALID_ARG;
+    if (!aligned(idx, 4) || !aligned(counts, 4) || !aligned(offsets, 4) || !aligned(pairs, 4) ||
+        (status_dev && !aligned(status_dev, 4)))
+        return QMOE_ERR_ALIGNMENT;
+    DevState *d;
+    qmoe_status s;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    GroupArgs a;
+    a.idx = idx;
+    a.T = tokens;
+    a.top_k = top_k;
+    a.E = num_experts;
+    a.counts = counts;
+    a.offsets = offsets;
+    a.pairs = pairs;
+    a.status = status_dev ? status_dev : d->status;
+    return cuda_status(launch_group(a, launch_cfg(d, stream)));
+}
+
+size_t moe_prefill_workspace_bytes(const qmoe_moe_layer *L, int32_t tokens, int32_t top_k)
+{
+    if (!L || tokens < 1 || top_k < 1 || L->num_experts < 1)
+        return 0;
+    return prefill_workspace_layout(L->num_experts, L->hidden, L->inter, tokens, top_k, nullptr,
+                                    nullptr);
+}
+
+qmoe_status moe_prefill_qgemm(const qmoe_moe_layer *L, const uint16_t *x, int32_t tokens,
+                              const int32_t *idx, const float *weights, int32_t top_k,
+                              uint16_t *y, void *workspace, size_t workspace_bytes,
+                              int32_t *status_dev, void *stream)
+{
+    qmoe_status s = check_expert_common(L, top_k);
+    if (s != QMOE_OK)
+        return s;
+    if (!x || !idx || !weights || !y)
+        return QMOE_ERR_INVALID_ARG;
+    if (tokens < 1 || tokens > 128)
+        return QMOE_ERR_INVALID_ARG;
+    if (!aligned(x, 2) || !aligned(idx, 4) || !aligned(weights, 4) || !aligned(y, 2) ||
+        (status_dev && !aligned(status_dev, 4)))
+        return QMOE_ERR_ALIGNMENT;
+    if (!workspace)
+        return QMOE_ERR_WORKSPACE;
+    if (!aligned(workspace, 16))
+        return QMOE_ERR_ALIGNMENT;
+    if (workspace_bytes < moe_prefill_workspace_bytes(L, tokens, top_k))
+        return QMOE_ERR_WORKSPACE;
+    DevState *d;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    PrefillArgs a;
+    a.gate = qmat(L->gate);
+    a.up = qmat(L->up);
+    a.down = qmat(L->down);
+    a.sh_gate = qmat(L->sh_gate);
+    a.sh_up = qmat(L->sh_up);
+    a.sh_down = qmat(L->sh_down);
+    a.E = L->num_experts;
+    a.H = L->hidden;
+    a.I = L->inter;
+    a.T = tokens;
+    a.top_k = top_k;
+    a.x = reinterpret_cast<const __half *>(x);
+    a.idx = idx;
+    a.weights = weights;
+    a.y = reinterpret_cast<__half *>(y);
+    a.status = status_dev ? status_dev : d->status;
+    prefill_workspace_layout(a.E, a.H, a.I, tokens, top_k, workspace, &a.ws);
+    return cuda_status(launch_prefill(a, launch_cfg(d, stream)));
+}
+
+qmoe_status qmoe_pack_codes(const uint8_t *codes, int32_t rows, int32_t cols, int32_t bits,
+                            uint32_t *packed, void *stream)
+{
+    if (!codes || !packed || rows < 1 || cols < 1 || (bits != 4 && bits != 8))
+        return QMOE_ERR_INVALID_ARG;
+    if (cols % (32 / bits))
+        return QMOE_ERR_INVALID_ARG;
+    if (!aligned(packed, 4))
+        return QMOE_ERR_ALIGNMENT;
+    DevState *d;
+    qmoe_status s;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    return cuda_status(launch_pack(codes, rows, cols, bits, packed, static_cast<cudaStream_t>(stream)));
+}
+
+qmoe_status qmoe_unpack_codes(const uint32_t *packed, int32_t rows, int32_t cols, int32_t bits,
+                              uint8_t *codes, void *stream)
+{
+    if (!codes || !packed || rows < 1 || cols < 1 || (bits != 4 && bits != 8))
+        return QMOE_ERR_INVALID_ARG;
+    if (cols % (32 / bits))
+        return QMOE_ERR_INVALID_ARG;
+    if (!aligned(packed, 4))
+        return QMOE_ERR_ALIGNMENT;
+    DevState *d;
+    qmoe_status s;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    return cuda_status(
+        launch_unpack(packed, rows, cols, bits, codes, static_cast<cudaStream_t>(stream)));
+}
+
+qmoe_status qmoe_check_status(int32_t *status_dev, void *stream, int32_t *flags_out)
+{
+    DevState *d;
+    qmoe_status s;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t *word = status_dev ? status_dev : d->status;
+    int32_t flags = 0;
+    if (cudaMemcpyAsync(&flags, word, sizeof(flags), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return QMOE_ERR_CUDA;
+    if (cudaMemsetAsync(word, 0, sizeof(int32_t), st) != cudaSuccess)
+        return QMOE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess)
+        return QMOE_ERR_CUDA;
+    if (flags_out)
+        *flags_out = flags;
+    if (flags & QMOE_DEV_TIMEOUT)
+        return QMOE_ERR_TIMEOUT;
+    if (flags)
+        return QMOE_ERR_DEVICE_STATUS;
+    return QMOE_OK;
+}
+
+const char *qmoe_status_string(qmoe_status s)
+{
+    switch (s) {
+    case QMOE_OK: return "QMOE_OK";
+    case QMOE_ERR_INVALID_ARG: return "QMOE_ERR_INVALID_ARG: invalid argument";
+    case QMOE_ERR_ALIGNMENT: return "QMOE_ERR_ALIGNMENT: misaligned pointer";
+    case QMOE_ERR_UNSUPPORTED: return "QMOE_ERR_UNSUPPORTED: unsupported shape or device";
+    case QMOE_ERR_CUDA: return "QMOE_ERR_CUDA: CUDA runtime error";
+    case QMOE_ERR_DEVICE_STATUS: return "QMOE_ERR_DEVICE_STATUS: a kernel flagged bad input";
+    case QMOE_ERR_TIMEOUT: return "QMOE_ERR_TIMEOUT: a kernel wait timed out";
+    case QMOE_ERR_WORKSPACE: return "QMOE_ERR_WORKSPACE: workspace missing or too small";
+    }
+    return "unknown qmoe_status";
+}
+
+int32_t qmoe_set_dependent_launch(int32_t enable)
+{
+    return g_pdl_enabled.exchange(enable ? 1 : 0);
+}
+
+int32_t qmoe_version(void) { return 100; }
+
+}  // extern "C"

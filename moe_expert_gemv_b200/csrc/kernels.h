@@ -1,0 +1,147 @@
+// kernels.h -- internal launch interface between the C-ABI layer (api.cu) and
+// the kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qmoe.h"
+
+namespace qmoe {
+
+struct LaunchCfg {
+    cudaStream_t stream;
+    int num_sms;
+    bool pdl;   // launch as a programmatic dependent of the previous kernel
+};
+
+// ------------------------------------------------------------ dense qGEMV --
+struct QgemvArgs {
+    const uint32_t *packed;
+    const __half *scales, *biases;
+    int N, K, bits;
+    const __half *x;   // [B][K]
+    int B;
+    __half *y;         // [B][N]
+    int32_t *status;
+};
+cudaError_t launch_qgemv(const QgemvArgs &a, const LaunchCfg &c);
+
+// ------------------------------------------------------------------ router --
+struct RouterArgs {
+    const uint32_t *packed;
+    const __half *scales, *biases;
+    int E, K, bits;
+    const __half *x;   // [T][K]
+    int T, top_k;
+    int32_t *idx;      // [T][top_k]
+    float *weights;    // [T][top_k]
+    float *logits;     // [T][E] or null
+    int32_t *status;
+};
+cudaError_t launch_router(const RouterArgs &a, const LaunchCfg &c);
+
+// ------------------------------------------------------- decode experts --
+struct QMat {
+    const uint32_t *packed;
+    const __half *scales, *biases;
+};
+
+struct ExpertWorkspace {
+    float *h;          // [top_k + 1][inter]   (slot top_k: shared expert)
+    float *part;       // [top_k + 1][hidden]
+    int32_t *counters; // [hidden / 16]
+};
+size_t expert_workspace_layout(int hidden, int inter, int top_k, void *base, ExpertWorkspace *ws);
+
+struct ExpertArgs {
+    QMat gate, up, down, sh_gate, sh_up, sh_down;
+    int E, H, I, top_k;
+    const __half *x;        // [H]
+    const int32_t *idx;     // [top_k]
+    const float *weights;   // [top_k]
+    __half *y;              // [H]
+    ExpertWorkspace ws;
+    int32_t *status;
+};
+cudaError_t launch_expert_gateup(const ExpertArgs &a, const LaunchCfg &c);
+cudaError_t launch_expert_down(const ExpertArgs &a, const LaunchCfg &c);
+
+// ---------------------------------------------------------------- prefill --
+struct PrefillWorkspace {
+    int32_t *counts;    // [E]
+    int32_t *offsets;   // [E + 1]
+    int32_t *pairs;     // [T * top_k]
+    float *h;           // [T * top_k + T][inter]   (last T rows: shared expert)
+    float *r;           // [T * top_k + T][hidden]  (unweighted expert outputs)
+};
+size_t prefill_workspace_layout(int E, int hidden, int inter, int T, int top_k, void *base,
+                                PrefillWorkspace *ws);
+
+struct GroupArgs {
+    const int32_t *idx;
+    int T, top_k, E;
+    int32_t *counts, *offsets, *pairs;
+    int32_t *status;
+};
+cudaError_t launch_group(const GroupArgs &a, const LaunchCfg &c);
+
+struct PrefillArgs {
+    QMat gate, up, down, sh_gate, sh_up, sh_down;
+    int E, H, I, T, top_k;
+    const __half *x;       // [T][H]
+    const int32_t *idx;    // [T][top_k]
+    const float *weights;  // [T][top_k]
+    __half *y;             // [T][H]
+    PrefillWorkspace ws;
+    int32_t *status;
+};
+cudaError_t launch_prefill(const PrefillArgs &a, const LaunchCfg &c);
+
+// ------------------------------------------------------------ pack helpers --
+cudaError_t launch_pack(const uint8_t *codes, int rows, int cols, int bits, uint32_t *packed,
+                        cudaStream_t s);
+cudaError_t launch_unpack(const uint32_t *packed, int rows, int cols, int bits, uint8_t *codes,
+                          cudaStream_t s);
+
+// ---------------------------------------------------------------- helpers --
+template <class Kern, class... Args>
+cudaError_t launch_ex(Kern kernel, dim3 grid, dim3 block, size_t smem, const LaunchCfg &c,
+                      int cluster_x, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = c.stream;
+    cudaLaunchAttribute attrs[2];
+    int n = 0;
+    if (c.pdl) {
+        attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attrs[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (cluster_x > 1) {
+        attrs[n].id = cudaLaunchAttributeClusterDimension;
+        attrs[n].val.clusterDim.x = cluster_x;
+        attrs[n].val.clusterDim.y = 1;
+        attrs[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attrs;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory (once per
+// device and kernel; cheap to repeat).
+template <class Kern>
+cudaError_t set_smem(Kern kernel, size_t bytes)
+{
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace qmoe

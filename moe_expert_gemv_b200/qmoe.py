@@ -1,0 +1,313 @@
+"""Thin ctypes binding of libqmoe.so (C ABI in include/qmoe.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI.  Tensors are torch CUDA tensors (PyTorch supplies
+device memory and the current stream); fp16 data travels as torch.float16,
+packed words as torch.int32 (same bits as the uint32 words of the format).
+A non-zero status raises QmoeError.  There is no CPU fallback: if the library
+is missing or the device is not an sm_100 GPU the calls fail loudly.
+"""
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+_lib = None
+
+OK = 0
+DEV_BAD_EXPERT = 0x1
+DEV_TIMEOUT = 0x2
+
+
+class QmoeError(RuntimeError):
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__("%s: %s" % (what, status_string(code)))
+
+
+class CQMatrix(ctypes.Structure):
+    _fields_ = [("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("biases", ctypes.c_void_p), ("rows", ctypes.c_int32), ("cols", ctypes.c_int32),
+                ("bits", ctypes.c_int32), ("group", ctypes.c_int32)]
+
+
+class CMoeLayer(ctypes.Structure):
+    _fields_ = [("gate", CQMatrix), ("up", CQMatrix), ("down", CQMatrix),
+                ("sh_gate", CQMatrix), ("sh_up", CQMatrix), ("sh_down", CQMatrix),
+                ("num_experts", ctypes.c_int32), ("hidden", ctypes.c_int32),
+                ("inter", ctypes.c_int32)]
+
+
+def lib():
+    """Load libqmoe.so (building it first if it has never been built)."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB
+        if not os.path.exists(path):
+            _build.build()
+        L = ctypes.CDLL(path)
+        p, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        sig = {
+            "qgemv_affine": [p, p, i32, p, p, p],
+            "moe_router_topk": [p, p, i32, i32, p, p, p, p, p],
+            "moe_expert_workspace_bytes": [p, i32],
+            "moe_expert_qmlp": [p, p, p, p, i32, p, p, sz, p, p],
+            "moe_expert_gateup": [p, p, p, i32, p, sz, p, p],
+            "moe_expert_down": [p, p, p, i32, p, p, sz, p, p],
+            "moe_group_tokens": [p, i32, i32, i32, p, p, p, p, p],
+            "moe_prefill_workspace_bytes": [p, i32, i32],
+            "moe_prefill_qgemm": [p, p, i32, p, p, i32, p, p, sz, p, p],
+            "qmoe_pack_codes": [p, i32, i32, i32, p, p],
+            "qmoe_unpack_codes": [p, i32, i32, i32, p, p],
+            "qmoe_check_status": [p, p, p],
+            "qmoe_status_string": [ctypes.c_int],
+            "qmoe_set_dependent_launch": [i32],
+            "qmoe_version": [],
+        }
+        for name, args in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.moe_expert_workspace_bytes.restype = sz
+        L.moe_prefill_workspace_bytes.restype = sz
+        L.qmoe_status_string.restype = ctypes.c_char_p
+        L.qmoe_version.restype = i32
+        L.qmoe_set_dependent_launch.restype = i32
+        _lib = L
+    return _lib
+
+
+def status_string(code):
+    return lib().qmoe_status_string(int(code)).decode()
+
+
+def _check(code, what):
+    if code != OK:
+        raise QmoeError(code, what)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(None)
+
+
+def _need(t, dtype, what, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % what)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (what, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % what)
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (what, tuple(shape), tuple(t.shape)))
+    return t
+
+
+# ----------------------------------------------------------------- weights --
+class QMatrix:
+    """One affine-quantized matrix (or a stack of `stack` of them) on the GPU.
+
+    packed: int32 [*, rows, cols*bits/32]; scales/biases: float16 [*, rows, cols/64]."""
+
+    def __init__(self, packed, scales, biases, rows, cols, bits, stack=1):
+        self.packed, self.scales, self.biases = packed, scales, biases
+        self.rows, self.cols, self.bits, self.stack = rows, cols, bits, stack
+        _need(packed, torch.int32, "packed")
+        _need(scales, torch.float16, "scales")
+        _need(biases, torch.float16, "biases")
+        if packed.numel() != stack * rows * cols * bits // 32:
+            raise ValueError("packed has %d words, expected %d" %
+                             (packed.numel(), stack * rows * cols * bits // 32))
+        if scales.numel() != stack * rows * cols // 64 or biases.numel() != scales.numel():
+            raise ValueError("scales/biases size mismatch")
+        self.c = CQMatrix(packed.data_ptr(), scales.data_ptr(), biases.data_ptr(), rows, cols,
+                          bits, 64)
+
+    @classmethod
+    def from_numpy(cls, P, S, B, rows, cols, bits, device="cuda"):
+        """From (packed uint32, scales/biases fp16 bits as uint16) numpy arrays."""
+        stack = P.size // (rows * cols * bits // 32)
+        packed = torch.from_numpy(P.view("int32").copy()).to(device)
+        scales = torch.from_numpy(S.view("float16").copy()).to(device)
+        biases = torch.from_numpy(B.view("float16").copy()).to(device)
+        return cls(packed, scales, biases, rows, cols, bits, stack)
+
+
+class MoELayer:
+    """Routed experts (stacked gate/up/down) + shared expert (+ optional router)."""
+
+    def __init__(self, gate, up, down, sh_gate, sh_up, sh_down, num_experts, hidden, inter,
+                 router=None):
+        self.mats = dict(gate=gate, up=up, down=down, sh_gate=sh_gate, sh_up=sh_up,
+                         sh_down=sh_down)
+        self.router = router
+        self.num_experts, self.hidden, self.inter = num_experts, hidden, inter
+        self.c = CMoeLayer(gate.c, up.c, down.c, sh_gate.c, sh_up.c, sh_down.c, num_experts,
+                           hidden, inter)
+
+    @classmethod
+    def from_numpy(cls, m, E, H, I, device="cuda"):
+        """From a dict like moe_expert_gemv_b200.synth.moe_layer() returns."""
+        q = {}
+        for name, rows, cols in (("gate", I, H), ("up", I, H), ("down", H, I),
+                                 ("sh_gate", I, H), ("sh_up", I, H), ("sh_down", H, I)):
+            q[name] = QMatrix.from_numpy(*m[name], rows, cols, 4, device)
+        router = None
+        if "router" in m:
+            router = QMatrix.from_numpy(*m["router"], E, H, 8, device)
+        return cls(q["gate"], q["up"], q["down"], q["sh_gate"], q["sh_up"], q["sh_down"], E, H,
+                   I, router)
+
+
+# ------------------------------------------------------------- operations --
+def qgemv_affine(W, x, y=None, status=None):
+    """y[b] = W x[b] for x [B][K] float16 (B <= 8).  Returns y [B][N] float16."""
+    x = _need(x, torch.float16, "x")
+    x2 = x.reshape(-1, W.cols)
+    if y is None:
+        y = torch.empty(x2.shape[0], W.rows, dtype=torch.float16, device=x.device)
+    _need(y, torch.float16, "y", (x2.shape[0], W.rows))
+    _check(lib().qgemv_affine(ctypes.byref(W.c), _ptr(x2), x2.shape[0], _ptr(y), _ptr(status),
+                              _stream()), "qgemv_affine")
+    return y
+
+
+def moe_router_topk(router, x, top_k, idx=None, weights=None, logits=None, want_logits=False,
+                    status=None):
+    """Router logits -> softmax -> top-k -> renormalised weights for x [T][K].
+    Returns (idx int32 [T][k], weights float32 [T][k], logits float32 [T][E] or None)."""
+    x = _need(x, torch.float16, "x")
+    x2 = x.reshape(-1, router.cols)
+    T = x2.shape[0]
+    dev = x.device
+    if idx is None:
+        idx = torch.empty(T, top_k, dtype=torch.int32, device=dev)
+    if weights is None:
+        weights = torch.empty(T, top_k, dtype=torch.float32, device=dev)
+    if logits is None and want_logits:
+        logits = torch.empty(T, router.rows, dtype=torch.float32, device=dev)
+    _need(idx, torch.int32, "idx", (T, top_k))
+    _need(weights, torch.float32, "weights", (T, top_k))
+    if logits is not None:
+        _need(logits, torch.float32, "logits", (T, router.rows))
+    _check(lib().moe_router_topk(ctypes.byref(router.c), _ptr(x2), T, top_k, _ptr(idx),
+                                 _ptr(weights), _ptr(logits), _ptr(status), _stream()),
+           "moe_router_topk")
+    return idx, weights, logits
+
+
+def moe_expert_workspace_bytes(layer, top_k):
+    return lib().moe_expert_workspace_bytes(ctypes.byref(layer.c), top_k)
+
+
+def expert_workspace(layer, top_k, device="cuda"):
+    """A zero-filled workspace for moe_expert_qmlp (reusable across calls)."""
+    n = moe_expert_workspace_bytes(layer, top_k)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def moe_expert_qmlp(layer, x, idx, weights, y=None, workspace=None, status=None):
+    """y = shared(x) + sum_j weights[j] * expert_{idx[j]}(x) for one token x [H]."""
+    x = _need(x, torch.float16, "x").reshape(-1)
+    top_k = idx.numel()
+    _need(idx, torch.int32, "idx")
+    _need(weights, torch.float32, "weights")
+    if y is None:
+        y = torch.empty(layer.hidden, dtype=torch.float16, device=x.device)
+    if workspace is None:
+        workspace = expert_workspace(layer, top_k, x.device)
+    _check(lib().moe_expert_qmlp(ctypes.byref(layer.c), _ptr(x), _ptr(idx), _ptr(weights), top_k,
+                                 _ptr(y), _ptr(workspace), workspace.numel(), _ptr(status),
+                                 _stream()), "moe_expert_qmlp")
+    return y
+
+
+def moe_expert_gateup(layer, x, idx, workspace, status=None):
+    x = _need(x, torch.float16, "x").reshape(-1)
+    _check(lib().moe_expert_gateup(ctypes.byref(layer.c), _ptr(x), _ptr(idx), idx.numel(),
+                                   _ptr(workspace), workspace.numel(), _ptr(status), _stream()),
+           "moe_expert_gateup")
+
+
+def moe_expert_down(layer, idx, weights, y, workspace, status=None):
+    _check(lib().moe_expert_down(ctypes.byref(layer.c), _ptr(idx), _ptr(weights), idx.numel(),
+                                 _ptr(y), _ptr(workspace), workspace.numel(), _ptr(status),
+                                 _stream()), "moe_expert_down")
+    return y
+
+
+def moe_group_tokens(idx, num_experts, status=None):
+    """Counting sort of a chunk's (token, slot) pairs by expert.
+    Returns (counts [E], offsets [E+1], pairs [T*k]) int32."""
+    _need(idx, torch.int32, "idx")
+    T, k = idx.shape
+    dev = idx.device
+    counts = torch.empty(num_experts, dtype=torch.int32, device=dev)
+    offsets = torch.empty(num_experts + 1, dtype=torch.int32, device=dev)
+    pairs = torch.empty(T * k, dtype=torch.int32, device=dev)
+    _check(lib().moe_group_tokens(_ptr(idx), T, k, num_experts, _ptr(counts), _ptr(offsets),
+                                  _ptr(pairs), _ptr(status), _stream()), "moe_group_tokens")
+    return counts, offsets, pairs
+
+
+def moe_prefill_workspace_bytes(layer, tokens, top_k):
+    return lib().moe_prefill_workspace_bytes(ctypes.byref(layer.c), tokens, top_k)
+
+
+def moe_prefill_qgemm(layer, x, idx, weights, y=None, workspace=None, status=None):
+    """y[t] = shared(x[t]) + sum_j weights[t][j] expert_{idx[t][j]}(x[t]), x [T][H]."""
+    x = _need(x, torch.float16, "x")
+    T = x.shape[0]
+    _need(idx, torch.int32, "idx")
+    _need(weights, torch.float32, "weights")
+    top_k = idx.shape[1]
+    if y is None:
+        y = torch.empty(T, layer.hidden, dtype=torch.float16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(moe_prefill_workspace_bytes(layer, T, top_k), dtype=torch.uint8,
+                                device=x.device)
+    _check(lib().moe_prefill_qgemm(ctypes.byref(layer.c), _ptr(x), T, _ptr(idx), _ptr(weights),
+                                   top_k, _ptr(y), _ptr(workspace), workspace.numel(),
+                                   _ptr(status), _stream()), "moe_prefill_qgemm")
+    return y
+
+
+def qmoe_pack_codes(codes, bits):
+    """uint8 codes [rows][cols] -> int32 packed words [rows][cols*bits/32]."""
+    _need(codes, torch.uint8, "codes")
+    rows, cols = codes.shape
+    packed = torch.empty(rows, cols * bits // 32, dtype=torch.int32, device=codes.device)
+    _check(lib().qmoe_pack_codes(_ptr(codes), rows, cols, bits, _ptr(packed), _stream()),
+           "qmoe_pack_codes")
+    return packed
+
+
+def qmoe_unpack_codes(packed, rows, cols, bits):
+    _need(packed, torch.int32, "packed")
+    codes = torch.empty(rows, cols, dtype=torch.uint8, device=packed.device)
+    _check(lib().qmoe_unpack_codes(_ptr(packed), rows, cols, bits, _ptr(codes), _stream()),
+           "qmoe_unpack_codes")
+    return codes
+
+
+def qmoe_check_status(status=None):
+    """Synchronise the current stream; return the device flags (and clear them).
+    Raises QmoeError on a CUDA failure; flags are returned, not raised."""
+    flags = ctypes.c_int32(0)
+    rc = lib().qmoe_check_status(_ptr(status), _stream(), ctypes.byref(flags))
+    if rc not in (OK, -5, -6):
+        raise QmoeError(rc, "qmoe_check_status")
+    return flags.value
+
+
+def qmoe_set_dependent_launch(enable):
+    return bool(lib().qmoe_set_dependent_launch(1 if enable else 0))
+
+
+def qmoe_version():
+    return lib().qmoe_version()

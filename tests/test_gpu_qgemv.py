@@ -1,0 +1,111 @@
+"""qgemv_affine and the pack helpers on the GPU against the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_expert_gemv_b200 import qmoe, synth
+from tests._util import assert_close, f16_bits, to_dev_f16
+
+pytestmark = pytest.mark.gpu
+
+
+def run_qgemv(P, S, B, N, K, bits, x16):
+    W = qmoe.QMatrix.from_numpy(P, S, B, N, K, bits)
+    y = qmoe.qgemv_affine(W, to_dev_f16(x16))
+    assert qmoe.qmoe_check_status() == 0
+    return f16_bits(y)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_pack_unpack_bit_exact(cuda_dev, bits):
+    g = np.random.default_rng(bits)
+    for rows, cols in ((1, 8), (7, 64), (33, 2816)):
+        if cols % (32 // bits):
+            continue
+        codes = g.integers(0, 2 ** bits, (rows, cols)).astype(np.uint8)
+        packed = qmoe.qmoe_pack_codes(torch.from_numpy(codes).cuda(), bits)
+        want = oracle.pack(codes, bits)
+        assert np.array_equal(packed.cpu().numpy().view(np.uint32), want)
+        back = qmoe.qmoe_unpack_codes(packed, rows, cols, bits)
+        assert np.array_equal(back.cpu().numpy(), codes)
+        words = g.integers(0, 2 ** 32, (rows, cols * bits // 32), dtype=np.uint64).astype(np.uint32)
+        un = qmoe.qmoe_unpack_codes(torch.from_numpy(words.view(np.int32)).cuda(), rows, cols, bits)
+        assert np.array_equal(un.cpu().numpy(), oracle.unpack(words, rows, cols, bits))
+
+
+def test_config0_single_qgemv(cuda_dev):
+    """N=512, K=1024, batch 1 (the small dense case)."""
+    N, K = 512, 1024
+    P, S, B = synth.dense(0, N, K)
+    x16 = synth.activations(0, 1, K)
+    y = run_qgemv(P, S, B, N, K, 4, x16)
+    y64, _ = oracle.qgemv(P, S, B, N, K, 4, x16)
+    assert_close(y.view(np.float16), y64, what="config 0")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("N", [14336, 4096])
+@pytest.mark.parametrize("Bt", [1, 4, 8])
+def test_config1_decode_sweep(cuda_dev, N, Bt):
+    """K=4096, N in {14336, 4096}, batch 1/4/8, full output against the oracle."""
+    K = 4096
+    P, S, B = synth.dense(1, N, K)
+    x16 = synth.activations(1 + Bt, Bt, K)
+    y = run_qgemv(P, S, B, N, K, 4, x16)
+    y64, _ = oracle.qgemv(P, S, B, N, K, 4, x16)
+    assert_close(y.view(np.float16), y64, what="config 1 N=%d B=%d" % (N, Bt))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("N,K", [(8, 64), (24, 192), (40, 704), (136, 128), (16, 2816)])
+def test_small_and_ragged_shapes(cuda_dev, bits, N, K):
+    """Tile tails (N % 16 == 8), a single group, K = 704 (11 groups), every batch."""
+    P, S, B = synth.qmatrix(synth.rng(N, K, bits), N, K, bits)
+    for Bt in range(1, 9):
+        x16 = synth.activations(N + K + Bt, Bt, K)
+        y = run_qgemv(P, S, B, N, K, bits, x16)
+        y64, _ = oracle.qgemv(P, S, B, N, K, bits, x16)
+        assert_close(y.view(np.float16), y64, what="N=%d K=%d B=%d bits=%d" % (N, K, Bt, bits))
+
+
+def test_zero_input_positive_zero(cuda_dev):
+    N, K = 64, 256
+    P, S, B = synth.dense(3, N, K)
+    y = run_qgemv(P, S, B, N, K, 4, np.zeros((3, K), np.uint16))
+    assert np.all(y == 0)
+
+
+def test_zero_codes_bias_only(cuda_dev):
+    N, K = 48, 512
+    _, S, B = synth.dense(4, N, K)
+    P = np.zeros((N, K // 8), np.uint32)
+    x16 = synth.activations(4, 2, K)
+    y = run_qgemv(P, S, B, N, K, 4, x16)
+    y64, _ = oracle.qgemv(P, S, B, N, K, 4, x16)
+    assert_close(y.view(np.float16), y64, what="bias only")
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_unit_vectors_exact(cuda_dev, bits):
+    """x = e_k: every output is one dequantised weight, exact after fp16 rounding."""
+    N, K = 32, 256
+    P, S, B = synth.qmatrix(synth.rng(9, bits), N, K, bits)
+    ks = [0, 1, 5, 63, 64, 130, 255]
+    x = np.zeros((len(ks), K))
+    for i, k in enumerate(ks):
+        x[i, k] = 1.0
+    x16 = synth.to_f16_bits(x)
+    y = run_qgemv(P, S, B, N, K, bits, x16)
+    _, y16 = oracle.qgemv(P, S, B, N, K, bits, x16)
+    assert np.array_equal(y, y16)
+
+
+def test_repeat_calls_bitwise_identical(cuda_dev):
+    N, K = 4096, 4096
+    P, S, B = synth.dense(5, N, K)
+    W = qmoe.QMatrix.from_numpy(P, S, B, N, K, 4)
+    x = to_dev_f16(synth.activations(5, 4, K))
+    a = qmoe.qgemv_affine(W, x).clone()
+    for _ in range(3):
+        assert torch.equal(qmoe.qgemv_affine(W, x), a)
