@@ -47,7 +47,7 @@ ROUTER_CALL_BYTES = ROUTER_BYTES + H * 2 + TOPK * 8
 
 # DRAM traffic per launch of the dominant kernel from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
-# source it was taken on (sha256 of csrc/expert.cu); otherwise reported null.
+# source it was taken on (sha256 of csrc/decode.cu); otherwise reported null.
 NCU_TRAFFIC = {}
 
 
@@ -246,58 +246,44 @@ def run_decode(args, dist):
     torch.cuda.set_device(dev)
     layers, m0, x, idx, wt, y, ws = build_decode(args, dev)
     nl = args.layers
+    stack = qmoe.DecodeStack(layers, TOPK, dev)
 
-    def step():
+    def fused_step():
+        qmoe.moe_decode_layers(stack, x, y, idx, wt)
+
+    # the same step as per-layer calls (router, gate/up, down kernels)
+    def unfused_step():
         for l in range(nl):
             qmoe.moe_router_topk(layers[l].router, x[l:l + 1], TOPK, idx[l:l + 1], wt[l:l + 1])
             qmoe.moe_expert_qmlp(layers[l], x[l], idx[l], wt[l], y[l], ws[l])
 
-    def gateup_only():
-        for l in range(nl):
-            qmoe.moe_expert_gateup(layers[l], x[l], idx[l], ws[l])
-
-    def down_only():
-        for l in range(nl):
-            qmoe.moe_expert_down(layers[l], idx[l], wt[l], y[l], ws[l])
-
-    def router_only():
-        for l in range(nl):
-            qmoe.moe_router_topk(layers[l].router, x[l:l + 1], TOPK, idx[l:l + 1], wt[l:l + 1])
-
     stream = torch.cuda.Stream()
-    graphs = {}
     with torch.cuda.stream(stream):
-        step()   # eager warm-up (first-use set-up happens outside capture)
-        gateup_only()
-        down_only()
+        fused_step()
+        unfused_step()
         torch.cuda.synchronize()
         assert qmoe.qmoe_check_status() == 0
-        for name, fn in (("step", step), ("gateup", gateup_only), ("down", down_only),
-                         ("router", router_only)):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                fn()
-            graphs[name] = g
+        g_unfused = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_unfused, stream=stream):
+            unfused_step()
         torch.cuda.synchronize()
 
         for _ in range(args.warmup):
-            graphs["step"].replay()
+            fused_step()
         torch.cuda.synchronize()
         clocks = ClockSampler(dev.index) if dist.rank == 0 else None
         if clocks:
             clocks.start()
-        ms = timed_replays(graphs["step"].replay, args.steps, dist)
+        ms = timed_replays(fused_step, args.steps, dist)
         clk = clocks.stop() if clocks else None
         ms = dist.max(ms)
         flags = qmoe.qmoe_check_status()
 
-        # per-kernel averages (each graph chains the kernel over the 30 layers)
+        # the per-layer kernel path, for comparison
         reps = max(20, args.steps // 10)
-        kern = {}
-        for name in ("gateup", "down", "router"):
-            for _ in range(3):
-                graphs[name].replay()
-            kern[name] = timed_replays(graphs[name].replay, reps) / (reps * nl)
+        for _ in range(3):
+            g_unfused.replay()
+        unfused_ms = timed_replays(g_unfused.replay, reps) / reps
 
         # end to end through host buffers: H2D of every layer's input token,
         # the step, D2H of every layer's output, each step
@@ -306,16 +292,16 @@ def run_decode(args, dist):
 
         def e2e_step():
             x.copy_(x_host, non_blocking=True)
-            graphs["step"].replay()
+            fused_step()
             y_host.copy_(y, non_blocking=True)
 
         for _ in range(3):
             e2e_step()
         e2e_steps = max(10, args.steps // 4)
         e2e_ms = dist.max(timed_replays(e2e_step, e2e_steps, dist))
-    graphs.clear()
-    return dict(ms=ms, kern=kern, clk=clk, flags=flags, e2e_ms=e2e_ms, e2e_steps=e2e_steps,
-                m0=m0, h2d=x.numel() * 2, d2h=y.numel() * 2)
+    del g_unfused
+    return dict(ms=ms, unfused_ms=unfused_ms, clk=clk, flags=flags, e2e_ms=e2e_ms,
+                e2e_steps=e2e_steps, m0=m0, h2d=x.numel() * 2, d2h=y.numel() * 2)
 
 
 def main_decode(args):
@@ -327,10 +313,11 @@ def main_decode(args):
     hbm, _, peak_kind = peaks()
     nl, K, N = args.layers, args.steps, dist.world
     value = nl * K * N / (r["ms"] / 1e3)
-    gu_ms = r["kern"]["gateup"]
-    gu_gbs = GATEUP_BYTES / (gu_ms / 1e3) / 1e9
-    trf = NCU_TRAFFIC.get("expert_gateup_kernel")
-    traffic = trf["bytes"] if trf and trf["sha"] == source_sha("expert.cu") else None
+    launch_ms = r["ms"] / K
+    step_bytes = nl * (LAYER_BYTES + 2 * H * 2)
+    gbs = step_bytes / (launch_ms / 1e3) / 1e9
+    trf = NCU_TRAFFIC.get("moe_decode_kernel")
+    traffic = trf["bytes"] if trf and trf["sha"] == source_sha("decode.cu") else None
     line = {
         "metric": "qGEMV/MoE-layer weight-stream GB/s vs HBM peak; MoE decode layers/s",
         "value": round(value, 1),
@@ -338,7 +325,7 @@ def main_decode(args):
         "n_gpus": N,
         "steps": K,
         "warmup": args.warmup,
-        "ms_per_step": round(r["ms"] / K, 5),
+        "ms_per_step": round(launch_ms, 5),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -349,29 +336,23 @@ def main_decode(args):
                         "SwiGLU experts %dx%d 4-bit g64 + shared expert)" % (nl, H, TOPK, E, I, H),
             "layers": nl, "experts": E, "hidden": H, "inter": I, "top_k": TOPK,
             "bytes_per_layer": LAYER_BYTES,
-            "weight_stream_gbs": round(LAYER_BYTES * nl * K / (r["ms"] / 1e3) / 1e9, 1),
+            "weight_stream_gbs": round(LAYER_BYTES * nl / (launch_ms / 1e3) / 1e9, 1),
             "l2": "inputs larger than L2: 12.96 GB of weights, each step streams 915 MB",
-            "graph": "CUDA graph of the 30-layer step, kernels chained by programmatic "
-                     "dependent launch",
+            "path": "moe_decode_layers: one persistent cooperative launch per step",
             "parallelism": "replicas" if N > 1 else "single GPU",
         },
         "roofline": {
-            "bound": "hbm", "kernel": "expert_gateup_kernel",
-            "achieved": round(gu_gbs, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
-            "frac": round(gu_gbs / hbm, 4), "traffic": traffic,
-            "algorithmic_bytes_per_launch": GATEUP_BYTES,
-            "launch_us": round(gu_ms * 1e3, 3),
+            "bound": "hbm", "kernel": "moe_decode_kernel",
+            "achieved": round(gbs, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+            "frac": round(gbs / hbm, 4), "traffic": traffic,
+            "algorithmic_bytes_per_launch": step_bytes,
+            "launch_us": round(launch_ms * 1e3, 2),
         },
-        "kernels_us": {k: round(v * 1e3, 3) for k, v in r["kern"].items()},
-        "kernels_gbs": {
-            "gateup": round(GATEUP_BYTES / (r["kern"]["gateup"] / 1e3) / 1e9, 1),
-            "down": round(DOWN_BYTES / (r["kern"]["down"] / 1e3) / 1e9, 1),
-            "router": round(ROUTER_CALL_BYTES / (r["kern"]["router"] / 1e3) / 1e9, 1),
-        },
+        "unfused_layers_per_s": round(nl / (r["unfused_ms"] / 1e3), 1),
         "e2e": {"value": round(nl * r["e2e_steps"] * N / (r["e2e_ms"] / 1e3), 1),
                 "unit": "layers/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
-        "gpu_launches": 3 * nl * K,
+        "gpu_launches": K,
         "device_flags": r["flags"],
     }
     if r["clk"]:

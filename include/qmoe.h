@@ -167,6 +167,37 @@ qmoe_status moe_expert_down(const qmoe_moe_layer *L, const int32_t *idx, const f
                             int32_t *status_dev, void *stream);
 
 /* ---------------------------------------------------------------------------
+ * The decode loop over a stack of MoE layers for one token per layer, fused
+ * into one persistent launch ("내부 구조" section: the router picks the top-8
+ * experts of each layer, the shared expert's output is added to the routed
+ * output, and generation repeats this routed-layer loop token by token).
+ * For each layer l < n_layers:
+ *   logits = router_l x[l];  idx[l], weights[l] = top_k of softmax(logits)
+ *   y[l] = shared_l(x[l]) + sum_j weights[l][j] * expert_{l, idx[l][j]}(x[l])
+ * with exactly the arithmetic of moe_router_topk followed by moe_expert_qmlp.
+ * Layer l+1 starts after layer l has finished, as it would if it consumed
+ * y[l]; the weights of later layers are streamed ahead of time.
+ * layers: host array of n_layers descriptors (same shapes); routers: host
+ * array of n_layers router matrices (rows = num_experts <= 128, a multiple
+ * of 8, cols = hidden).  x, y: fp16 [n_layers][hidden]; idx: int32
+ * [n_layers][top_k], weights: fp32 [n_layers][top_k], logits: fp32
+ * [n_layers][num_experts]; idx, weights, logits may be NULL.
+ * Shapes: hidden % 256 == 0, inter % 64 == 0, top_k 1..16.
+ * workspace: moe_decode_workspace_bytes() bytes, 16-byte aligned, ZERO-FILLED
+ * before first use; each successful call leaves it zero-filled again.  Calls
+ * sharing a workspace must not overlap in time.  Stacks of more than 32
+ * layers are processed 32 layers per launch.  The launch is cooperative (one
+ * CTA per SM, all resident); it fails with QMOE_ERR_CUDA if the GPU is busy
+ * with other work that prevents co-residency.
+ * ------------------------------------------------------------------------- */
+size_t moe_decode_workspace_bytes(const qmoe_moe_layer *L, int32_t top_k);
+
+qmoe_status moe_decode_layers(const qmoe_moe_layer *layers, const qmoe_qmatrix *routers,
+                              int32_t n_layers, const uint16_t *x, int32_t top_k, uint16_t *y,
+                              int32_t *idx, float *weights, float *logits, void *workspace,
+                              size_t workspace_bytes, int32_t *status_dev, void *stream);
+
+/* ---------------------------------------------------------------------------
  * Prefill grouping ("내부 구조" section: a chunk's tokens are gathered per
  * expert so one fetched expert serves many rows).
  *   counts[e]  = number of (token, slot) pairs with idx == e

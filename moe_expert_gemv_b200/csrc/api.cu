@@ -310,6 +310,79 @@ qmoe_status moe_expert_qmlp(const qmoe_moe_layer *L, const uint16_t *x, const in
     return cuda_status(launch_expert_down(a, c));
 }
 
+size_t moe_decode_workspace_bytes(const qmoe_moe_layer *L, int32_t top_k)
+{
+    if (!L || L->hidden <= 0 || L->inter <= 0 || L->num_experts <= 0 || top_k < 1)
+        return 0;
+    return decode_workspace_layout(L->num_experts, L->hidden, L->inter, top_k, nullptr, nullptr);
+}
+
+qmoe_status moe_decode_layers(const qmoe_moe_layer *layers, const qmoe_qmatrix *routers,
+                              int32_t n_layers, const uint16_t *x, int32_t top_k, uint16_t *y,
+                              int32_t *idx, float *weights, float *logits, void *workspace,
+                              size_t workspace_bytes, int32_t *status_dev, void *stream)
+{
+    if (!layers || !routers || !x || !y || n_layers < 1)
+        return QMOE_ERR_INVALID_ARG;
+    const qmoe_moe_layer &L0 = layers[0];
+    qmoe_status s;
+    for (int l = 0; l < n_layers; ++l) {
+        const qmoe_moe_layer &Ll = layers[l];
+        if (Ll.num_experts != L0.num_experts || Ll.hidden != L0.hidden || Ll.inter != L0.inter)
+            return QMOE_ERR_INVALID_ARG;
+        if ((s = check_expert_common(&Ll, top_k)) != QMOE_OK)
+            return s;
+        if ((s = check_qmatrix(&routers[l], L0.num_experts, L0.hidden, 8)) != QMOE_OK)
+            return s;
+    }
+    if (L0.num_experts > 128 || L0.hidden % 256)
+        return QMOE_ERR_UNSUPPORTED;
+    if (!aligned(x, 2) || !aligned(y, 2) || (idx && !aligned(idx, 4)) ||
+        (weights && !aligned(weights, 4)) || (logits && !aligned(logits, 4)) ||
+        (status_dev && !aligned(status_dev, 4)))
+        return QMOE_ERR_ALIGNMENT;
+    if (!workspace)
+        return QMOE_ERR_WORKSPACE;
+    if (!aligned(workspace, 16))
+        return QMOE_ERR_ALIGNMENT;
+    if (workspace_bytes < moe_decode_workspace_bytes(&L0, top_k))
+        return QMOE_ERR_WORKSPACE;
+    DevState *d;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    const LaunchCfg c = launch_cfg(d, stream);
+    DecodeArgs a;
+    a.E = L0.num_experts;
+    a.H = L0.hidden;
+    a.I = L0.inter;
+    a.top_k = top_k;
+    a.NS_r = 0;
+    a.status = status_dev ? status_dev : d->status;
+    decode_workspace_layout(a.E, a.H, a.I, top_k, workspace, &a.ws);
+    for (int l0 = 0; l0 < n_layers; l0 += kDecodeMaxLayers) {
+        const int n = n_layers - l0 < kDecodeMaxLayers ? n_layers - l0 : kDecodeMaxLayers;
+        a.L = n;
+        a.x = reinterpret_cast<const __half *>(x) + (size_t)l0 * a.H;
+        a.y = reinterpret_cast<__half *>(y) + (size_t)l0 * a.H;
+        a.idx = idx ? idx + (size_t)l0 * top_k : nullptr;
+        a.weights = weights ? weights + (size_t)l0 * top_k : nullptr;
+        a.logits = logits ? logits + (size_t)l0 * a.E : nullptr;
+        for (int l = 0; l < n; ++l) {
+            const qmoe_moe_layer &Ll = layers[l0 + l];
+            const qmoe_qmatrix *m[7] = {&routers[l0 + l], &Ll.gate, &Ll.up, &Ll.down,
+                                        &Ll.sh_gate, &Ll.sh_up, &Ll.sh_down};
+            for (int i = 0; i < 7; ++i) {
+                a.layer[l].P[i] = m[i]->packed;
+                a.layer[l].S[i] = reinterpret_cast<const __half *>(m[i]->scales);
+                a.layer[l].B[i] = reinterpret_cast<const __half *>(m[i]->biases);
+            }
+        }
+        if ((s = cuda_status(launch_decode(a, c))) != QMOE_OK)
+            return s;
+    }
+    return QMOE_OK;
+}
+
 qmoe_status moe_group_tokens(const int32_t *idx, int32_t tokens, int32_t top_k,
                              int32_t num_experts, int32_t *counts, int32_t *offsets,
                              int32_t *pairs, int32_t *status_dev, void *stream)

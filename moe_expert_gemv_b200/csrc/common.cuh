@@ -15,7 +15,7 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
-#include "../../include/qmoe.h"
+#include "qmoe.h"
 
 namespace qmoe {
 
@@ -290,7 +290,7 @@ __host__ __device__ __forceinline__ int tile_stride_words(int cols, int bits)
 // (group, column) sit in 8 consecutive lanes; each lane loads its 8 values at
 // once and the group sum is reduced with shuffles, so no thread walks a group
 // serially.  All `nthreads` threads (a multiple of 32) starting at `tid` must
-// take part.
+// take part.  With xsum == nullptr only the fragments are written.
 template <int BITS, class Load>
 __device__ __forceinline__ void stage_x(uint4 *xs, float *xsum, int G, int ncol, int nvec, Load load,
                                         int tid, int nthreads)
@@ -327,13 +327,14 @@ __device__ __forceinline__ void stage_x(uint4 *xs, float *xsum, int G, int ncol,
         part += __shfl_xor_sync(0xffffffffu, part, 1);
         part += __shfl_xor_sync(0xffffffffu, part, 2);
         part += __shfl_xor_sync(0xffffffffu, part, 4);
-        if (t < total && (t & 7) == 0)
+        if (xsum && t < total && (t & 7) == 0)
             xsum[(size_t)v * G * 8 + g * 8 + n] = part;
     }
     // columns ncol..7 of the sums are zero
-    for (int t = tid; t < nvec * G * 8; t += nthreads)
-        if ((t & 7) >= ncol)
-            xsum[t] = 0.f;
+    if (xsum)
+        for (int t = tid; t < nvec * G * 8; t += nthreads)
+            if ((t & 7) >= ncol)
+                xsum[t] = 0.f;
 }
 
 }  // namespace qmoe

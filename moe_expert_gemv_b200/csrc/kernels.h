@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/qmoe.h"
+#include "qmoe.h"
 
 namespace qmoe {
 
@@ -67,6 +67,38 @@ struct ExpertArgs {
 };
 cudaError_t launch_expert_gateup(const ExpertArgs &a, const LaunchCfg &c);
 cudaError_t launch_expert_down(const ExpertArgs &a, const LaunchCfg &c);
+
+// ------------------------------------------------ fused multi-layer decode --
+constexpr int kDecodeMaxLayers = 32;
+
+struct DecodeLayerPtrs {   // router, gate, up, down, shared gate, shared up, shared down
+    const uint32_t *P[7];
+    const __half *S[7];
+    const __half *B[7];
+};
+
+struct DecodeWorkspace {
+    unsigned *ctl;                   // control words: router / done / exit / abort counters,
+                                     // then one readiness counter per slot (zero between launches)
+    int *counters;                   // [H / 32] arrival counters (zero between launches)
+    float *logits_part;              // [2][E]
+    uint4 *hfrag;                    // [top_k + 1][I/64][2][2][4] fp16 fragments of h (hi, lo)
+    float *part;                     // [top_k + 1][H] per-expert down outputs
+};
+size_t decode_workspace_layout(int E, int H, int I, int top_k, void *base, DecodeWorkspace *ws);
+
+struct DecodeArgs {
+    int L, E, H, I, top_k, NS_r;
+    const __half *x;      // [L][H]
+    __half *y;            // [L][H]
+    int32_t *idx;         // [L][top_k] or null
+    float *weights;       // [L][top_k] or null
+    float *logits;        // [L][E] or null
+    DecodeWorkspace ws;
+    int32_t *status;
+    DecodeLayerPtrs layer[kDecodeMaxLayers];
+};
+cudaError_t launch_decode(const DecodeArgs &a, const LaunchCfg &c);
 
 // ---------------------------------------------------------------- prefill --
 struct PrefillWorkspace {

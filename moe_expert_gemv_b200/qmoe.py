@@ -57,6 +57,8 @@ def lib():
             "moe_expert_gateup": [p, p, p, i32, p, sz, p, p],
             "moe_expert_down": [p, p, p, i32, p, p, sz, p, p],
             "moe_group_tokens": [p, i32, i32, i32, p, p, p, p, p],
+            "moe_decode_workspace_bytes": [p, i32],
+            "moe_decode_layers": [p, p, i32, p, i32, p, p, p, p, p, sz, p, p],
             "moe_prefill_workspace_bytes": [p, i32, i32],
             "moe_prefill_qgemm": [p, p, i32, p, p, i32, p, p, sz, p, p],
             "qmoe_pack_codes": [p, i32, i32, i32, p, p],
@@ -72,6 +74,7 @@ def lib():
             fn.restype = ctypes.c_int
         L.moe_expert_workspace_bytes.restype = sz
         L.moe_prefill_workspace_bytes.restype = sz
+        L.moe_decode_workspace_bytes.restype = sz
         L.qmoe_status_string.restype = ctypes.c_char_p
         L.qmoe_version.restype = i32
         L.qmoe_set_dependent_launch.restype = i32
@@ -238,6 +241,43 @@ def moe_expert_down(layer, idx, weights, y, workspace, status=None):
     _check(lib().moe_expert_down(ctypes.byref(layer.c), _ptr(idx), _ptr(weights), idx.numel(),
                                  _ptr(y), _ptr(workspace), workspace.numel(), _ptr(status),
                                  _stream()), "moe_expert_down")
+    return y
+
+
+class DecodeStack:
+    """Host-side descriptors of a stack of MoE layers (with routers) for
+    moe_decode_layers, plus its zero-filled workspace."""
+
+    def __init__(self, layers, top_k, device="cuda"):
+        self.layers = list(layers)
+        n = len(self.layers)
+        self.top_k = top_k
+        self.c_layers = (CMoeLayer * n)(*[L.c for L in self.layers])
+        self.c_routers = (CQMatrix * n)(*[L.router.c for L in self.layers])
+        nbytes = lib().moe_decode_workspace_bytes(ctypes.byref(self.layers[0].c), top_k)
+        self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+
+def moe_decode_layers(stack, x, y=None, idx=None, weights=None, logits=None, status=None):
+    """One token per layer through the whole stack in one fused launch.
+    x, y: float16 [n_layers][hidden]; idx int32 / weights float32 [n_layers][top_k];
+    logits float32 [n_layers][num_experts] (optional)."""
+    n = len(stack.layers)
+    L0 = stack.layers[0]
+    x = _need(x, torch.float16, "x", (n, L0.hidden))
+    if y is None:
+        y = torch.empty(n, L0.hidden, dtype=torch.float16, device=x.device)
+    _need(y, torch.float16, "y", (n, L0.hidden))
+    if idx is not None:
+        _need(idx, torch.int32, "idx", (n, stack.top_k))
+    if weights is not None:
+        _need(weights, torch.float32, "weights", (n, stack.top_k))
+    if logits is not None:
+        _need(logits, torch.float32, "logits", (n, L0.num_experts))
+    _check(lib().moe_decode_layers(stack.c_layers, stack.c_routers, n, _ptr(x), stack.top_k,
+                                   _ptr(y), _ptr(idx), _ptr(weights), _ptr(logits),
+                                   _ptr(stack.workspace), stack.workspace.numel(), _ptr(status),
+                                   _stream()), "moe_decode_layers")
     return y
 
 

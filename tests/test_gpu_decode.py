@@ -1,0 +1,102 @@
+"""Fused multi-layer decode (moe_decode_layers) against the CPU oracle: for
+every layer the router's indices (bit-exact rules as in the router tests) and
+the layer output y = shared(x) + sum_j wt_j expert_{idx_j}(x)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_expert_gemv_b200 import qmoe, synth
+from tests._util import assert_close, f16_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def make_stack(seed, n, E, H, I, top_k):
+    ms = [synth.moe_layer(seed, l, E=E, H=H, I=I) for l in range(n)]
+    layers = [qmoe.MoELayer.from_numpy(m, E, H, I) for m in ms]
+    return ms, qmoe.DecodeStack(layers, top_k)
+
+
+def check_layers(ms, E, H, I, k, x16, y, idx, wt, lg, layers=None):
+    for l in (range(len(ms)) if layers is None else layers):
+        m = ms[l]
+        l64, oidx, _ = oracle.router(*m["router"], E, H, 8, x16[l:l + 1], k)
+        assert np.abs(lg[l] - l64[0]).max() <= 1e-5 * np.abs(l64).max()
+        sidx, swt = oracle.topk_from_logits(lg[l:l + 1], k)
+        assert np.array_equal(idx[l], sidx[0]), "layer %d: selection on device logits" % l
+        assert_close(wt[l], swt[0], what="layer %d weights" % l)
+        assert np.array_equal(idx[l], oidx[0]), "layer %d: indices differ from the fp64 oracle" % l
+        y64, _ = oracle.Layer(m, E, H, I).moe(x16[l:l + 1], idx[l:l + 1],
+                                              wt[l:l + 1].astype(np.float64))
+        assert_close(y[l].view(np.float16), y64[0], what="layer %d output" % l)
+
+
+def run(stack, x16, E, k):
+    n = x16.shape[0]
+    x = torch.from_numpy(x16.view(np.float16).copy()).cuda()
+    idx = torch.empty(n, k, dtype=torch.int32, device="cuda")
+    wt = torch.empty(n, k, dtype=torch.float32, device="cuda")
+    lg = torch.empty(n, E, dtype=torch.float32, device="cuda")
+    y = qmoe.moe_decode_layers(stack, x, idx=idx, weights=wt, logits=lg)
+    assert qmoe.qmoe_check_status() == 0
+    return f16_bits(y), idx.cpu().numpy(), wt.cpu().numpy(), lg.cpu().numpy()
+
+
+@pytest.mark.parametrize("E,H,I,k,n", [(16, 256, 64, 4, 3), (32, 512, 128, 8, 2),
+                                       (128, 1024, 256, 8, 2), (64, 768, 192, 16, 2),
+                                       (8, 256, 64, 1, 4)])
+def test_small_stacks(cuda_dev, E, H, I, k, n):
+    ms, stack = make_stack(E + H, n, E, H, I, k)
+    x16 = np.concatenate([synth.activations(7 + l, 1, H, layer=l) for l in range(n)])
+    y, idx, wt, lg = run(stack, x16, E, k)
+    check_layers(ms, E, H, I, k, x16, y, idx, wt, lg)
+
+
+def test_config3_three_layers_and_repeat(cuda_dev):
+    E, H, I, k = synth.MOE_E, synth.MOE_H, synth.MOE_I, synth.MOE_TOPK
+    ms, stack = make_stack(3, 3, E, H, I, k)
+    x16 = np.concatenate([synth.activations(3, 1, H, layer=l) for l in range(3)])
+    y, idx, wt, lg = run(stack, x16, E, k)
+    check_layers(ms, E, H, I, k, x16, y, idx, wt, lg)
+    # the workspace is back to zero and a second call reproduces every bit
+    assert torch.count_nonzero(stack.workspace[:16]) == 0
+    y2, idx2, wt2, lg2 = run(stack, x16, E, k)
+    assert np.array_equal(y, y2) and np.array_equal(idx, idx2)
+    assert np.array_equal(wt, wt2) and np.array_equal(lg, lg2)
+
+
+def test_matches_unfused_path(cuda_dev):
+    """Same bits as moe_router_topk + moe_expert_qmlp would give within the
+    tolerance, and identical routing."""
+    E, H, I, k = synth.MOE_E, synth.MOE_H, synth.MOE_I, synth.MOE_TOPK
+    ms, stack = make_stack(5, 2, E, H, I, k)
+    x16 = np.concatenate([synth.activations(5, 1, H, layer=l) for l in range(2)])
+    y, idx, wt, lg = run(stack, x16, E, k)
+    for l in range(2):
+        G = stack.layers[l]
+        xd = torch.from_numpy(x16[l].view(np.float16).copy()).cuda()
+        i2, w2, _ = qmoe.moe_router_topk(G.router, xd[None], k)
+        y2 = qmoe.moe_expert_qmlp(G, xd, i2.reshape(-1), w2.reshape(-1))
+        assert np.array_equal(i2.cpu().numpy()[0], idx[l])
+        assert_close(y[l].view(np.float16), f16_bits(y2).view(np.float16).astype(np.float64),
+                     what="fused vs unfused")
+
+
+@pytest.mark.slow
+def test_config3_thirty_layers_sampled(cuda_dev):
+    """The full decode step: 30 layers, 12.96 GB of weights; every layer's
+    routing is checked, outputs of a sample of layers against the oracle."""
+    E, H, I, k, n = synth.MOE_E, synth.MOE_H, synth.MOE_I, synth.MOE_TOPK, synth.MOE_LAYERS
+    layers, ms = [], []
+    for l in range(n):
+        m = synth.moe_layer(0, l)
+        layers.append(qmoe.MoELayer.from_numpy(m, E, H, I))
+        ms.append({"router": m["router"]} if l not in (0, 13, 29) else m)
+    stack = qmoe.DecodeStack(layers, k)
+    x16 = np.concatenate([synth.activations(0, 1, H, layer=l) for l in range(n)])
+    y, idx, wt, lg = run(stack, x16, E, k)
+    for l in range(n):
+        l64, oidx, _ = oracle.router(*ms[l]["router"], E, H, 8, x16[l:l + 1], k)
+        assert np.array_equal(idx[l], oidx[0])
+    check_layers(ms, E, H, I, k, x16, y, idx, wt, lg, layers=(0, 13, 29))
