@@ -154,6 +154,24 @@ qmoe_status moe_expert_qmlp(const qmoe_moe_layer *L, const uint16_t *x, const in
                             const float *weights, int32_t top_k, uint16_t *y, void *workspace,
                             size_t workspace_bytes, int32_t *status_dev, void *stream);
 
+/* moe_expert_qmlp for callers that cannot allocate device memory.  The pages
+ * have no counterpart: this exists for callers with no way to obtain a
+ * workspace -- a plugin or embedded runtime handed only a stream and tensor
+ * pointers, a framework whose memory pool may not be touched from the calling
+ * thread, a real-time path that must not enter an allocator.  It computes
+ * exactly what moe_expert_qmlp computes, using a scratch buffer built into
+ * the library: a 1 MiB __device__ array that every GPU loading the library
+ * holds until the process exits.  Requests whose workspace
+ * (moe_expert_workspace_bytes) exceeds 1 MiB return QMOE_ERR_WORKSPACE.
+ * It allocates and frees nothing.  The first call on each device looks up the
+ * array's device address (with that device current); make that first call
+ * before any stream capture.  Each call clears the buffer's counters on
+ * `stream` before its kernels run.  Every call shares the one buffer, so
+ * calls that overlap on the GPU (for instance on two streams) race. */
+qmoe_status moe_expert_qmlp_noalloc(const qmoe_moe_layer *L, const uint16_t *x,
+                                    const int32_t *idx, const float *weights, int32_t top_k,
+                                    uint16_t *y, int32_t *status_dev, void *stream);
+
 /* h_j = silu(gate_e x) * (up_e x) for the top_k routed experts e = idx[j] and
  * the shared expert (slot top_k), fp32, kept in the workspace. */
 qmoe_status moe_expert_gateup(const qmoe_moe_layer *L, const uint16_t *x, const int32_t *idx,
