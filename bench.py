@@ -455,6 +455,39 @@ def main_other(args):
             ms = timed_replays(g.replay, reps) / (reps * 20)
             out["results"].append({"T": T, "us": round(ms * 1e3, 3),
                                    "tokens_per_s": round(T / (ms / 1e3), 1)})
+    elif args.workload == "prefill":
+        # 128-token chunk, Zipf(1.1) routing, rotating over 4 layers (1.7 GB of
+        # weights) so consecutive calls do not find their experts in L2
+        nl = 4
+        Gs = [qmoe.MoELayer.from_numpy(synth.moe_layer(args.seed, l), E, H, I, dev)
+              for l in range(nl)]
+        idx_np, wt_np = synth.zipf_routing(args.seed)
+        T = idx_np.shape[0]
+        x = torch.from_numpy(synth.activations(args.seed, T, H).view(np.float16).copy()).to(dev)
+        idx = torch.from_numpy(idx_np).to(dev)
+        wt = torch.from_numpy(wt_np).to(dev)
+        y = torch.empty(T, H, dtype=torch.float16, device=dev)
+        ws = torch.empty(qmoe.moe_prefill_workspace_bytes(Gs[0], T, TOPK), dtype=torch.uint8,
+                         device=dev)
+
+        def run():
+            for G in Gs:
+                qmoe.moe_prefill_qgemm(G, x, idx, wt, y, ws)
+        run()
+        torch.cuda.synchronize()
+        assert qmoe.qmoe_check_status() == 0
+        for _ in range(3):
+            run()
+        reps = max(5, args.steps // 50)
+        ms = timed_replays(run, reps) / (reps * nl)
+        touched = int(np.unique(idx_np).size)
+        nbytes = (touched + 1) * EXPERT_BYTES
+        flops = 2.0 * (T * TOPK + T) * 3 * I * H
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out["results"].append({"T": T, "experts_touched": touched, "us": round(ms * 1e3, 2),
+                               "tokens_per_s": round(T / (ms / 1e3), 1),
+                               "weight_GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                               "useful_TFLOP/s": round(flops / (ms / 1e3) / 1e12, 2)})
     else:
         out["error"] = "workload not available"
     print(json.dumps(out), flush=True)

@@ -105,8 +105,14 @@ struct PrefillWorkspace {
     int32_t *counts;    // [E]
     int32_t *offsets;   // [E + 1]
     int32_t *pairs;     // [T * top_k]
-    float *h;           // [T * top_k + T][inter]   (last T rows: shared expert)
-    float *r;           // [T * top_k + T][hidden]  (unweighted expert outputs)
+    int32_t *inv;       // [T * top_k] position of each (token, slot) pair
+    int32_t *tile_off;  // [E + 2] first 8-token tile of each slot (slot E: shared expert)
+    int32_t *unit_ctr;  // [2] work counters of the gate/up and down kernels
+    uint4 *xfrag;       // [T][H/64][2][4] x in mma fragment order
+    float *xsum;        // [T][H/64][8] group sums of x (column 0)
+    uint4 *hfrag;       // [T * top_k + T][I/64][2][2][4] h (hi, lo) fragments per position
+    float *hsum;        // [T * top_k + T][I/64][2] group sums of h hi / lo
+    float *r;           // [T * top_k + T][H] unweighted expert outputs per position
 };
 size_t prefill_workspace_layout(int E, int hidden, int inter, int T, int top_k, void *base,
                                 PrefillWorkspace *ws);
