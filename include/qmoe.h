@@ -189,18 +189,28 @@ qmoe_status moe_expert_down(const qmoe_moe_layer *L, const int32_t *idx, const f
  * into one persistent launch ("내부 구조" section: the router picks the top-8
  * experts of each layer, the shared expert's output is added to the routed
  * output, and generation repeats this routed-layer loop token by token).
- * For each layer l < n_layers:
+ *
+ * The layers are first repacked once (like the pages' install-time repack)
+ * into the kernel's streaming layout: every work item's codes, scales and
+ * biases become one contiguous block, so each item is a single large copy.
+ * The packed layer holds exactly the bytes of the row-major one (router +
+ * all experts + shared expert), permuted.
+ *   moe_decode_pack_bytes(L)            bytes of one packed layer
+ *   moe_decode_pack_layer(L, router, packed, bytes, stream)
+ *       L: the layer in the row-major format; router: rows = num_experts
+ *       (<= 128, a multiple of 8), cols = hidden, 8-bit; hidden % 256 == 0,
+ *       inter % 64 == 0.  packed: device memory, 16-byte aligned.
+ *
+ * For each layer l < n_layers (packed_layers: host array of device pointers):
  *   logits = router_l x[l];  idx[l], weights[l] = top_k of softmax(logits)
  *   y[l] = shared_l(x[l]) + sum_j weights[l][j] * expert_{l, idx[l][j]}(x[l])
- * with exactly the arithmetic of moe_router_topk followed by moe_expert_qmlp.
- * Layer l+1 starts after layer l has finished, as it would if it consumed
- * y[l]; the weights of later layers are streamed ahead of time.
- * layers: host array of n_layers descriptors (same shapes); routers: host
- * array of n_layers router matrices (rows = num_experts <= 128, a multiple
- * of 8, cols = hidden).  x, y: fp16 [n_layers][hidden]; idx: int32
- * [n_layers][top_k], weights: fp32 [n_layers][top_k], logits: fp32
- * [n_layers][num_experts]; idx, weights, logits may be NULL.
- * Shapes: hidden % 256 == 0, inter % 64 == 0, top_k 1..16.
+ * with the arithmetic of moe_router_topk followed by moe_expert_qmlp (fp32
+ * accumulation of exact products).  Layer l+1 starts after layer l has
+ * finished, as it would if it consumed y[l]; the weights of later layers
+ * that do not depend on the routing are streamed ahead of time.
+ * x, y: fp16 [n_layers][hidden]; idx: int32 [n_layers][top_k], weights: fp32
+ * [n_layers][top_k], logits: fp32 [n_layers][num_experts]; idx, weights and
+ * logits may be NULL.  top_k 1..16.
  * workspace: moe_decode_workspace_bytes() bytes, 16-byte aligned, ZERO-FILLED
  * before first use; each successful call leaves it zero-filled again.  Calls
  * sharing a workspace must not overlap in time.  Stacks of more than 32
@@ -208,11 +218,18 @@ qmoe_status moe_expert_down(const qmoe_moe_layer *L, const int32_t *idx, const f
  * CTA per SM, all resident); it fails with QMOE_ERR_CUDA if the GPU is busy
  * with other work that prevents co-residency.
  * ------------------------------------------------------------------------- */
-size_t moe_decode_workspace_bytes(const qmoe_moe_layer *L, int32_t top_k);
+size_t moe_decode_pack_bytes(const qmoe_moe_layer *L);
 
-qmoe_status moe_decode_layers(const qmoe_moe_layer *layers, const qmoe_qmatrix *routers,
-                              int32_t n_layers, const uint16_t *x, int32_t top_k, uint16_t *y,
-                              int32_t *idx, float *weights, float *logits, void *workspace,
+qmoe_status moe_decode_pack_layer(const qmoe_moe_layer *L, const qmoe_qmatrix *router,
+                                  void *packed, size_t packed_bytes, void *stream);
+
+size_t moe_decode_workspace_bytes(int32_t num_experts, int32_t hidden, int32_t inter,
+                                  int32_t top_k);
+
+qmoe_status moe_decode_layers(const void *const *packed_layers, int32_t n_layers,
+                              int32_t num_experts, int32_t hidden, int32_t inter,
+                              const uint16_t *x, int32_t top_k, uint16_t *y, int32_t *idx,
+                              float *weights, float *logits, void *workspace,
                               size_t workspace_bytes, int32_t *status_dev, void *stream);
 
 /* ---------------------------------------------------------------------------

@@ -310,33 +310,73 @@ qmoe_status moe_expert_qmlp(const qmoe_moe_layer *L, const uint16_t *x, const in
     return cuda_status(launch_expert_down(a, c));
 }
 
-size_t moe_decode_workspace_bytes(const qmoe_moe_layer *L, int32_t top_k)
+size_t moe_decode_pack_bytes(const qmoe_moe_layer *L)
 {
-    if (!L || L->hidden <= 0 || L->inter <= 0 || L->num_experts <= 0 || top_k < 1)
+    if (!L || L->num_experts < 1 || L->hidden < 256 || L->inter < 64)
         return 0;
-    return decode_workspace_layout(L->num_experts, L->hidden, L->inter, top_k, nullptr, nullptr);
+    return decode_pack_bytes(L->num_experts, L->hidden, L->inter);
 }
 
-qmoe_status moe_decode_layers(const qmoe_moe_layer *layers, const qmoe_qmatrix *routers,
-                              int32_t n_layers, const uint16_t *x, int32_t top_k, uint16_t *y,
-                              int32_t *idx, float *weights, float *logits, void *workspace,
+qmoe_status moe_decode_pack_layer(const qmoe_moe_layer *L, const qmoe_qmatrix *router, void *packed,
+                                  size_t packed_bytes, void *stream)
+{
+    qmoe_status s = check_layer(L);
+    if (s != QMOE_OK)
+        return s;
+    if ((s = check_qmatrix(router, L->num_experts, L->hidden, 8)) != QMOE_OK)
+        return s;
+    if (L->num_experts > 128 || L->num_experts % 8 || L->hidden % 256)
+        return QMOE_ERR_UNSUPPORTED;
+    if (!packed)
+        return QMOE_ERR_INVALID_ARG;
+    if (!aligned(packed, 16))
+        return QMOE_ERR_ALIGNMENT;
+    if (packed_bytes < moe_decode_pack_bytes(L))
+        return QMOE_ERR_WORKSPACE;
+    DevState *d;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    DecodePackArgs a;
+    a.router = qmat(*router);
+    a.gate = qmat(L->gate);
+    a.up = qmat(L->up);
+    a.down = qmat(L->down);
+    a.sh_gate = qmat(L->sh_gate);
+    a.sh_up = qmat(L->sh_up);
+    a.sh_down = qmat(L->sh_down);
+    a.E = L->num_experts;
+    a.H = L->hidden;
+    a.I = L->inter;
+    return cuda_status(launch_decode_pack(a, packed, static_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_decode_workspace_bytes(int32_t num_experts, int32_t hidden, int32_t inter,
+                                  int32_t top_k)
+{
+    if (num_experts < 1 || hidden <= 0 || inter <= 0 || top_k < 1)
+        return 0;
+    return decode_workspace_layout(num_experts, hidden, inter, top_k, nullptr, nullptr);
+}
+
+qmoe_status moe_decode_layers(const void *const *packed_layers, int32_t n_layers,
+                              int32_t num_experts, int32_t hidden, int32_t inter,
+                              const uint16_t *x, int32_t top_k, uint16_t *y, int32_t *idx,
+                              float *weights, float *logits, void *workspace,
                               size_t workspace_bytes, int32_t *status_dev, void *stream)
 {
-    if (!layers || !routers || !x || !y || n_layers < 1)
+    if (!packed_layers || !x || !y || n_layers < 1)
         return QMOE_ERR_INVALID_ARG;
-    const qmoe_moe_layer &L0 = layers[0];
-    qmoe_status s;
-    for (int l = 0; l < n_layers; ++l) {
-        const qmoe_moe_layer &Ll = layers[l];
-        if (Ll.num_experts != L0.num_experts || Ll.hidden != L0.hidden || Ll.inter != L0.inter)
-            return QMOE_ERR_INVALID_ARG;
-        if ((s = check_expert_common(&Ll, top_k)) != QMOE_OK)
-            return s;
-        if ((s = check_qmatrix(&routers[l], L0.num_experts, L0.hidden, 8)) != QMOE_OK)
-            return s;
-    }
-    if (L0.num_experts > 128 || L0.hidden % 256)
+    if (num_experts < 8 || num_experts > 128 || num_experts % 8 || hidden < 256 ||
+        hidden % 256 || inter < 64 || inter % 64)
         return QMOE_ERR_UNSUPPORTED;
+    if (top_k < 1 || top_k > 16 || top_k > num_experts)
+        return QMOE_ERR_INVALID_ARG;
+    for (int l = 0; l < n_layers; ++l) {
+        if (!packed_layers[l])
+            return QMOE_ERR_INVALID_ARG;
+        if (!aligned(packed_layers[l], 16))
+            return QMOE_ERR_ALIGNMENT;
+    }
     if (!aligned(x, 2) || !aligned(y, 2) || (idx && !aligned(idx, 4)) ||
         (weights && !aligned(weights, 4)) || (logits && !aligned(logits, 4)) ||
         (status_dev && !aligned(status_dev, 4)))
@@ -345,16 +385,17 @@ qmoe_status moe_decode_layers(const qmoe_moe_layer *layers, const qmoe_qmatrix *
         return QMOE_ERR_WORKSPACE;
     if (!aligned(workspace, 16))
         return QMOE_ERR_ALIGNMENT;
-    if (workspace_bytes < moe_decode_workspace_bytes(&L0, top_k))
+    if (workspace_bytes < moe_decode_workspace_bytes(num_experts, hidden, inter, top_k))
         return QMOE_ERR_WORKSPACE;
     DevState *d;
+    qmoe_status s;
     if ((s = device_state(&d)) != QMOE_OK)
         return s;
     const LaunchCfg c = launch_cfg(d, stream);
     DecodeArgs a;
-    a.E = L0.num_experts;
-    a.H = L0.hidden;
-    a.I = L0.inter;
+    a.E = num_experts;
+    a.H = hidden;
+    a.I = inter;
     a.top_k = top_k;
     a.NS_r = 0;
     a.status = status_dev ? status_dev : d->status;
@@ -367,16 +408,8 @@ qmoe_status moe_decode_layers(const qmoe_moe_layer *layers, const qmoe_qmatrix *
         a.idx = idx ? idx + (size_t)l0 * top_k : nullptr;
         a.weights = weights ? weights + (size_t)l0 * top_k : nullptr;
         a.logits = logits ? logits + (size_t)l0 * a.E : nullptr;
-        for (int l = 0; l < n; ++l) {
-            const qmoe_moe_layer &Ll = layers[l0 + l];
-            const qmoe_qmatrix *m[7] = {&routers[l0 + l], &Ll.gate, &Ll.up, &Ll.down,
-                                        &Ll.sh_gate, &Ll.sh_up, &Ll.sh_down};
-            for (int i = 0; i < 7; ++i) {
-                a.layer[l].P[i] = m[i]->packed;
-                a.layer[l].S[i] = reinterpret_cast<const __half *>(m[i]->scales);
-                a.layer[l].B[i] = reinterpret_cast<const __half *>(m[i]->biases);
-            }
-        }
+        for (int l = 0; l < n; ++l)
+            a.layer[l] = packed_layers[l0 + l];
         if ((s = cuda_status(launch_decode(a, c))) != QMOE_OK)
             return s;
     }

@@ -69,15 +69,20 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+// try_wait with a suspend-time hint: the waiting thread is parked (it issues
+// nothing) until the phase completes or the hint expires, so waiting warps do
+// not take issue slots from the warps doing the math.
+constexpr uint32_t kSuspendHintNs = 100000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -191,16 +196,57 @@ __device__ __forceinline__ void dequant8_word(uint32_t w, uint32_t *p)
     p[1] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w >> 8, 0x00FF00FFu, magic)), k1024));
 }
 
+// Cheaper dequantisation for the streaming kernels: the code itself becomes
+// the fp16 bit pattern (no exponent bits), i.e. the subnormal q * 2^-24, or
+// 16q * 2^-24 for a nibble in bits 4..7.  fp16 subnormals enter the tensor
+// core without being flushed (measured: group partials within ~2e-6 relative
+// of exact), so a whole word costs one shift and four ANDs.  Pairs:
+//   p[0] = (c0, c4) * 2^-24     p[1] = (c1, c5) * 2^-20
+//   p[2] = (c2, c6) * 2^-24     p[3] = (c3, c7) * 2^-20
+// The 2^-24 and 2^-20 classes go to separate mma accumulators c (class 0)
+// and d (class 1) and are recombined as 2^20 * (16 c + d).
+__device__ __forceinline__ void dequant4s_word(uint32_t w, uint32_t *p)
+{
+    const uint32_t ws = w >> 8;
+    p[0] = w & 0x000F000Fu;
+    p[1] = w & 0x00F000F0u;
+    p[2] = ws & 0x000F000Fu;
+    p[3] = ws & 0x00F000F0u;
+}
+// 8-bit: bytes as subnormals q * 2^-24: p[0] = (c0, c2), p[1] = (c1, c3).
+__device__ __forceinline__ void dequant8s_word(uint32_t w, uint32_t *p)
+{
+    p[0] = w & 0x00FF00FFu;
+    p[1] = (w >> 8) & 0x00FF00FFu;
+}
+constexpr float kSub24 = 16777216.f;   // 2^24
+constexpr float kSub20 = 1048576.f;    // 2^20
+
+// x order matching dequant4s_word, k-blocks (c0,c4)(c2,c6) | (c8,c12)(c10,c14)
+// | (c1,c5)(c3,c7) | (c9,c13)(c11,c15): class-0 codes in the first 8 slots.
+__host__ __device__ __forceinline__ int xperm_s4(int i)
+{
+    const int hi = (i & 4) << 1;           // +8 for i = 4..7 and 12..15
+    const int odd = (i >> 3) & 1;          // class 1 for i >= 8
+    const int j = i & 3;                   // (0,4)(2,6) pattern
+    return hi + odd + ((j >> 1) << 1) + ((j & 1) << 2);
+}
+
 // Order in which a thread (quad index tig) needs the 16 x values
 // x[64g + 16 tig + perm[i]] of group g so that its two 16-byte x fragments
 // line up with the A fragments produced above (k-slot order of m16n8k16).
-__host__ __device__ __forceinline__ int xperm(int bits, int i)
+// `kind`: 4 (dequant4_word), 8 (dequant8_word / dequant8s_word), or
+// kPermS4 (dequant4s_word).
+constexpr int kPermS4 = 5;
+__host__ __device__ __forceinline__ int xperm(int kind, int i)
 {
     // 4-bit: pairs (0,4)(1,5)(2,6)(3,7)(8,12)(9,13)(10,14)(11,15)
     // 8-bit: pairs (0,2)(1,3)(4,6)(5,7)(8,10)(9,11)(12,14)(13,15)
+    if (kind == kPermS4)
+        return xperm_s4(i);
     const int hi = i & 8;
     const int j = i & 7;
-    if (bits == 4)
+    if (kind == 4)
         return hi + (j >> 1) + ((j & 1) << 2);
     return hi + ((j >> 2) << 2) + ((j >> 1) & 1) + ((j & 1) << 1);
 }

@@ -71,11 +71,12 @@ cudaError_t launch_expert_down(const ExpertArgs &a, const LaunchCfg &c);
 // ------------------------------------------------ fused multi-layer decode --
 constexpr int kDecodeMaxLayers = 32;
 
-struct DecodeLayerPtrs {   // router, gate, up, down, shared gate, shared up, shared down
-    const uint32_t *P[7];
-    const __half *S[7];
-    const __half *B[7];
+struct DecodePackArgs {   // one MoE layer in the row-major (MLX) format
+    QMat router, gate, up, down, sh_gate, sh_up, sh_down;
+    int E, H, I;
 };
+size_t decode_pack_bytes(int E, int H, int I);
+cudaError_t launch_decode_pack(const DecodePackArgs &a, void *dst, cudaStream_t s);
 
 struct DecodeWorkspace {
     unsigned *ctl;                   // control words: router / done / exit / abort counters,
@@ -96,7 +97,7 @@ struct DecodeArgs {
     float *logits;        // [L][E] or null
     DecodeWorkspace ws;
     int32_t *status;
-    DecodeLayerPtrs layer[kDecodeMaxLayers];
+    const void *layer[kDecodeMaxLayers];   // packed layers (decode_pack layout)
 };
 cudaError_t launch_decode(const DecodeArgs &a, const LaunchCfg &c);
 

@@ -57,8 +57,10 @@ def lib():
             "moe_expert_gateup": [p, p, p, i32, p, sz, p, p],
             "moe_expert_down": [p, p, p, i32, p, p, sz, p, p],
             "moe_group_tokens": [p, i32, i32, i32, p, p, p, p, p],
-            "moe_decode_workspace_bytes": [p, i32],
-            "moe_decode_layers": [p, p, i32, p, i32, p, p, p, p, p, sz, p, p],
+            "moe_decode_pack_bytes": [p],
+            "moe_decode_pack_layer": [p, p, p, sz, p],
+            "moe_decode_workspace_bytes": [i32, i32, i32, i32],
+            "moe_decode_layers": [p, i32, i32, i32, i32, p, i32, p, p, p, p, p, sz, p, p],
             "moe_prefill_workspace_bytes": [p, i32, i32],
             "moe_prefill_qgemm": [p, p, i32, p, p, i32, p, p, sz, p, p],
             "qmoe_pack_codes": [p, i32, i32, i32, p, p],
@@ -75,6 +77,7 @@ def lib():
         L.moe_expert_workspace_bytes.restype = sz
         L.moe_prefill_workspace_bytes.restype = sz
         L.moe_decode_workspace_bytes.restype = sz
+        L.moe_decode_pack_bytes.restype = sz
         L.qmoe_status_string.restype = ctypes.c_char_p
         L.qmoe_version.restype = i32
         L.qmoe_set_dependent_launch.restype = i32
@@ -245,37 +248,47 @@ def moe_expert_down(layer, idx, weights, y, workspace, status=None):
 
 
 class DecodeStack:
-    """Host-side descriptors of a stack of MoE layers (with routers) for
-    moe_decode_layers, plus its zero-filled workspace."""
+    """A stack of MoE layers (each with its router) repacked once into the
+    fused decode kernel's streaming layout, plus its zero-filled workspace."""
 
     def __init__(self, layers, top_k, device="cuda"):
         self.layers = list(layers)
-        n = len(self.layers)
+        L0 = self.layers[0]
         self.top_k = top_k
-        self.c_layers = (CMoeLayer * n)(*[L.c for L in self.layers])
-        self.c_routers = (CQMatrix * n)(*[L.router.c for L in self.layers])
-        nbytes = lib().moe_decode_workspace_bytes(ctypes.byref(self.layers[0].c), top_k)
-        self.workspace = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        self.E, self.H, self.I = L0.num_experts, L0.hidden, L0.inter
+        nbytes = lib().moe_decode_pack_bytes(ctypes.byref(L0.c))
+        if nbytes == 0:
+            raise ValueError("layer shape not supported by the fused decode")
+        self.packed = []
+        for L in self.layers:
+            buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+            _check(lib().moe_decode_pack_layer(ctypes.byref(L.c), ctypes.byref(L.router.c),
+                                               _ptr(buf), nbytes, _stream()),
+                   "moe_decode_pack_layer")
+            self.packed.append(buf)
+        torch.cuda.current_stream().synchronize()
+        self.c_packed = (ctypes.c_void_p * len(self.packed))(*[b.data_ptr() for b in self.packed])
+        ws = lib().moe_decode_workspace_bytes(self.E, self.H, self.I, top_k)
+        self.workspace = torch.zeros(ws, dtype=torch.uint8, device=device)
 
 
 def moe_decode_layers(stack, x, y=None, idx=None, weights=None, logits=None, status=None):
     """One token per layer through the whole stack in one fused launch.
     x, y: float16 [n_layers][hidden]; idx int32 / weights float32 [n_layers][top_k];
     logits float32 [n_layers][num_experts] (optional)."""
-    n = len(stack.layers)
-    L0 = stack.layers[0]
-    x = _need(x, torch.float16, "x", (n, L0.hidden))
+    n = len(stack.packed)
+    x = _need(x, torch.float16, "x", (n, stack.H))
     if y is None:
-        y = torch.empty(n, L0.hidden, dtype=torch.float16, device=x.device)
-    _need(y, torch.float16, "y", (n, L0.hidden))
+        y = torch.empty(n, stack.H, dtype=torch.float16, device=x.device)
+    _need(y, torch.float16, "y", (n, stack.H))
     if idx is not None:
         _need(idx, torch.int32, "idx", (n, stack.top_k))
     if weights is not None:
         _need(weights, torch.float32, "weights", (n, stack.top_k))
     if logits is not None:
-        _need(logits, torch.float32, "logits", (n, L0.num_experts))
-    _check(lib().moe_decode_layers(stack.c_layers, stack.c_routers, n, _ptr(x), stack.top_k,
-                                   _ptr(y), _ptr(idx), _ptr(weights), _ptr(logits),
+        _need(logits, torch.float32, "logits", (n, stack.E))
+    _check(lib().moe_decode_layers(stack.c_packed, n, stack.E, stack.H, stack.I, _ptr(x),
+                                   stack.top_k, _ptr(y), _ptr(idx), _ptr(weights), _ptr(logits),
                                    _ptr(stack.workspace), stack.workspace.numel(), _ptr(status),
                                    _stream()), "moe_decode_layers")
     return y

@@ -100,3 +100,51 @@ def test_config3_thirty_layers_sampled(cuda_dev):
         l64, oidx, _ = oracle.router(*ms[l]["router"], E, H, 8, x16[l:l + 1], k)
         assert np.array_equal(idx[l], oidx[0])
     check_layers(ms, E, H, I, k, x16, y, idx, wt, lg, layers=(0, 13, 29))
+
+
+def expected_pack(m, E, H, I):
+    """The packed streaming layout, rebuilt with numpy from the row-major
+    arrays (bytes)."""
+    GH, GI = H // 64, I // 64
+    out = []
+    rP = m["router"][0].view(np.uint8).reshape(E, H)
+    rS, rB = m["router"][1].reshape(E, GH), m["router"][2].reshape(E, GH)
+    sb = lambda S, B: np.stack([S, B], axis=-1).astype(np.uint16).view(np.uint8).reshape(-1)
+    for rb in range(E // 8):
+        for kh in range(2):
+            codes = rP[rb * 8:rb * 8 + 8, kh * H // 2:(kh + 1) * H // 2].reshape(8, H // 32, 16)
+            perm = np.array([[c ^ (4 * (r & 1)) for c in range(H // 32)] for r in range(8)])
+            codes = np.stack([codes[r][perm[r]] for r in range(8)])
+            rows = slice(rb * 8, rb * 8 + 8)
+            half = slice(kh * GH // 2, (kh + 1) * GH // 2)
+            out += [codes.reshape(-1), sb(rS[rows, half], rB[rows, half])]
+    def mat(name, e, rows_n, cols):
+        P, S, B = m[name]
+        P = P.reshape(-1, rows_n, cols // 8)[e if P.ndim == 3 else 0]
+        S = S.reshape(-1, rows_n, cols // 64)[e if S.ndim == 3 else 0]
+        Bb = B.reshape(-1, rows_n, cols // 64)[e if B.ndim == 3 else 0]
+        return P.view(np.uint8).reshape(rows_n, cols // 2), S, Bb
+    for e in range(E + 1):
+        g, u, d = ("gate", "up", "down") if e < E else ("sh_gate", "sh_up", "sh_down")
+        gP, gS, gB = mat(g, e, I, H)
+        uP, uS, uB = mat(u, e, I, H)
+        dP, dS, dB = mat(d, e, H, I)
+        for o in range(I // 4):
+            r = slice(4 * o, 4 * o + 4)
+            codes = np.concatenate([gP[r], uP[r]]).reshape(8, H // 32, 16)
+            perm = np.array([[c ^ (2 * (rr & 3)) for c in range(H // 32)] for rr in range(8)])
+            codes = np.stack([codes[rr][perm[rr]] for rr in range(8)])
+            out += [codes.reshape(-1), sb(np.concatenate([gS[r], uS[r]]), np.concatenate([gB[r], uB[r]]))]
+        for t in range(H // 32):
+            r = slice(32 * t, 32 * t + 32)
+            out += [dP[r].reshape(-1), sb(dS[r], dB[r])]
+    return np.concatenate(out)
+
+
+def test_pack_layout_bit_exact(cuda_dev):
+    E, H, I = 16, 512, 128
+    ms, stack = make_stack(91, 1, E, H, I, 4)
+    got = stack.packed[0].cpu().numpy()
+    want = expected_pack(ms[0], E, H, I)
+    assert got.size == want.size
+    assert np.array_equal(got, want)
