@@ -48,7 +48,10 @@ ROUTER_CALL_BYTES = ROUTER_BYTES + H * 2 + TOPK * 8
 # DRAM traffic per launch of the dominant kernel from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source it was taken on (sha256 of csrc/decode.cu); otherwise reported null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # 6-layer capture (186,702,592 B) scaled to the 30 layers of one launch
+    "moe_decode_kernel": {"bytes": 933512960, "sha": "d09a383d19ca7a25"},
+}
 
 
 def parse():
@@ -172,6 +175,11 @@ class Dist:
         if self.pg:
             import torch.distributed as dist
             dist.destroy_process_group()
+
+
+def whole_job_rate(units_per_rank, n_ranks, ms_max):
+    """Units all ranks processed per second, over the slowest rank's time."""
+    return units_per_rank * n_ranks / (ms_max / 1e3)
 
 
 def timed_replays(fn, iters, dist=None):
@@ -304,6 +312,19 @@ def run_decode(args, dist):
                 e2e_steps=e2e_steps, m0=m0, h2d=x.numel() * 2, d2h=y.numel() * 2)
 
 
+def decode_config(nl, n_ranks):
+    return {
+        "workload": "moe_decode: 1 token x %d MoE layers (router 8-bit 128x%d, top-%d of %d "
+                    "SwiGLU experts %dx%d 4-bit g64 + shared expert)" % (nl, H, TOPK, E, I, H),
+        "layers": nl, "experts": E, "hidden": H, "inter": I, "top_k": TOPK,
+        "bytes_per_layer": LAYER_BYTES,
+        "l2": "inputs larger than L2: %.2f GB of weights, each step streams %.0f MB"
+              % (nl * LAYER_BYTES / 1e9, nl * LAYER_BYTES / 1e6),
+        "path": "moe_decode_layers: one persistent cooperative launch per step",
+        "parallelism": "replicas x%d" % n_ranks if n_ranks > 1 else "single GPU",
+    }
+
+
 def main_decode(args):
     dist = Dist()
     r = run_decode(args, dist)
@@ -312,7 +333,7 @@ def main_decode(args):
         return
     hbm, _, peak_kind = peaks()
     nl, K, N = args.layers, args.steps, dist.world
-    value = nl * K * N / (r["ms"] / 1e3)
+    value = whole_job_rate(nl * K, N, r["ms"])
     launch_ms = r["ms"] / K
     step_bytes = nl * (LAYER_BYTES + 2 * H * 2)
     gbs = step_bytes / (launch_ms / 1e3) / 1e9
@@ -331,16 +352,8 @@ def main_decode(args):
         "vs_baseline": None,
         "dtype": "f16xf16->f32 (affine int4 weights)",
         "data": "synthetic (seeded; value distributions of the pages' workloads)",
-        "config": {
-            "workload": "moe_decode: 1 token x %d MoE layers (router 8-bit 128x%d, top-%d of %d "
-                        "SwiGLU experts %dx%d 4-bit g64 + shared expert)" % (nl, H, TOPK, E, I, H),
-            "layers": nl, "experts": E, "hidden": H, "inter": I, "top_k": TOPK,
-            "bytes_per_layer": LAYER_BYTES,
-            "weight_stream_gbs": round(LAYER_BYTES * nl / (launch_ms / 1e3) / 1e9, 1),
-            "l2": "inputs larger than L2: 12.96 GB of weights, each step streams 915 MB",
-            "path": "moe_decode_layers: one persistent cooperative launch per step",
-            "parallelism": "replicas" if N > 1 else "single GPU",
-        },
+        "config": dict(decode_config(nl, N),
+                       weight_stream_gbs=round(LAYER_BYTES * nl / (launch_ms / 1e3) / 1e9, 1)),
         "roofline": {
             "bound": "hbm", "kernel": "moe_decode_kernel",
             "achieved": round(gbs, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
@@ -349,7 +362,7 @@ def main_decode(args):
             "launch_us": round(launch_ms * 1e3, 2),
         },
         "unfused_layers_per_s": round(nl / (r["unfused_ms"] / 1e3), 1),
-        "e2e": {"value": round(nl * r["e2e_steps"] * N / (r["e2e_ms"] / 1e3), 1),
+        "e2e": {"value": round(whole_job_rate(nl * r["e2e_steps"], N, r["e2e_ms"]), 1),
                 "unit": "layers/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": K,
@@ -385,14 +398,17 @@ def main_reference(args):
     line = {
         "impl": "reference",
         "metric": "qGEMV/MoE-layer weight-stream GB/s vs HBM peak; MoE decode layers/s",
-        "value": round(value, 3), "unit": "layers/s", "n_gpus": 1, "steps": done,
+        "value": round(value, 3), "unit": "layers/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": done,
         "warmup": warm, "ms_per_step": round(el / done * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "moe_decode (CPU oracle, one layer per step)", "layers": 1,
-                   "experts": E, "hidden": H, "inter": I, "top_k": TOPK},
+        "config": dict(decode_config(args.layers, 1),
+                       path="CPU oracle (fp64), one layer of the stack per step"),
         "cpu_baseline": {"value": round(value, 3), "unit": "layers/s", "cores": 1,
                          "kind": "oracle",
-                         "sample": "%d decode layers of layer 0's weights, single thread" % done},
+                         "sample": "%d decode layers (router + shared + 8 routed experts) "
+                                   "of layer 0's weights, fresh seeded tokens, single thread"
+                                   % done},
         "e2e": {"value": round(value, 3), "unit": "layers/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

@@ -69,6 +69,20 @@ def test_small_and_ragged_shapes(cuda_dev, bits, N, K):
         assert_close(y.view(np.float16), y64, what="N=%d K=%d B=%d bits=%d" % (N, K, Bt, bits))
 
 
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("N,K", [(200, 1024), (1000, 4096), (9, 256), (24, 512)])
+def test_tensor_copy_tiles_with_row_tail(cuda_dev, bits, N, K):
+    """Rows of 128-byte multiples (K % 256 == 0 at 4 bits, K % 128 == 0 at 8
+    bits) take whole 16-row tiles in one swizzled tensor copy; the last tile
+    here is partial (N % 16 != 0), its missing rows arrive zero-filled."""
+    P, S, B = synth.qmatrix(synth.rng(N, K, bits, 7), N, K, bits)
+    for Bt in (1, 3, 8):
+        x16 = synth.activations(N + K + 10 * Bt, Bt, K)
+        y = run_qgemv(P, S, B, N, K, bits, x16)
+        y64, _ = oracle.qgemv(P, S, B, N, K, bits, x16)
+        assert_close(y.view(np.float16), y64, what="N=%d K=%d B=%d bits=%d" % (N, K, Bt, bits))
+
+
 def test_zero_input_positive_zero(cuda_dev):
     N, K = 64, 256
     P, S, B = synth.dense(3, N, K)
