@@ -250,10 +250,14 @@ qmoe_status moe_group_tokens(const int32_t *idx, int32_t tokens, int32_t top_k,
  * Prefill chunk through the MoE layer as a grouped qGEMM (same formula as
  * moe_expert_qmlp, row by row):
  *   y[t] = shared(x[t]) + sum_j weights[t][j] * expert_{idx[t][j]}(x[t])
- * x: fp16 [tokens][hidden], tokens 1..128; idx: int32 [tokens][top_k];
+ * x: fp16 [tokens][hidden], 16-byte aligned, tokens 1..128; idx: int32 [tokens][top_k];
  * weights: fp32 [tokens][top_k]; y: fp16 [tokens][hidden].
  * workspace: moe_prefill_workspace_bytes() bytes, 16-byte aligned; no
  * initial contents are required.
+ * Every expert touched by the chunk (and the shared expert) is read from
+ * memory once per call.  Returns QMOE_ERR_UNSUPPORTED when two 16-row
+ * gate+up tiles (2 x 16 x hidden/2 bytes of codes plus scales and biases)
+ * do not fit the kernels' shared-memory ring (hidden > ~12,000).
  * ------------------------------------------------------------------------- */
 size_t moe_prefill_workspace_bytes(const qmoe_moe_layer *L, int32_t tokens, int32_t top_k);
 

@@ -125,6 +125,25 @@ __device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gsrc, uint3
         : "memory");
 }
 
+// 3-D tiled TMA tensor copy global -> this CTA's shared memory (no multicast),
+// completing on `bar`; `tmap` is the address of a __grid_constant__ tensor map
+// kernel parameter.  Coordinates are element indices, innermost first.
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, int c0, int c1,
+                                            int c2, uint64_t *bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)),
+        "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const void *tmap)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
 // --------------------------------------------------- dependent launches --
 // Wait until the preceding kernel of the stream has completed and its memory
 // is visible (no-op when the kernel was not launched as a dependent).
@@ -258,11 +277,13 @@ __host__ __device__ __forceinline__ int xperm(int kind, int i)
 //   xs: x fragments, uint4 [G][2][ncol][4]; columns >= ncol read as zero
 //   xsum: fp32 [G][8] sum of x over each group, per column (bias folding:
 //         sum_k (s q_k + b) x_k = s * sum_k q_k x_k + b * sum_k x_k)
-template <int BITS>
-__device__ __forceinline__ void tile_group(const uint32_t *tile, int stride, const __half *sc,
-                                           const __half *bi, int G, const uint4 *xs,
-                                           const float *xsum, int ncol, int g, int gid, int tig,
-                                           float (&acc)[4])
+//   frag(r): address of this lane's codes of row r (r = gid or gid + 8) in
+//         group g: 8 bytes (words 2tig, 2tig+1 of the group) for 4-bit,
+//         16 bytes (words 4tig..4tig+3) for 8-bit
+template <int BITS, class Frag>
+__device__ __forceinline__ void tile_group_f(Frag frag, const __half *sc, const __half *bi, int G,
+                                             const uint4 *xs, const float *xsum, int ncol, int g,
+                                             int gid, int tig, float (&acc)[4])
 {
     uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
     if (gid < ncol) {
@@ -271,9 +292,8 @@ __device__ __forceinline__ void tile_group(const uint32_t *tile, int stride, con
     }
     float c[4] = {0.f, 0.f, 0.f, 0.f};
     if (BITS == 4) {
-        const uint2 wa = *reinterpret_cast<const uint2 *>(tile + gid * stride + g * 8 + 2 * tig);
-        const uint2 wb =
-            *reinterpret_cast<const uint2 *>(tile + (gid + 8) * stride + g * 8 + 2 * tig);
+        const uint2 wa = *reinterpret_cast<const uint2 *>(frag(gid));
+        const uint2 wb = *reinterpret_cast<const uint2 *>(frag(gid + 8));
         uint32_t pa[8], pb[8];
         dequant4_word(wa.x, pa);
         dequant4_word(wa.y, pa + 4);
@@ -284,9 +304,8 @@ __device__ __forceinline__ void tile_group(const uint32_t *tile, int stride, con
         mma_16816(c, pa[4], pb[4], pa[5], pb[5], x1.x, x1.y);
         mma_16816(c, pa[6], pb[6], pa[7], pb[7], x1.z, x1.w);
     } else {
-        const uint4 wa = *reinterpret_cast<const uint4 *>(tile + gid * stride + g * 16 + 4 * tig);
-        const uint4 wb =
-            *reinterpret_cast<const uint4 *>(tile + (gid + 8) * stride + g * 16 + 4 * tig);
+        const uint4 wa = *reinterpret_cast<const uint4 *>(frag(gid));
+        const uint4 wb = *reinterpret_cast<const uint4 *>(frag(gid + 8));
         uint32_t pa[2], pb[2];
         dequant8_word(wa.x, pa);
         dequant8_word(wb.x, pb);
@@ -310,6 +329,78 @@ __device__ __forceinline__ void tile_group(const uint32_t *tile, int stride, con
     acc[1] = fmaf(s_lo, c[1], fmaf(b_lo, X.y, acc[1]));
     acc[2] = fmaf(s_hi, c[2], fmaf(b_hi, X.x, acc[2]));
     acc[3] = fmaf(s_hi, c[3], fmaf(b_hi, X.y, acc[3]));
+}
+
+// Row-padded tile: row r of the codes at tile + r*stride (words).
+template <int BITS>
+__device__ __forceinline__ void tile_group(const uint32_t *tile, int stride, const __half *sc,
+                                           const __half *bi, int G, const uint4 *xs,
+                                           const float *xsum, int ncol, int g, int gid, int tig,
+                                           float (&acc)[4])
+{
+    const int col = BITS == 4 ? g * 8 + 2 * tig : g * 16 + 4 * tig;
+    tile_group_f<BITS>([&](int r) { return tile + r * stride + col; }, sc, bi, G, xs, xsum, ncol,
+                       g, gid, tig, acc);
+}
+
+// Tile as written by a 3-D TMA tensor copy with 128-byte swizzling (box = 32
+// words x R rows x C chunks of 128 bytes, chunk-major, chunk_bytes = R*128):
+// the 16-byte unit u of row r, chunk c sits at byte
+// c*chunk_bytes + r*128 + 16*(u ^ (r & 7)).  The eight rows of a fragment land
+// on eight different bank quads, so the fragment loads are conflict-free
+// without row padding.
+template <int BITS>
+__device__ __forceinline__ const void *swz128_frag(const unsigned char *tile, int chunk_bytes, int r,
+                                                   int g, int tig)
+{
+    if (BITS == 4) {
+        const int u = (2 * (g & 3) + (tig >> 1)) ^ (r & 7);
+        return tile + (g >> 2) * chunk_bytes + r * 128 + u * 16 + (tig & 1) * 8;
+    }
+    const int u = (4 * (g & 1) + tig) ^ (r & 7);
+    return tile + (g >> 1) * chunk_bytes + r * 128 + u * 16;
+}
+
+// Subnormal-code group product of a 16-row tile (rows gid, gid+8 from wa, wb;
+// x fragments in the order of xperm(kPermS4, .) for 4-bit, xperm(8, .) for
+// 8-bit): returns sum_k q x per C element, scaled by 2^-20 (4-bit) or 2^-24
+// (8-bit).  4-bit: class-0 k-blocks accumulate in c, class-1 in d, combined
+// as 16c + d.
+__device__ __forceinline__ void mma_group_s4(float (&r)[4], uint2 wa, uint2 wb, uint4 x0, uint4 x1)
+{
+    uint32_t pa[8], pb[8];
+    dequant4s_word(wa.x, pa);
+    dequant4s_word(wa.y, pa + 4);
+    dequant4s_word(wb.x, pb);
+    dequant4s_word(wb.y, pb + 4);
+    float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
+    mma_16816(c, pa[0], pb[0], pa[2], pb[2], x0.x, x0.y);
+    mma_16816(d, pa[1], pb[1], pa[3], pb[3], x1.x, x1.y);
+    mma_16816(c, pa[4], pb[4], pa[6], pb[6], x0.z, x0.w);
+    mma_16816(d, pa[5], pb[5], pa[7], pb[7], x1.z, x1.w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        r[i] = fmaf(16.f, c[i], d[i]);
+}
+__device__ __forceinline__ void mma_group_s8(float (&r)[4], uint4 wa, uint4 wb, uint4 x0, uint4 x1)
+{
+    uint32_t pa[8], pb[8];
+    dequant8s_word(wa.x, pa);
+    dequant8s_word(wb.x, pb);
+    dequant8s_word(wa.y, pa + 2);
+    dequant8s_word(wb.y, pb + 2);
+    dequant8s_word(wa.z, pa + 4);
+    dequant8s_word(wb.z, pb + 4);
+    dequant8s_word(wa.w, pa + 6);
+    dequant8s_word(wb.w, pb + 6);
+    float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
+    mma_16816(c, pa[0], pb[0], pa[1], pb[1], x0.x, x0.y);
+    mma_16816(d, pa[2], pb[2], pa[3], pb[3], x0.z, x0.w);
+    mma_16816(c, pa[4], pb[4], pa[5], pb[5], x1.x, x1.y);
+    mma_16816(d, pa[6], pb[6], pa[7], pb[7], x1.z, x1.w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        r[i] = c[i] + d[i];
 }
 
 // Smem row stride (in 32-bit words) for a tile of `cols` inputs so that the
@@ -381,6 +472,60 @@ __device__ __forceinline__ void stage_x(uint4 *xs, float *xsum, int G, int ncol,
         for (int t = tid; t < nvec * G * 8; t += nthreads)
             if ((t & 7) >= ncol)
                 xsum[t] = 0.f;
+}
+
+// Stage x [ncol][G*64] (fp16, global, 16-byte aligned rows) into the fragment
+// layout of tile_group / mma_group_s*, one thread per (column, group): the
+// thread reads the group's 128 bytes with eight 16-byte loads, writes its
+// eight permuted 16-byte fragment slots and the group sum.  KIND as xperm.
+// All `nthreads` threads starting at `tid` take part.  The sum of (column n,
+// group g) goes to xsum[g * sum_stride + n]; with sum_stride 8 (the
+// tile_group layout) columns ncol..7 of the sums are zeroed.
+template <int KIND>
+__device__ __forceinline__ void stage_x_groups(uint4 *xs, float *xsum, int G, int ncol,
+                                               const __half *x, int K, int tid, int nthreads,
+                                               int sum_stride = 8)
+{
+    for (int t = tid; t < ncol * G; t += nthreads) {
+        const int n = t / G, g = t - n * G;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)n * K + (size_t)g * kGroup);
+        uint4 raw[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            raw[i] = __ldg(src + i);
+        const __half *hv = reinterpret_cast<const __half *>(raw);
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float2 f = __half22float2(reinterpret_cast<const __half2 *>(raw)[i]);
+            sum += f.x + f.y;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int tig = 0; tig < 4; ++tig) {
+                uint32_t w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const __half lo = hv[16 * tig + xperm(KIND, 8 * h + 2 * i)];
+                    const __half hi = hv[16 * tig + xperm(KIND, 8 * h + 2 * i + 1)];
+                    w[i] = h2_as_u32(__halves2half2(lo, hi));
+                }
+                xs[((g * 2 + h) * ncol + n) * 4 + tig] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        xsum[g * sum_stride + n] = sum;
+    }
+    if (sum_stride == 8)
+        for (int t = tid; t < G * 8; t += nthreads)
+            if ((t & 7) >= ncol)
+                xsum[t] = 0.f;
+}
+
+// Position i (0..15) of the x order xperm(kPermS4, .) that holds input p of a
+// 16-input block: the inverse permutation of xperm_s4.
+__host__ __device__ __forceinline__ int xperm_s4_inv(int p)
+{
+    return ((p & 1) << 3) | (((p >> 3) & 1) << 2) | (((p >> 1) & 1) << 1) | ((p >> 2) & 1);
 }
 
 }  // namespace qmoe

@@ -2,6 +2,7 @@
 // the kernel translation units.  Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -27,6 +28,14 @@ struct QgemvArgs {
     int32_t *status;
 };
 cudaError_t launch_qgemv(const QgemvArgs &a, const LaunchCfg &c);
+
+// Tensor map over the 4/8-bit codes of a row-major [rows][Kw words] matrix
+// (Kw % 32 == 0) as a 3-D tensor [Kw/32 chunks][rows][32 words]: one copy
+// brings `box_rows` whole rows, 128-byte swizzled (16-byte unit u of row r,
+// chunk c at byte c*box_rows*128 + r*128 + 16*(u ^ (r & 7)) of a 1024-byte
+// aligned destination).  False when the driver entry point is unavailable
+// or refuses the shape.
+bool encode_codes_map(CUtensorMap *m, const uint32_t *packed, long rows, int Kw, int box_rows);
 
 // ------------------------------------------------------------------ router --
 struct RouterArgs {
@@ -107,12 +116,12 @@ struct PrefillWorkspace {
     int32_t *offsets;   // [E + 1]
     int32_t *pairs;     // [T * top_k]
     int32_t *inv;       // [T * top_k] position of each (token, slot) pair
-    int32_t *tile_off;  // [E + 2] first 8-token tile of each slot (slot E: shared expert)
-    int32_t *unit_ctr;  // [2] work counters of the gate/up and down kernels
-    uint4 *xfrag;       // [T][H/64][2][4] x in mma fragment order
-    float *xsum;        // [T][H/64][8] group sums of x (column 0)
-    uint4 *hfrag;       // [T * top_k + T][I/64][2][2][4] h (hi, lo) fragments per position
-    float *hsum;        // [T * top_k + T][I/64][2] group sums of h hi / lo
+    int32_t *tiles;     // 8-position token tiles of all slots: (slot << 4) | tile
+    int32_t *unit_ctr;  // [4] gate/up and down work counters, number of tiles
+    uint4 *xfrag;       // per position: x of its token in mma fragment order (+64 B pad)
+    float *xsum;        // per position: group sums of x
+    uint4 *hfrag;       // per position: h (hi, lo) fragments (+64 B pad)
+    float *hsum;        // per position: group sums of h hi / lo
     float *r;           // [T * top_k + T][H] unweighted expert outputs per position
 };
 size_t prefill_workspace_layout(int E, int hidden, int inter, int T, int top_k, void *base,
@@ -137,6 +146,8 @@ struct PrefillArgs {
     int32_t *status;
 };
 cudaError_t launch_prefill(const PrefillArgs &a, const LaunchCfg &c);
+// the shared-memory ring of the grouped kernels holds at least two units
+bool prefill_shape_supported(int hidden, int inter);
 
 // ------------------------------------------------------------ pack helpers --
 cudaError_t launch_pack(const uint8_t *codes, int rows, int cols, int bits, uint32_t *packed,

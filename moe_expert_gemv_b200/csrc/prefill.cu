@@ -9,21 +9,33 @@
 //   y[t] = shared(x_t) + sum_j wt[t][j] * down_e( silu(gate_e x_t) * (up_e x_t) ).
 //
 // Pipeline (all launches chained with programmatic dependent launch):
-//   1. group   : (token, slot) pairs listed per expert (misc.cu);
-//   2. prep    : x of every token in mma fragment order + group sums; the
-//                position of every pair; per-expert 8-token tile offsets;
-//   3. gate/up : one warp per (expert, 8 gate + 8 up rows, 8 tokens): the
-//                expert's weight tile is read from memory by the warps of its
-//                token tiles (from L2 after the first), codes enter the
-//                tensor cores as exact fp16 integers, per-group fp32 scale;
-//                SwiGLU in registers; h written as fp16 (hi, lo) fragments;
+//   1. group   : (token, slot) pairs listed per expert (misc.cu); a pair's
+//                index in that list is its position; the shared expert's
+//                positions follow, one per token;
+//   2. prep    : x of every position in mma fragment order (gathered, so
+//                that the 8 positions of a token tile are contiguous) + group
+//                sums; the list of 8-position token tiles of every slot;
+//   3. gate/up : persistent CTAs; a unit is (token tile, 64 gate + 64 up
+//                rows).  A producer warp takes units from a global queue and
+//                streams the tile's x (one copy) and the unit's weights in
+//                8+8-row sub-blocks into shared-memory rings; each consumer
+//                warp owns one sub-block: codes enter the tensor cores as
+//                exact fp16 values (subnormal code bits), per-group fp32
+//                scale, SwiGLU in registers, h written as fp16 (hi, lo)
+//                fragments per position;
 //   4. hsum    : per-group sums of h (bias folding of the down projection);
-//   5. down    : one warp per (expert, 16 rows, 8 tokens), hi and lo passes;
-//                unweighted expert outputs r[pair position][H] in fp32;
+//   5. down    : the same scheme, a unit is (token tile, 256 rows of the
+//                hidden size) in 32-row sub-blocks, h hi and lo passes
+//                sharing the dequantised codes; unweighted expert outputs
+//                r[position][H] in fp32;
 //   6. combine : y[t] = r_shared[t] + sum_j wt[t][j] r[pos(t, j)], in slot
 //                order, rounded once to fp16.
-// Units of steps 3 and 5 are taken from an atomic counter (heavy experts have
-// many token tiles, light ones one), so warps stay busy whatever the skew.
+// Every operand of the inner loops is in shared memory.  A light expert (at
+// most 8 tokens: most of them under skewed routing) is streamed from HBM
+// exactly once; a heavy one once per token tile, the repeats hitting L2.
+#include <cuda.h>
+#include <string.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -31,11 +43,28 @@ namespace qmoe {
 
 namespace {
 
-constexpr int PF_WARPS = 8;   // warps per CTA in the unit kernels
+constexpr int PF_CW = 8;                      // consumer warps = sub-blocks per unit
+constexpr int PF_THREADS = (PF_CW + 1) * 32;  // + one producer warp
+constexpr int PF_MAX_STAGES = 12;
+constexpr int TILE_T = 8;                     // positions per token tile
+constexpr int GU_ROWS = 8;                    // gate rows (and the same up rows) per sub-block
+constexpr int DN_ROWS = 32;                   // down rows per sub-block
+
+// how a weight tile reaches shared memory
+enum TileMode {
+    TILE_CONTIG = 1,   // rows already at a conflict-free stride: one 1-D bulk copy
+    TILE_SWZ = 2,      // rows of 128-byte multiples: one swizzled 3-D tensor copy
+    TILE_ROWS = 3,     // otherwise: one bulk copy per row into padded rows
+};
 
 struct PfDims {
     int E, H, I, T, K;        // K = top_k
     int GH, GI, npos;         // npos = T*K + T (shared expert positions last)
+    int xg_stride;            // uint4 per position of the gathered x fragments (+64 B pad)
+    int xs_stride;            // floats per position of the x group sums
+    int hf_stride;            // uint4 per position of the h fragments (+64 B pad)
+    int hs_stride;            // floats per position of the h group sums
+    int max_tiles;
 };
 
 __host__ __device__ inline PfDims pf_dims(int E, int H, int I, int T, int K)
@@ -49,6 +78,11 @@ __host__ __device__ inline PfDims pf_dims(int E, int H, int I, int T, int K)
     d.GH = H / kGroup;
     d.GI = I / kGroup;
     d.npos = T * K + T;
+    d.xg_stride = d.GH * 8 + 4;
+    d.xs_stride = (d.GH + 3) & ~3;
+    d.hf_stride = d.GI * 16 + 4;
+    d.hs_stride = (d.GI * 2 + 3) & ~3;
+    d.max_tiles = (T * K + T) / TILE_T + E + 2;
     return d;
 }
 
@@ -68,143 +102,433 @@ __device__ __forceinline__ int pos_token(const PrefillArgs &a, int p)
     return p < tk ? a.ws.pairs[p] / a.top_k : p - tk;
 }
 
+// ------------------------------------------------------------- stage layout --
+struct PfStage {
+    int rows;           // rows per matrix tile
+    int S;              // shared-memory row stride of a tile (words)
+    int mode;           // TileMode
+    size_t codes;       // bytes of one matrix tile's codes region (1024-aligned)
+    size_t sb;          // bytes of one scales (or biases) array of a tile
+    size_t bytes;       // one ring stage, 1024-aligned
+};
+
+__host__ __device__ inline PfStage pf_stage(int rows, int Kw, int mode, int S, int G, int nmat)
+{
+    PfStage st;
+    st.rows = rows;
+    st.S = S;
+    st.mode = mode;
+    st.codes = ((size_t)rows * (mode == TILE_ROWS ? S : Kw) * 4 + 1023) & ~(size_t)1023;
+    st.sb = (size_t)rows * G * 2;
+    st.bytes = ((size_t)nmat * (st.codes + 2 * st.sb) + 1023) & ~(size_t)1023;
+    return st;
+}
+
+// barriers: ring full/empty, activation-buffer full/empty (2 each)
+constexpr int PF_BARS = 2 * PF_MAX_STAGES + 4;
+
+struct PfLayout {
+    size_t bar_off, unit_off, act_off, act_bytes, stage_off, total;
+};
+
+// offsets from a 1024-byte aligned base; total includes the alignment slack
+__host__ __device__ inline PfLayout pf_layout(const PfStage &st, size_t act_bytes, int NS)
+{
+    PfLayout L;
+    size_t off = 0;
+    L.bar_off = off;
+    off += PF_BARS * 8;
+    L.unit_off = off;
+    off += (4 + PF_MAX_STAGES) * 4;   // unit id per activation buffer, abort word, pad,
+                                       // then the sequence number each ring slot holds
+    off = (off + 1023) & ~(size_t)1023;
+    L.act_off = off;
+    L.act_bytes = (act_bytes + 1023) & ~(size_t)1023;
+    off += 2 * L.act_bytes;
+    L.stage_off = off;
+    off += (size_t)NS * st.bytes;
+    L.total = off + 1024;
+    return L;
+}
+
+__host__ __device__ inline size_t gu_act_bytes(const PfDims &d)
+{
+    return (size_t)TILE_T * d.xg_stride * 16 + (size_t)TILE_T * d.xs_stride * 4;
+}
+__host__ __device__ inline size_t dn_act_bytes(const PfDims &d)
+{
+    return (size_t)TILE_T * d.hf_stride * 16 + (size_t)TILE_T * d.hs_stride * 4;
+}
+
+// this lane's 8 code bytes of row r, group g (4-bit, fragment words 2tig, 2tig+1)
+__device__ __forceinline__ uint2 tile_frag(const unsigned char *tile, const PfStage &st, int r,
+                                           int g, int tig)
+{
+    const void *p;
+    if (st.mode == TILE_SWZ)
+        p = swz128_frag<4>(tile, st.rows * 128, r, g, tig);
+    else
+        p = tile + ((size_t)r * st.S + g * 8 + 2 * tig) * 4;
+    return *reinterpret_cast<const uint2 *>(p);
+}
+
+// issue the copies of one matrix tile (rows [row0, row0 + st.rows) of a
+// row-major [.][Kw] code array) into `dst`
+__device__ __forceinline__ void issue_tile(unsigned char *dst, const PfStage &st,
+                                           const CUtensorMap *map, const uint32_t *packed,
+                                           size_t row0, int Kw, uint64_t *bar, uint64_t pol)
+{
+    const uint32_t row_bytes = (uint32_t)Kw * 4;
+    if (st.mode == TILE_SWZ)
+        tma_load_3d(dst, map, 0, (int)row0, 0, bar, pol);
+    else if (st.mode == TILE_CONTIG)
+        bulk_g2s(dst, packed + row0 * Kw, row_bytes * st.rows, bar, pol);
+    else
+        for (int r = 0; r < st.rows; ++r)
+            bulk_g2s(dst + (size_t)r * st.S * 4, packed + (row0 + r) * Kw, row_bytes, bar, pol);
+}
+
+// Subnormal-code product of rows (gid, gid+8) with two activation columns
+// sets (the hi and lo fp16 parts of h) summed: 2^-20 * sum_k q (hi + lo).
+__device__ __forceinline__ void mma_group_s4_hilo(float (&r)[4], uint2 wa, uint2 wb, uint4 h0,
+                                                  uint4 h1, uint4 l0, uint4 l1)
+{
+    uint32_t pa[8], pb[8];
+    dequant4s_word(wa.x, pa);
+    dequant4s_word(wa.y, pa + 4);
+    dequant4s_word(wb.x, pb);
+    dequant4s_word(wb.y, pb + 4);
+    float c[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
+    mma_16816(c, pa[0], pb[0], pa[2], pb[2], h0.x, h0.y);
+    mma_16816(e, pa[1], pb[1], pa[3], pb[3], h1.x, h1.y);
+    mma_16816(c, pa[4], pb[4], pa[6], pb[6], h0.z, h0.w);
+    mma_16816(e, pa[5], pb[5], pa[7], pb[7], h1.z, h1.w);
+    mma_16816(c, pa[0], pb[0], pa[2], pb[2], l0.x, l0.y);
+    mma_16816(e, pa[1], pb[1], pa[3], pb[3], l1.x, l1.y);
+    mma_16816(c, pa[4], pb[4], pa[6], pb[6], l0.z, l0.w);
+    mma_16816(e, pa[5], pb[5], pa[7], pb[7], l1.z, l1.w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        r[i] = fmaf(16.f, c[i], e[i]);
+}
+
+// h of intermediate index kidx at position pos from its gate and up values,
+// stored as fp16 (hi, lo) in the fragment order of the down projection:
+// [g][k half][column: 0 = hi, 1 = lo][tig][8], k order xperm(kPermS4, .)
+__device__ __forceinline__ void write_h(const PrefillArgs &a, const PfDims &d, int pos, int kidx,
+                                        float gv, float uv)
+{
+    const float h = gv / (1.f + expf(-gv)) * uv;
+    const __half hh = __float2half_rn(h);
+    const __half hl = __float2half_rn(h - __half2float(hh));
+    __half *hf = reinterpret_cast<__half *>(a.ws.hfrag + (size_t)pos * d.hf_stride);
+    const int gg = kidx >> 6, kk = kidx & 63, tg = kk >> 4;
+    const int i = xperm_s4_inv(kk & 15);
+    const int base = (((gg * 2 + (i >> 3)) * 2) * 4 + tg) * 8 + (i & 7);
+    hf[base] = hh;
+    hf[base + 4 * 8] = hl;   // column 1 is 4 uint4 (32 halves) further
+}
+
+// bounded wait that gives up at once after another thread of the CTA gave up
+__device__ __forceinline__ bool pf_wait(uint64_t *bar, uint32_t parity, int32_t *status,
+                                        volatile int *abort_word)
+{
+    if (*abort_word)
+        return false;
+    if (mbar_wait(bar, parity, status))
+        return true;
+    *abort_word = 1;
+    return false;
+}
+
+// Wait until ring slot `seq_word` has been armed for ring sequence k.  A
+// consumer warp may run up to two units ahead of the slowest one, i.e. more
+// than a ring's length, while the slot still holds sequence k - NS; a parity
+// wait on the full barrier would then see the earlier phase as complete.
+__device__ __forceinline__ bool pf_wait_seq(const volatile int *seq_word, int k, int32_t *status,
+                                            volatile int *abort_word)
+{
+    if (*seq_word == k)
+        return true;
+    const unsigned long long t0 = global_timer_ns();
+    while (*seq_word != k) {
+        if (*abort_word)
+            return false;
+        __nanosleep(32);
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            flag_status(status, QMOE_DEV_TIMEOUT);
+            *abort_word = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
 // ------------------------------------------------------------------ prep --
-// grid: T CTAs of 128 threads.  CTA t: fragments and group sums of x_t;
-// CTA 0 also the per-slot tile offsets, pair positions, unit counters.
+// grid: npos CTAs of 128 threads.  CTA p: x of position p's token, gathered
+// in fragment order, and its group sums; CTA 0 also the token-tile list,
+// the pair positions and the unit counters.
 __global__ void __launch_bounds__(128) prefill_prep_kernel(PrefillArgs a)
 {
     pdl_wait();
     pdl_trigger();
     const PfDims d = pf_dims(a.E, a.H, a.I, a.T, a.top_k);
-    const int t = blockIdx.x;
-    const __half *x = a.x + (size_t)t * d.H;
-    uint4 *xf = a.ws.xfrag + (size_t)t * d.GH * 2 * 4;
-    float *xs = a.ws.xsum + (size_t)t * d.GH * 8;
-    stage_x<4>(xf, xs, d.GH, 1, 1, [&](int, int, int k) { return __half2float(x[k]); },
-               threadIdx.x, 128);
-    if (t == 0) {
+    const int p = blockIdx.x;
+    const int nvalid = a.ws.offsets[d.E];
+    if (p < nvalid || p >= d.T * d.K) {
+        const int tok = pos_token(a, p);
+        stage_x_groups<kPermS4>(a.ws.xfrag + (size_t)p * d.xg_stride,
+                                a.ws.xsum + (size_t)p * d.xs_stride, d.GH, 1,
+                                a.x + (size_t)tok * d.H, d.H, threadIdx.x, 128, 1);
+    }
+    if (p == 0) {
         if (threadIdx.x == 0) {
-            int acc = 0;
+            int n = 0;
             for (int s = 0; s <= d.E; ++s) {
-                a.ws.tile_off[s] = acc;
-                acc += (slot_count(a, s) + 7) / 8;
+                const int nt = (slot_count(a, s) + TILE_T - 1) / TILE_T;
+                for (int t = 0; t < nt; ++t)
+                    a.ws.tiles[n++] = (s << 4) | t;
             }
-            a.ws.tile_off[d.E + 1] = acc;
             a.ws.unit_ctr[0] = 0;
             a.ws.unit_ctr[1] = 0;
+            a.ws.unit_ctr[2] = n;
         }
         // positions of the valid pairs (ids out of range were dropped by the
         // grouping, so only offsets[E] positions hold a pair)
-        const int nvalid = a.ws.offsets[d.E];
-        for (int p = threadIdx.x; p < nvalid; p += blockDim.x)
-            a.ws.inv[a.ws.pairs[p]] = p;
+        for (int q = threadIdx.x; q < nvalid; q += blockDim.x)
+            a.ws.inv[a.ws.pairs[q]] = q;
     }
 }
 
-// slot s of 8-token tile index `tile` (global over slots): binary search
-__device__ __forceinline__ int tile_slot(const PrefillArgs &a, int tile)
+// ------------------------------------------------------ unit kernel frame --
+struct UnitTile {
+    int s, p0, nv;   // slot, first position, valid positions (<= 8)
+};
+
+__device__ __forceinline__ UnitTile unit_tile(const PrefillArgs &a, int i)
 {
-    int lo = 0, hi = a.E;   // tile_off[lo] <= tile < tile_off[hi + 1]
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (a.ws.tile_off[mid] <= tile)
-            lo = mid;
-        else
-            hi = mid - 1;
+    const int tl = a.ws.tiles[i];
+    UnitTile u;
+    u.s = tl >> 4;
+    const int t = tl & 15;
+    u.p0 = slot_offset(a, u.s) + t * TILE_T;
+    u.nv = min(TILE_T, slot_count(a, u.s) - t * TILE_T);
+    return u;
+}
+
+// Producer of both unit kernels.  Unit u = (chunk u / ntiles, tile
+// u % ntiles): tiles of one slot are consecutive, so the CTAs that take them
+// read the slot's weights at about the same time (one HBM read, L2 hits).
+// For each unit: the tile's activations into activation buffer (q & 1), then
+// nsub(chunk) weight sub-blocks into the ring.  A unit id of -1 in an
+// activation buffer tells the consumers that the queue is empty.
+template <class ActCopy, class SubCopy>
+__device__ __forceinline__ void unit_producer(const PrefillArgs &a, int *ctr, int nunits,
+                                              int ntiles, int nsub_total, int NS,
+                                              const PfStage &st, const PfLayout &L,
+                                              unsigned char *smem, uint64_t *full,
+                                              uint64_t *empty, uint64_t *afull, uint64_t *aempty,
+                                              int *s_unit, volatile int *abort_word,
+                                              ActCopy act_copy, SubCopy sub_copy)
+{
+    volatile int *s_seq = s_unit + 4;
+    int last_use[PF_MAX_STAGES], act_last[2] = {-1, -1};
+    for (int s = 0; s < PF_MAX_STAGES; ++s)
+        last_use[s] = -1;
+    int k = 0;
+    for (int q = 0;; ++q) {
+        const int b = q & 1;
+        if (q >= 2 && !pf_wait(&aempty[b], ((q >> 1) - 1) & 1, a.status, abort_word))
+            break;
+        act_last[b] = -1;   // the buffer's previous copies were consumed
+        const int u = atomicAdd(ctr, 1);
+        if (u >= nunits) {
+            s_unit[b] = -1;
+            mbar_arrive(&afull[b]);
+            break;
+        }
+        s_unit[b] = u;
+        const int c = u / ntiles;
+        const UnitTile ut = unit_tile(a, u - c * ntiles);
+        act_copy(ut, smem + L.act_off + b * L.act_bytes, &afull[b]);
+        act_last[b] = q >> 1;
+        const int nsub = min(PF_CW, nsub_total - c * PF_CW);
+        bool ok = true;
+        for (int j = 0; j < nsub; ++j, ++k) {
+            const int slot = k % NS, use = k / NS;
+            if (use > 0 && !pf_wait(&empty[slot], (use - 1) & 1, a.status, abort_word)) {
+                ok = false;
+                break;
+            }
+            s_seq[slot] = k;   // published by the arrive that arms the barrier
+            sub_copy(ut, c * PF_CW + j, smem + L.stage_off + (size_t)slot * st.bytes, &full[slot]);
+            last_use[slot] = use;
+        }
+        if (!ok)
+            break;
     }
-    return lo;
+    // no copy may still be landing when the CTA exits
+    for (int s = 0; s < NS; ++s)
+        if (last_use[s] >= 0)
+            mbar_wait(&full[s], last_use[s] & 1, a.status);
+    for (int b = 0; b < 2; ++b)
+        if (act_last[b] >= 0)
+            mbar_wait(&afull[b], act_last[b] & 1, a.status);
+}
+
+__device__ __forceinline__ void init_bars(uint64_t *full, uint64_t *empty, uint64_t *afull,
+                                          uint64_t *aempty, int NS, int *s_unit)
+{
+    for (int s = 0; s < NS; ++s) {
+        mbar_init(&full[s], 1);
+        mbar_init(&empty[s], 1);   // one consumer warp per sub-block
+    }
+    for (int b = 0; b < 2; ++b) {
+        mbar_init(&afull[b], 1);
+        mbar_init(&aempty[b], PF_CW);
+    }
+    s_unit[2] = 0;   // abort word
+    for (int s = 0; s < PF_MAX_STAGES; ++s)
+        s_unit[4 + s] = -1;
+    mbar_init_fence();
 }
 
 // ------------------------------------------------------------- gate / up --
-// unit = (token tile, octet o): 8 gate rows o*8.. and the same 8 up rows of
-// the tile's expert, over the tile's <= 8 tokens.
-__global__ void __launch_bounds__(PF_WARPS * 32) prefill_gateup_kernel(PrefillArgs a)
+// Sub-block o of a slot: gate rows 8o .. 8o+7 and the same up rows.  mma A
+// rows (gid, gid+8) = (gate row, up row), so each C fragment holds a gate
+// and an up value of one intermediate index, tokens 2tig and 2tig+1.
+__global__ void __launch_bounds__(PF_THREADS, 1)
+    prefill_gateup_kernel(PrefillArgs a, PfStage st, int NS,
+                          const __grid_constant__ CUtensorMap gate_map,
+                          const __grid_constant__ CUtensorMap up_map,
+                          const __grid_constant__ CUtensorMap sh_gate_map,
+                          const __grid_constant__ CUtensorMap sh_up_map)
 {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const PfDims d = pf_dims(a.E, a.H, a.I, a.T, a.top_k);
+    const PfLayout L = pf_layout(st, gu_act_bytes(d), NS);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bar_off);
+    uint64_t *empty = full + PF_MAX_STAGES, *afull = empty + PF_MAX_STAGES, *aempty = afull + 2;
+    int *s_unit = reinterpret_cast<int *>(smem + L.unit_off);
+    volatile int *abort_word = s_unit + 2;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0)
+        init_bars(full, empty, afull, aempty, NS, s_unit);
+    __syncthreads();
     pdl_wait();
     pdl_trigger();
-    const PfDims d = pf_dims(a.E, a.H, a.I, a.T, a.top_k);
-    const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
-    const int octs = d.I / 8;
-    const int ntiles = a.ws.tile_off[d.E + 1];
-    const int nunits = ntiles * octs;
-    const int Hw = d.H / 8;
-    while (true) {
-        int u = 0;
-        if (lane == 0)
-            u = atomicAdd(a.ws.unit_ctr + 0, 1);
-        u = __shfl_sync(0xffffffffu, u, 0);
-        if (u >= nunits)
+    const int ntiles = a.ws.unit_ctr[2];
+    const int nsub_total = d.I / GU_ROWS;
+    const int nunits = ntiles * ((nsub_total + PF_CW - 1) / PF_CW);
+    const int Kw = d.H / 8;
+    const size_t sb_row = (size_t)d.GH;   // fp16 scales per row
+
+    if (warp == PF_CW) {
+        if (lane == 0) {
+            if (st.mode == TILE_SWZ) {
+                prefetch_tensormap(&gate_map);
+                prefetch_tensormap(&up_map);
+                prefetch_tensormap(&sh_gate_map);
+                prefetch_tensormap(&sh_up_map);
+            }
+            const uint64_t pol = l2_evict_first_policy();
+            const uint32_t sub_bytes = (uint32_t)(2 * GU_ROWS * Kw * 4 + 4 * st.sb);
+            unit_producer(
+                a, a.ws.unit_ctr + 0, nunits, ntiles, nsub_total, NS, st, L, smem, full, empty,
+                afull, aempty, s_unit, abort_word,
+                [&](const UnitTile &ut, unsigned char *dst, uint64_t *bar) {
+                    const uint32_t fb = (uint32_t)ut.nv * d.xg_stride * 16;
+                    const uint32_t sbb = (uint32_t)ut.nv * d.xs_stride * 4;
+                    mbar_arrive_expect_tx(bar, fb + sbb);
+                    bulk_g2s(dst, a.ws.xfrag + (size_t)ut.p0 * d.xg_stride, fb, bar, pol);
+                    bulk_g2s(dst + (size_t)TILE_T * d.xg_stride * 16,
+                             a.ws.xsum + (size_t)ut.p0 * d.xs_stride, sbb, bar, pol);
+                },
+                [&](const UnitTile &ut, int o, unsigned char *dst, uint64_t *bar) {
+                    const bool sh = ut.s >= d.E;
+                    const QMat gm = sh ? a.sh_gate : a.gate, um = sh ? a.sh_up : a.up;
+                    const size_t row0 = (size_t)(sh ? 0 : ut.s) * d.I + (size_t)o * GU_ROWS;
+                    mbar_arrive_expect_tx(bar, sub_bytes);
+                    issue_tile(dst, st, sh ? &sh_gate_map : &gate_map, gm.packed, row0, Kw, bar,
+                               pol);
+                    issue_tile(dst + st.codes, st, sh ? &sh_up_map : &up_map, um.packed, row0, Kw,
+                               bar, pol);
+                    unsigned char *sb = dst + 2 * st.codes;
+                    bulk_g2s(sb, gm.scales + row0 * sb_row, (uint32_t)st.sb, bar, pol);
+                    bulk_g2s(sb + st.sb, gm.biases + row0 * sb_row, (uint32_t)st.sb, bar, pol);
+                    bulk_g2s(sb + 2 * st.sb, um.scales + row0 * sb_row, (uint32_t)st.sb, bar, pol);
+                    bulk_g2s(sb + 3 * st.sb, um.biases + row0 * sb_row, (uint32_t)st.sb, bar, pol);
+                });
+        }
+        return;
+    }
+
+    // -------------------- consumers: warp j takes sub-block j of every unit
+    const int gid = lane >> 2, tig = lane & 3;
+    int k = 0;
+    for (int q = 0;; ++q) {
+        const int b = q & 1;
+        if (!pf_wait(&afull[b], (q >> 1) & 1, a.status, abort_word))
             break;
-        // consecutive units share the weight tile: octet-major over tiles of a slot
-        const int s_tile = u / octs, o = u % octs;
-        const int s = tile_slot(a, s_tile);
-        const int c = s_tile - a.ws.tile_off[s];        // token tile within the slot
-        const int cnt = slot_count(a, s), off = slot_offset(a, s);
-        const QMat gm = s < d.E ? a.gate : a.sh_gate;
-        const QMat um = s < d.E ? a.up : a.sh_up;
-        const size_t r0 = (size_t)(s < d.E ? s : 0) * d.I + (size_t)o * 8 + gid;
-        const uint32_t *ga = gm.packed + r0 * Hw + 2 * tig;
-        const uint32_t *ua = um.packed + r0 * Hw + 2 * tig;
-        const __half *gs = gm.scales + r0 * d.GH, *gb = gm.biases + r0 * d.GH;
-        const __half *us = um.scales + r0 * d.GH, *ub = um.biases + r0 * d.GH;
-        // B column n = gid <-> token of position off + c*8 + gid
-        const int pn = c * 8 + gid;
-        const bool nvalid = pn < cnt;
-        const int tok_n = nvalid ? pos_token(a, off + pn) : 0;
-        const uint4 *xf = a.ws.xfrag + (size_t)tok_n * d.GH * 2 * 4;
-        // C columns 2tig, 2tig+1 <-> their tokens (for the x group sums)
-        const int pc0 = c * 8 + 2 * tig, pc1 = pc0 + 1;
-        const float *xs0 = a.ws.xsum + (size_t)(pc0 < cnt ? pos_token(a, off + pc0) : 0) * d.GH * 8;
-        const float *xs1 = a.ws.xsum + (size_t)(pc1 < cnt ? pos_token(a, off + pc1) : 0) * d.GH * 8;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        const int u = s_unit[b];
+        if (u < 0)
+            break;
+        const int c = u / ntiles;
+        const UnitTile ut = unit_tile(a, u - c * ntiles);
+        const int nsub = min(PF_CW, nsub_total - c * PF_CW);
+        const unsigned char *act = smem + L.act_off + b * L.act_bytes;
+        const uint4 *xf = reinterpret_cast<const uint4 *>(act);
+        const float *xsm = reinterpret_cast<const float *>(act + (size_t)TILE_T * d.xg_stride * 16);
+        if (warp < nsub) {
+            const int kk = k + warp, slot = kk % NS;
+            if (pf_wait_seq(s_unit + 4 + slot, kk, a.status, abort_word) &&
+                pf_wait(&full[slot], (kk / NS) & 1, a.status, abort_word)) {
+                const unsigned char *stage = smem + L.stage_off + (size_t)slot * st.bytes;
+                const unsigned char *gt = stage, *utl = stage + st.codes;
+                const __half *gs = reinterpret_cast<const __half *>(stage + 2 * st.codes);
+                const __half *gb = gs + GU_ROWS * d.GH, *us = gb + GU_ROWS * d.GH,
+                             *ub = us + GU_ROWS * d.GH;
+                const bool nvalid = gid < ut.nv;
+                const uint4 *xr = xf + gid * d.xg_stride;
+                const float *xs0 = xsm + (2 * tig) * d.xs_stride;
+                const float *xs1 = xs0 + d.xs_stride;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 2
-        for (int g = 0; g < d.GH; ++g) {
-            const uint2 wa = *reinterpret_cast<const uint2 *>(ga + g * 8);
-            const uint2 wb = *reinterpret_cast<const uint2 *>(ua + g * 8);
-            uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
-            if (nvalid) {
-                x0 = __ldcg(xf + (g * 2 + 0) * 4 + tig);
-                x1 = __ldcg(xf + (g * 2 + 1) * 4 + tig);
-            }
-            uint32_t pa[8], pb[8];
-            dequant4_word(wa.x, pa);
-            dequant4_word(wa.y, pa + 4);
-            dequant4_word(wb.x, pb);
-            dequant4_word(wb.y, pb + 4);
-            float cc[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_16816(cc, pa[0], pb[0], pa[1], pb[1], x0.x, x0.y);
-            mma_16816(cc, pa[2], pb[2], pa[3], pb[3], x0.z, x0.w);
-            mma_16816(cc, pa[4], pb[4], pa[5], pb[5], x1.x, x1.y);
-            mma_16816(cc, pa[6], pb[6], pa[7], pb[7], x1.z, x1.w);
-            const float sg = __half2float(gs[g]), bg = __half2float(gb[g]);
-            const float su = __half2float(us[g]), bu = __half2float(ub[g]);
-            const float X0 = xs0[g * 8], X1 = xs1[g * 8];
-            acc[0] = fmaf(sg, cc[0], fmaf(bg, X0, acc[0]));   // gate row, token col 2tig
-            acc[1] = fmaf(sg, cc[1], fmaf(bg, X1, acc[1]));   // gate row, token col 2tig+1
-            acc[2] = fmaf(su, cc[2], fmaf(bu, X0, acc[2]));   // up row
-            acc[3] = fmaf(su, cc[3], fmaf(bu, X1, acc[3]));
-        }
-        // h for intermediate index o*8 + gid, tokens of columns 2tig, 2tig+1
-        const int kidx = o * 8 + gid;
+                for (int g = 0; g < d.GH; ++g) {
+                    uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
+                    if (nvalid) {
+                        x0 = xr[(g * 2 + 0) * 4 + tig];
+                        x1 = xr[(g * 2 + 1) * 4 + tig];
+                    }
+                    float r[4];
+                    mma_group_s4(r, tile_frag(gt, st, gid, g, tig), tile_frag(utl, st, gid, g, tig),
+                                 x0, x1);
+                    const float X0 = xs0[g], X1 = xs1[g];
+                    const float sg = __half2float(gs[gid * d.GH + g]) * kSub20;
+                    const float bg = __half2float(gb[gid * d.GH + g]);
+                    const float su = __half2float(us[gid * d.GH + g]) * kSub20;
+                    const float bu = __half2float(ub[gid * d.GH + g]);
+                    acc[0] = fmaf(sg, r[0], fmaf(bg, X0, acc[0]));   // gate, token 2tig
+                    acc[1] = fmaf(sg, r[1], fmaf(bg, X1, acc[1]));   // gate, token 2tig+1
+                    acc[2] = fmaf(su, r[2], fmaf(bu, X0, acc[2]));   // up
+                    acc[3] = fmaf(su, r[3], fmaf(bu, X1, acc[3]));
+                }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&empty[slot]);
+                const int kidx = (c * PF_CW + warp) * GU_ROWS + gid;
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int pq = c * 8 + 2 * tig + q;
-            if (pq < cnt) {
-                const float gv = acc[q], uv = acc[2 + q];
-                const float h = gv / (1.f + expf(-gv)) * uv;
-                const __half hh = __float2half_rn(h);
-                const __half hl = __float2half_rn(h - __half2float(hh));
-                __half *hf = reinterpret_cast<__half *>(a.ws.hfrag + (size_t)(off + pq) * d.GI * 2 * 2 * 4);
-                // fragment order of the down projection: [g][hh][col][tig][8],
-                // columns: 0 = hi, 1 = lo
-                const int gg = kidx >> 6, kk = kidx & 63, tg = kk >> 4, p = kk & 15;
-                const int qq = p & 7;
-                const int i = (p & 8) + 2 * (qq & 3) + (qq >> 2);   // inverse of xperm(4, .)
-                const int base = (((gg * 2 + (i >> 3)) * 2) * 4 + tg) * 8 + (i & 7);
-                hf[base] = hh;
-                hf[base + 4 * 8] = hl;   // column 1 is 4 uint4 (32 halves) further
+                for (int qq = 0; qq < 2; ++qq)
+                    if (2 * tig + qq < ut.nv)
+                        write_h(a, d, ut.p0 + 2 * tig + qq, kidx, acc[qq], acc[2 + qq]);
             }
         }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&aempty[b]);
+        k += nsub;
     }
 }
 
@@ -215,108 +539,167 @@ __global__ void __launch_bounds__(256) prefill_hsum_kernel(PrefillArgs a)
     pdl_wait();
     pdl_trigger();
     const PfDims d = pf_dims(a.E, a.H, a.I, a.T, a.top_k);
+    const int nvalid = a.ws.offsets[d.E];
     const int n = d.npos * d.GI * 2;
     for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
-        const int col = t & 1, pg = t >> 1;   // pg = pos * GI + g
-        const uint4 *f = a.ws.hfrag + (size_t)pg * 2 * 2 * 4;
+        const int col = t & 1, pg = t >> 1;
+        const int pos = pg / d.GI, g = pg - pos * d.GI;
+        if (pos >= nvalid && pos < d.T * d.K)
+            continue;   // no pair holds this position
+        const uint4 *f = a.ws.hfrag + (size_t)pos * d.hf_stride + g * 16;
         float s = 0.f;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
             for (int tg = 0; tg < 4; ++tg) {
-                const uint4 w = f[(hh * 2 + col) * 4 + tg];
+                const uint4 w = __ldcg(f + (hh * 2 + col) * 4 + tg);
                 const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float2 v = __half22float2(u32_as_h2(ws[q]));
+                for (int qq = 0; qq < 4; ++qq) {
+                    const float2 v = __half22float2(u32_as_h2(ws[qq]));
                     s += v.x + v.y;
                 }
             }
-        a.ws.hsum[t] = s;
+        a.ws.hsum[(size_t)pos * d.hs_stride + g * 2 + col] = s;
     }
 }
 
 // ------------------------------------------------------------------ down --
-// unit = (token tile, 16-row tile of H): rows of the tile's expert's down
-// projection over the tile's <= 8 positions; two passes (h hi, h lo).
-__global__ void __launch_bounds__(PF_WARPS * 32) prefill_down_kernel(PrefillArgs a)
+// Sub-block o of a slot: down rows 32o .. 32o+31, two 16-row mma tiles.
+__global__ void __launch_bounds__(PF_THREADS, 1)
+    prefill_down_kernel(PrefillArgs a, PfStage st, int NS,
+                        const __grid_constant__ CUtensorMap down_map,
+                        const __grid_constant__ CUtensorMap sh_down_map)
 {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const PfDims d = pf_dims(a.E, a.H, a.I, a.T, a.top_k);
+    const PfLayout L = pf_layout(st, dn_act_bytes(d), NS);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bar_off);
+    uint64_t *empty = full + PF_MAX_STAGES, *afull = empty + PF_MAX_STAGES, *aempty = afull + 2;
+    int *s_unit = reinterpret_cast<int *>(smem + L.unit_off);
+    volatile int *abort_word = s_unit + 2;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0)
+        init_bars(full, empty, afull, aempty, NS, s_unit);
+    __syncthreads();
     pdl_wait();
     pdl_trigger();
-    const PfDims d = pf_dims(a.E, a.H, a.I, a.T, a.top_k);
-    const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
-    const int rtiles = d.H / 16;
-    const int ntiles = a.ws.tile_off[d.E + 1];
-    const int nunits = ntiles * rtiles;
-    const int Iw = d.I / 8;
-    while (true) {
-        int u = 0;
-        if (lane == 0)
-            u = atomicAdd(a.ws.unit_ctr + 1, 1);
-        u = __shfl_sync(0xffffffffu, u, 0);
-        if (u >= nunits)
+    const int ntiles = a.ws.unit_ctr[2];
+    const int nsub_total = d.H / DN_ROWS;
+    const int nunits = ntiles * ((nsub_total + PF_CW - 1) / PF_CW);
+    const int Kw = d.I / 8;
+    const size_t sb_row = (size_t)d.GI;
+
+    if (warp == PF_CW) {
+        if (lane == 0) {
+            if (st.mode == TILE_SWZ) {
+                prefetch_tensormap(&down_map);
+                prefetch_tensormap(&sh_down_map);
+            }
+            const uint64_t pol = l2_evict_first_policy();
+            const uint32_t sub_bytes = (uint32_t)(DN_ROWS * Kw * 4 + 2 * st.sb);
+            unit_producer(
+                a, a.ws.unit_ctr + 1, nunits, ntiles, nsub_total, NS, st, L, smem, full, empty,
+                afull, aempty, s_unit, abort_word,
+                [&](const UnitTile &ut, unsigned char *dst, uint64_t *bar) {
+                    const uint32_t fb = (uint32_t)ut.nv * d.hf_stride * 16;
+                    const uint32_t sbb = (uint32_t)ut.nv * d.hs_stride * 4;
+                    mbar_arrive_expect_tx(bar, fb + sbb);
+                    bulk_g2s(dst, a.ws.hfrag + (size_t)ut.p0 * d.hf_stride, fb, bar, pol);
+                    bulk_g2s(dst + (size_t)TILE_T * d.hf_stride * 16,
+                             a.ws.hsum + (size_t)ut.p0 * d.hs_stride, sbb, bar, pol);
+                },
+                [&](const UnitTile &ut, int o, unsigned char *dst, uint64_t *bar) {
+                    const bool sh = ut.s >= d.E;
+                    const QMat dm = sh ? a.sh_down : a.down;
+                    const size_t row0 = (size_t)(sh ? 0 : ut.s) * d.H + (size_t)o * DN_ROWS;
+                    mbar_arrive_expect_tx(bar, sub_bytes);
+                    issue_tile(dst, st, sh ? &sh_down_map : &down_map, dm.packed, row0, Kw, bar,
+                               pol);
+                    bulk_g2s(dst + st.codes, dm.scales + row0 * sb_row, (uint32_t)st.sb, bar, pol);
+                    bulk_g2s(dst + st.codes + st.sb, dm.biases + row0 * sb_row, (uint32_t)st.sb,
+                             bar, pol);
+                });
+        }
+        return;
+    }
+
+    const int gid = lane >> 2, tig = lane & 3;
+    int k = 0;
+    for (int q = 0;; ++q) {
+        const int b = q & 1;
+        if (!pf_wait(&afull[b], (q >> 1) & 1, a.status, abort_word))
             break;
-        const int s_tile = u / rtiles, rt = u % rtiles;
-        const int s = tile_slot(a, s_tile);
-        const int c = s_tile - a.ws.tile_off[s];
-        const int cnt = slot_count(a, s), off = slot_offset(a, s);
-        const QMat dm = s < d.E ? a.down : a.sh_down;
-        const size_t rl = (size_t)(s < d.E ? s : 0) * d.H + (size_t)rt * 16 + gid;
-        const uint32_t *wa_p = dm.packed + rl * Iw + 2 * tig;
-        const uint32_t *wb_p = wa_p + 8 * Iw;
-        const __half *sl = dm.scales + rl * d.GI, *sh = sl + 8 * d.GI;
-        const __half *bl = dm.biases + rl * d.GI, *bh = bl + 8 * d.GI;
-        const int pn = c * 8 + gid;
-        const bool nvalid = pn < cnt;
-        const uint4 *hf = a.ws.hfrag + (size_t)(off + (nvalid ? pn : 0)) * d.GI * 2 * 2 * 4;
-        const int pc0 = c * 8 + 2 * tig, pc1 = pc0 + 1;
-        const float *hs0 = a.ws.hsum + (size_t)(off + (pc0 < cnt ? pc0 : 0)) * d.GI * 2;
-        const float *hs1 = a.ws.hsum + (size_t)(off + (pc1 < cnt ? pc1 : 0)) * d.GI * 2;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
-        for (int g = 0; g < d.GI; ++g) {
-            const uint2 wa = *reinterpret_cast<const uint2 *>(wa_p + g * 8);
-            const uint2 wb = *reinterpret_cast<const uint2 *>(wb_p + g * 8);
-            uint4 h0 = make_uint4(0, 0, 0, 0), h1 = h0, l0 = h0, l1 = h0;
-            if (nvalid) {
-                h0 = __ldcg(hf + ((g * 2 + 0) * 2 + 0) * 4 + tig);
-                h1 = __ldcg(hf + ((g * 2 + 1) * 2 + 0) * 4 + tig);
-                l0 = __ldcg(hf + ((g * 2 + 0) * 2 + 1) * 4 + tig);
-                l1 = __ldcg(hf + ((g * 2 + 1) * 2 + 1) * 4 + tig);
-            }
-            uint32_t pa[8], pb[8];
-            dequant4_word(wa.x, pa);
-            dequant4_word(wa.y, pa + 4);
-            dequant4_word(wb.x, pb);
-            dequant4_word(wb.y, pb + 4);
-            float cc[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_16816(cc, pa[0], pb[0], pa[1], pb[1], h0.x, h0.y);
-            mma_16816(cc, pa[2], pb[2], pa[3], pb[3], h0.z, h0.w);
-            mma_16816(cc, pa[4], pb[4], pa[5], pb[5], h1.x, h1.y);
-            mma_16816(cc, pa[6], pb[6], pa[7], pb[7], h1.z, h1.w);
-            mma_16816(cc, pa[0], pb[0], pa[1], pb[1], l0.x, l0.y);
-            mma_16816(cc, pa[2], pb[2], pa[3], pb[3], l0.z, l0.w);
-            mma_16816(cc, pa[4], pb[4], pa[5], pb[5], l1.x, l1.y);
-            mma_16816(cc, pa[6], pb[6], pa[7], pb[7], l1.z, l1.w);
-            const float s_l = __half2float(sl[g]), b_l = __half2float(bl[g]);
-            const float s_h = __half2float(sh[g]), b_h = __half2float(bh[g]);
-            const float X0 = __ldcg(hs0 + g * 2) + __ldcg(hs0 + g * 2 + 1);
-            const float X1 = __ldcg(hs1 + g * 2) + __ldcg(hs1 + g * 2 + 1);
-            acc[0] = fmaf(s_l, cc[0], fmaf(b_l, X0, acc[0]));
-            acc[1] = fmaf(s_l, cc[1], fmaf(b_l, X1, acc[1]));
-            acc[2] = fmaf(s_h, cc[2], fmaf(b_h, X0, acc[2]));
-            acc[3] = fmaf(s_h, cc[3], fmaf(b_h, X1, acc[3]));
-        }
-        const int row = rt * 16 + gid;
+        const int u = s_unit[b];
+        if (u < 0)
+            break;
+        const int c = u / ntiles;
+        const UnitTile ut = unit_tile(a, u - c * ntiles);
+        const int nsub = min(PF_CW, nsub_total - c * PF_CW);
+        const unsigned char *act = smem + L.act_off + b * L.act_bytes;
+        const uint4 *hb = reinterpret_cast<const uint4 *>(act);
+        const float *hsm = reinterpret_cast<const float *>(act + (size_t)TILE_T * d.hf_stride * 16);
+        if (warp < nsub) {
+            const int kk = k + warp, slot = kk % NS;
+            if (pf_wait_seq(s_unit + 4 + slot, kk, a.status, abort_word) &&
+                pf_wait(&full[slot], (kk / NS) & 1, a.status, abort_word)) {
+                const unsigned char *wt = smem + L.stage_off + (size_t)slot * st.bytes;
+                const __half *sc = reinterpret_cast<const __half *>(wt + st.codes);
+                const __half *bi = sc + DN_ROWS * d.GI;
+                const bool nvalid = gid < ut.nv;
+                const uint4 *hr = hb + gid * d.hf_stride;
+                const float *hs0 = hsm + (2 * tig) * d.hs_stride;
+                const float *hs1 = hs0 + d.hs_stride;
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                for (int g = 0; g < d.GI; ++g) {
+                    uint4 h0 = make_uint4(0, 0, 0, 0), h1 = h0, l0 = h0, l1 = h0;
+                    if (nvalid) {
+                        h0 = hr[((g * 2 + 0) * 2 + 0) * 4 + tig];
+                        h1 = hr[((g * 2 + 1) * 2 + 0) * 4 + tig];
+                        l0 = hr[((g * 2 + 0) * 2 + 1) * 4 + tig];
+                        l1 = hr[((g * 2 + 1) * 2 + 1) * 4 + tig];
+                    }
+                    const float X0 = hs0[g * 2] + hs0[g * 2 + 1];
+                    const float X1 = hs1[g * 2] + hs1[g * 2 + 1];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int pq = c * 8 + 2 * tig + q;
-            if (pq < cnt) {
-                float *r = a.ws.r + (size_t)(off + pq) * d.H;
-                r[row] = acc[q];
-                r[row + 8] = acc[2 + q];
+                    for (int half = 0; half < 2; ++half) {
+                        const int ra = half * 16 + gid, rb = ra + 8;
+                        float r[4];
+                        mma_group_s4_hilo(r, tile_frag(wt, st, ra, g, tig),
+                                          tile_frag(wt, st, rb, g, tig), h0, h1, l0, l1);
+                        const float sa = __half2float(sc[ra * d.GI + g]) * kSub20;
+                        const float ba = __half2float(bi[ra * d.GI + g]);
+                        const float sb = __half2float(sc[rb * d.GI + g]) * kSub20;
+                        const float bb = __half2float(bi[rb * d.GI + g]);
+                        acc[4 * half + 0] = fmaf(sa, r[0], fmaf(ba, X0, acc[4 * half + 0]));
+                        acc[4 * half + 1] = fmaf(sa, r[1], fmaf(ba, X1, acc[4 * half + 1]));
+                        acc[4 * half + 2] = fmaf(sb, r[2], fmaf(bb, X0, acc[4 * half + 2]));
+                        acc[4 * half + 3] = fmaf(sb, r[3], fmaf(bb, X1, acc[4 * half + 3]));
+                    }
+                }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&empty[slot]);
+                const int row0 = (c * PF_CW + warp) * DN_ROWS + gid;
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    const int pq = 2 * tig + qq;
+                    if (pq < ut.nv) {
+                        float *r = a.ws.r + (size_t)(ut.p0 + pq) * d.H + row0;
+                        r[0] = acc[qq];
+                        r[8] = acc[2 + qq];
+                        r[16] = acc[4 + qq];
+                        r[24] = acc[6 + qq];
+                    }
+                }
             }
         }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&aempty[b]);
+        k += nsub;
     }
 }
 
@@ -341,6 +724,28 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(PrefillArgs a)
     }
 }
 
+// tile mode and stride for rows of K 4-bit codes; `map_ok`: tensor maps encoded
+PfStage choose_stage(int rows, int K, int nmat, bool map_ok)
+{
+    const int Kw = K / 8, G = K / kGroup;
+    const int m = Kw & 31;
+    if (m == 8 || m == 24)
+        return pf_stage(rows, Kw, TILE_CONTIG, Kw, G, nmat);
+    if (m == 0 && map_ok)
+        return pf_stage(rows, Kw, TILE_SWZ, Kw, G, nmat);
+    return pf_stage(rows, Kw, TILE_ROWS, tile_stride_words(K, 4), G, nmat);
+}
+
+int stages_for(const PfStage &st, size_t act_bytes)
+{
+    const size_t budget = 227 * 1024;
+    const PfLayout L0 = pf_layout(st, act_bytes, 0);
+    if (L0.total + 2 * st.bytes > budget)
+        return 0;
+    const int NS = (int)((budget - L0.total) / st.bytes);
+    return NS > PF_MAX_STAGES ? PF_MAX_STAGES : NS;
+}
+
 }  // namespace
 
 size_t prefill_workspace_layout(int E, int H, int I, int T, int top_k, void *base,
@@ -357,12 +762,12 @@ size_t prefill_workspace_layout(int E, int H, int I, int T, int top_k, void *bas
     const size_t offsets_off = take((size_t)(E + 1) * 4);
     const size_t pairs_off = take((size_t)T * top_k * 4);
     const size_t inv_off = take((size_t)T * top_k * 4);
-    const size_t tile_off = take((size_t)(E + 2) * 4);
-    const size_t ctr_off = take(2 * 4);
-    const size_t xfrag_off = take((size_t)T * d.GH * 2 * 4 * 16);
-    const size_t xsum_off = take((size_t)T * d.GH * 8 * 4);
-    const size_t hfrag_off = take((size_t)d.npos * d.GI * 2 * 2 * 4 * 16);
-    const size_t hsum_off = take((size_t)d.npos * d.GI * 2 * 4);
+    const size_t tiles_off = take((size_t)d.max_tiles * 4);
+    const size_t ctr_off = take(4 * 4);
+    const size_t xfrag_off = take((size_t)d.npos * d.xg_stride * 16);
+    const size_t xsum_off = take((size_t)d.npos * d.xs_stride * 4);
+    const size_t hfrag_off = take((size_t)d.npos * d.hf_stride * 16);
+    const size_t hsum_off = take((size_t)d.npos * d.hs_stride * 4);
     const size_t r_off = take((size_t)d.npos * H * 4);
     if (base && ws) {
         unsigned char *b = static_cast<unsigned char *>(base);
@@ -370,7 +775,7 @@ size_t prefill_workspace_layout(int E, int H, int I, int T, int top_k, void *bas
         ws->offsets = reinterpret_cast<int32_t *>(b + offsets_off);
         ws->pairs = reinterpret_cast<int32_t *>(b + pairs_off);
         ws->inv = reinterpret_cast<int32_t *>(b + inv_off);
-        ws->tile_off = reinterpret_cast<int32_t *>(b + tile_off);
+        ws->tiles = reinterpret_cast<int32_t *>(b + tiles_off);
         ws->unit_ctr = reinterpret_cast<int32_t *>(b + ctr_off);
         ws->xfrag = reinterpret_cast<uint4 *>(b + xfrag_off);
         ws->xsum = reinterpret_cast<float *>(b + xsum_off);
@@ -381,9 +786,18 @@ size_t prefill_workspace_layout(int E, int H, int I, int T, int top_k, void *bas
     return off;
 }
 
+bool prefill_shape_supported(int H, int I)
+{
+    const PfDims d = pf_dims(1, H, I, 128, 16);
+    return H % DN_ROWS == 0 && I % GU_ROWS == 0 &&
+           stages_for(choose_stage(GU_ROWS, H, 2, false), gu_act_bytes(d)) >= 2 &&
+           stages_for(choose_stage(DN_ROWS, I, 1, false), dn_act_bytes(d)) >= 2;
+}
+
 cudaError_t launch_prefill(const PrefillArgs &a, const LaunchCfg &c)
 {
     cudaError_t e;
+    const PfDims d = pf_dims(a.E, a.H, a.I, a.T, a.top_k);
     GroupArgs g;
     g.idx = a.idx;
     g.T = a.T;
@@ -395,16 +809,50 @@ cudaError_t launch_prefill(const PrefillArgs &a, const LaunchCfg &c)
     g.status = a.status;
     if ((e = launch_group(g, c)) != cudaSuccess)
         return e;
-    if ((e = launch_ex(prefill_prep_kernel, dim3(a.T), dim3(128), 0, c, 1, a)) != cudaSuccess)
+    if ((e = launch_ex(prefill_prep_kernel, dim3(d.npos), dim3(128), 0, c, 1, a)) != cudaSuccess)
         return e;
-    const int grid = c.num_sms * 4;
-    if ((e = launch_ex(prefill_gateup_kernel, dim3(grid), dim3(PF_WARPS * 32), 0, c, 1, a)) !=
-        cudaSuccess)
+
+    // gate / up: tensor maps (8-row boxes) over the stacked routed matrices
+    // and the shared ones
+    CUtensorMap mg, mu, msg, msu;
+    memset(&mg, 0, sizeof(mg));
+    memset(&mu, 0, sizeof(mu));
+    memset(&msg, 0, sizeof(msg));
+    memset(&msu, 0, sizeof(msu));
+    const int Kw_gu = a.H / 8, Kw_dn = a.I / 8;
+    bool ok = (Kw_gu & 31) == 0;
+    ok = ok && encode_codes_map(&mg, a.gate.packed, (long)a.E * a.I, Kw_gu, GU_ROWS);
+    ok = ok && encode_codes_map(&mu, a.up.packed, (long)a.E * a.I, Kw_gu, GU_ROWS);
+    ok = ok && encode_codes_map(&msg, a.sh_gate.packed, a.I, Kw_gu, GU_ROWS);
+    ok = ok && encode_codes_map(&msu, a.sh_up.packed, a.I, Kw_gu, GU_ROWS);
+    const PfStage sgu = choose_stage(GU_ROWS, a.H, 2, ok);
+    const int ns_gu = stages_for(sgu, gu_act_bytes(d));
+    if (ns_gu < 2)
+        return cudaErrorInvalidValue;
+    const size_t smem_gu = pf_layout(sgu, gu_act_bytes(d), ns_gu).total;
+    if ((e = set_smem(prefill_gateup_kernel, smem_gu)) != cudaSuccess)
+        return e;
+    if ((e = launch_ex(prefill_gateup_kernel, dim3(c.num_sms), dim3(PF_THREADS), smem_gu, c, 1, a,
+                       sgu, ns_gu, mg, mu, msg, msu)) != cudaSuccess)
         return e;
     if ((e = launch_ex(prefill_hsum_kernel, dim3(c.num_sms), dim3(256), 0, c, 1, a)) != cudaSuccess)
         return e;
-    if ((e = launch_ex(prefill_down_kernel, dim3(grid), dim3(PF_WARPS * 32), 0, c, 1, a)) !=
-        cudaSuccess)
+
+    CUtensorMap md, msd;
+    memset(&md, 0, sizeof(md));
+    memset(&msd, 0, sizeof(msd));
+    bool okd = (Kw_dn & 31) == 0;
+    okd = okd && encode_codes_map(&md, a.down.packed, (long)a.E * a.H, Kw_dn, DN_ROWS);
+    okd = okd && encode_codes_map(&msd, a.sh_down.packed, a.H, Kw_dn, DN_ROWS);
+    const PfStage sdn = choose_stage(DN_ROWS, a.I, 1, okd);
+    const int ns_dn = stages_for(sdn, dn_act_bytes(d));
+    if (ns_dn < 2)
+        return cudaErrorInvalidValue;
+    const size_t smem_dn = pf_layout(sdn, dn_act_bytes(d), ns_dn).total;
+    if ((e = set_smem(prefill_down_kernel, smem_dn)) != cudaSuccess)
+        return e;
+    if ((e = launch_ex(prefill_down_kernel, dim3(c.num_sms), dim3(PF_THREADS), smem_dn, c, 1, a,
+                       sdn, ns_dn, md, msd)) != cudaSuccess)
         return e;
     return launch_ex(prefill_combine_kernel, dim3(c.num_sms * 2), dim3(256), 0, c, 1, a);
 }

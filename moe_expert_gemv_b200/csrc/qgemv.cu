@@ -10,20 +10,28 @@
 // (section "성능과 제약").
 //
 // Design (B200): persistent CTAs, one per SM.  A producer warp streams 16-row
-// weight tiles (codes + scales + biases) with cp.async.bulk into a ring of
-// shared-memory stages tracked by mbarriers; eight consumer warps split the
-// tile's 64-wide groups, dequantise codes to exact fp16 integers in registers
-// and run mma.sync m16n8k16 with the batch as the N=8 dimension; scale and
-// bias are applied per group in fp32; partial tiles are reduced through
-// shared memory and written as fp16.
+// weight tiles (codes + scales + biases) into a ring of shared-memory stages
+// tracked by mbarriers: when the row length is a multiple of 128 bytes the
+// codes of a tile arrive in ONE 3-D TMA tensor copy with 128-byte swizzling
+// (a 32 KB tile at K = 4096, so the copy engine runs at full rate); otherwise
+// each row is a 1-D bulk copy into a padded row.  Sixteen consumer warps
+// split the tile's 64-wide groups (a contiguous block each), place the codes
+// in registers as exact fp16 values (the code bits as subnormals) and run
+// mma.sync m16n8k16 with the batch as the N=8 dimension; scale and bias are
+// applied per group in fp32; partial tiles are reduced through shared memory
+// and written as fp16.  x is staged once per CTA, one thread per (row, group).
+#include <cuda.h>
+#include <string.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace qmoe {
 namespace {
 
-constexpr int QG_CW = 8;                      // consumer warps
-constexpr int QG_THREADS = (QG_CW + 1) * 32;  // + one producer warp
+constexpr int QG_CW = 16;                     // consumer warps
+constexpr int QG_CT = QG_CW * 32;             // consumer threads
+constexpr int QG_THREADS = QG_CT + 32;        // + one producer warp
 constexpr int QG_MAX_STAGES = 8;
 
 struct QgLayout {
@@ -32,11 +40,14 @@ struct QgLayout {
     size_t codes_bytes, sb_bytes, stage_bytes, total;
 };
 
-__host__ __device__ inline QgLayout qg_layout(int K, int bits, int ncol, int NS)
+// Offsets from a 1024-byte aligned base (the swizzled TMA destination must be
+// 1024-byte aligned); `total` includes the slack to align the dynamic
+// shared-memory window.
+__host__ __device__ inline QgLayout qg_layout(int K, int bits, int ncol, int NS, bool swz)
 {
     QgLayout L;
     L.G = K / kGroup;
-    L.S = tile_stride_words(K, bits);
+    L.S = swz ? K * bits / 32 : tile_stride_words(K, bits);
     size_t off = 0;
     L.xs_off = off;
     off += (size_t)L.G * 2 * ncol * 4 * 16;
@@ -47,21 +58,23 @@ __host__ __device__ inline QgLayout qg_layout(int K, int bits, int ncol, int NS)
     off += 2 * QG_CW * 32 * 16;
     L.bar_off = off;
     off += 2 * QG_MAX_STAGES * 8;
-    off = (off + 127) & ~(size_t)127;
+    off = (off + 1023) & ~(size_t)1023;
     L.stage_off = off;
     L.codes_bytes = (size_t)16 * L.S * 4;
     L.sb_bytes = (size_t)16 * L.G * 2;
-    L.stage_bytes = L.codes_bytes + 2 * L.sb_bytes;
+    L.stage_bytes = (L.codes_bytes + 2 * L.sb_bytes + 1023) & ~(size_t)1023;
     off += (size_t)NS * L.stage_bytes;
-    L.total = off;
+    L.total = off + 1024;
     return L;
 }
 
-template <int BITS>
-__global__ void __launch_bounds__(QG_THREADS, 1) qgemv_kernel(QgemvArgs a, int NS)
+template <int BITS, bool SWZ>
+__global__ void __launch_bounds__(QG_THREADS, 1)
+    qgemv_kernel(QgemvArgs a, int NS, const __grid_constant__ CUtensorMap codes_map)
 {
-    extern __shared__ __align__(128) unsigned char smem[];
-    const QgLayout L = qg_layout(a.K, BITS, a.B, NS);
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const QgLayout L = qg_layout(a.K, BITS, a.B, NS, SWZ);
     uint4 *xs = reinterpret_cast<uint4 *>(smem + L.xs_off);
     float *xsum = reinterpret_cast<float *>(smem + L.xsum_off);
     float4 *red = reinterpret_cast<float4 *>(smem + L.red_off);
@@ -85,6 +98,8 @@ __global__ void __launch_bounds__(QG_THREADS, 1) qgemv_kernel(QgemvArgs a, int N
         // ---------------- producer: weights are parameters, so they may be
         // streamed before the previous kernel of the stream has finished.
         if (lane == 0) {
+            if (SWZ)
+                prefetch_tensormap(&codes_map);
             const uint64_t pol = l2_evict_first_policy();
             int k = 0;
             int last_use[QG_MAX_STAGES];
@@ -99,10 +114,17 @@ __global__ void __launch_bounds__(QG_THREADS, 1) qgemv_kernel(QgemvArgs a, int N
                 const uint32_t row_bytes = (uint32_t)Kw * 4;
                 const uint32_t sb = (uint32_t)(rows * L.G * 2);
                 unsigned char *stage = smem + L.stage_off + (size_t)st * L.stage_bytes;
-                mbar_arrive_expect_tx(&full[st], rows * row_bytes + 2 * sb);
-                for (int r = 0; r < rows; ++r)
-                    bulk_g2s(stage + (size_t)r * L.S * 4, a.packed + (size_t)(r0 + r) * Kw,
-                             row_bytes, &full[st], pol);
+                if (SWZ) {
+                    // the tensor copy always delivers the whole 16-row box
+                    // (rows past N arrive zero-filled)
+                    mbar_arrive_expect_tx(&full[st], (uint32_t)L.codes_bytes + 2 * sb);
+                    tma_load_3d(stage, &codes_map, 0, r0, 0, &full[st], pol);
+                } else {
+                    mbar_arrive_expect_tx(&full[st], rows * row_bytes + 2 * sb);
+                    for (int r = 0; r < rows; ++r)
+                        bulk_g2s(stage + (size_t)r * L.S * 4, a.packed + (size_t)(r0 + r) * Kw,
+                                 row_bytes, &full[st], pol);
+                }
                 bulk_g2s(stage + L.codes_bytes, a.scales + (size_t)r0 * L.G, sb, &full[st], pol);
                 bulk_g2s(stage + L.codes_bytes + L.sb_bytes, a.biases + (size_t)r0 * L.G, sb,
                          &full[st], pol);
@@ -120,12 +142,21 @@ __global__ void __launch_bounds__(QG_THREADS, 1) qgemv_kernel(QgemvArgs a, int N
     pdl_wait();
     pdl_trigger();
     const int ctid = threadIdx.x;
-    const __half *x = a.x;
-    const int K = a.K;
-    stage_x<BITS>(xs, xsum, L.G, a.B, 1,
-                  [&](int, int n, int k) { return __half2float(x[n * K + k]); }, ctid, QG_CW * 32);
-    named_bar_sync(1, QG_CW * 32);
+    constexpr int KIND = BITS == 4 ? kPermS4 : 8;
+    constexpr float kCodeScale = BITS == 4 ? kSub20 : kSub24;   // undoes the subnormal codes
+    if ((reinterpret_cast<uintptr_t>(a.x) & 15u) == 0)
+        stage_x_groups<KIND>(xs, xsum, L.G, a.B, a.x, a.K, ctid, QG_CT);
+    else
+        stage_x<KIND>(xs, xsum, L.G, a.B, 1,
+                      [&](int, int n, int k) { return __half2float(a.x[(size_t)n * a.K + k]); },
+                      ctid, QG_CT);
+    named_bar_sync(1, QG_CT);
 
+    // this warp's groups: a contiguous block, so that with G % 64 == 0 the
+    // scales and biases of a row come as one 8-byte load per 4 groups
+    const int gpw = (L.G + QG_CW - 1) / QG_CW;
+    const int g0 = min(L.G, warp * gpw), g1 = min(L.G, g0 + gpw);
+    const bool vec_sb = (L.G & 63) == 0;
     const int gid = lane >> 2, tig = lane & 3;
     bool failed = false;
     int k = 0;
@@ -139,14 +170,75 @@ __global__ void __launch_bounds__(QG_THREADS, 1) qgemv_kernel(QgemvArgs a, int N
             const uint32_t *tile = reinterpret_cast<const uint32_t *>(stage);
             const __half *sc = reinterpret_cast<const __half *>(stage + L.codes_bytes);
             const __half *bi = reinterpret_cast<const __half *>(stage + L.codes_bytes + L.sb_bytes);
-            for (int g = warp; g < L.G; g += QG_CW)
-                tile_group<BITS>(tile, L.S, sc, bi, L.G, xs, xsum, a.B, g, gid, tig, acc);
+            // one group: codes of rows gid, gid+8 -> exact integer products,
+            // then scale (and the subnormal factor) and the folded bias
+            auto group = [&](int g, float s_lo, float s_hi, float b_lo, float b_hi) {
+                uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
+                if (gid < a.B) {
+                    x0 = xs[((g * 2 + 0) * a.B + gid) * 4 + tig];
+                    x1 = xs[((g * 2 + 1) * a.B + gid) * 4 + tig];
+                }
+                float r[4];
+                if (BITS == 4) {
+                    uint2 wa, wb;
+                    if (SWZ) {
+                        wa = *reinterpret_cast<const uint2 *>(swz128_frag<4>(stage, 2048, gid, g, tig));
+                        wb = *reinterpret_cast<const uint2 *>(
+                            swz128_frag<4>(stage, 2048, gid + 8, g, tig));
+                    } else {
+                        wa = *reinterpret_cast<const uint2 *>(tile + gid * L.S + g * 8 + 2 * tig);
+                        wb = *reinterpret_cast<const uint2 *>(tile + (gid + 8) * L.S + g * 8 +
+                                                              2 * tig);
+                    }
+                    mma_group_s4(r, wa, wb, x0, x1);
+                } else {
+                    uint4 wa, wb;
+                    if (SWZ) {
+                        wa = *reinterpret_cast<const uint4 *>(swz128_frag<8>(stage, 2048, gid, g, tig));
+                        wb = *reinterpret_cast<const uint4 *>(
+                            swz128_frag<8>(stage, 2048, gid + 8, g, tig));
+                    } else {
+                        wa = *reinterpret_cast<const uint4 *>(tile + gid * L.S + g * 16 + 4 * tig);
+                        wb = *reinterpret_cast<const uint4 *>(tile + (gid + 8) * L.S + g * 16 +
+                                                              4 * tig);
+                    }
+                    mma_group_s8(r, wa, wb, x0, x1);
+                }
+                const float2 X = *reinterpret_cast<const float2 *>(xsum + g * 8 + 2 * tig);
+                acc[0] = fmaf(s_lo * kCodeScale, r[0], fmaf(b_lo, X.x, acc[0]));
+                acc[1] = fmaf(s_lo * kCodeScale, r[1], fmaf(b_lo, X.y, acc[1]));
+                acc[2] = fmaf(s_hi * kCodeScale, r[2], fmaf(b_hi, X.x, acc[2]));
+                acc[3] = fmaf(s_hi * kCodeScale, r[3], fmaf(b_hi, X.y, acc[3]));
+            };
+            if (vec_sb) {
+                for (int gb = g0; gb < g1; gb += 4) {
+                    const uint2 slo = *reinterpret_cast<const uint2 *>(sc + gid * L.G + gb);
+                    const uint2 shi = *reinterpret_cast<const uint2 *>(sc + (gid + 8) * L.G + gb);
+                    const uint2 blo = *reinterpret_cast<const uint2 *>(bi + gid * L.G + gb);
+                    const uint2 bhi = *reinterpret_cast<const uint2 *>(bi + (gid + 8) * L.G + gb);
+                    const uint32_t sl[2] = {slo.x, slo.y}, sh[2] = {shi.x, shi.y};
+                    const uint32_t bl[2] = {blo.x, blo.y}, bh[2] = {bhi.x, bhi.y};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 fsl = __half22float2(u32_as_h2(sl[j >> 1]));
+                        const float2 fsh = __half22float2(u32_as_h2(sh[j >> 1]));
+                        const float2 fbl = __half22float2(u32_as_h2(bl[j >> 1]));
+                        const float2 fbh = __half22float2(u32_as_h2(bh[j >> 1]));
+                        group(gb + j, (j & 1) ? fsl.y : fsl.x, (j & 1) ? fsh.y : fsh.x,
+                              (j & 1) ? fbl.y : fbl.x, (j & 1) ? fbh.y : fbh.x);
+                    }
+                }
+            } else {
+                for (int g = g0; g < g1; ++g)
+                    group(g, __half2float(sc[gid * L.G + g]), __half2float(sc[(gid + 8) * L.G + g]),
+                          __half2float(bi[gid * L.G + g]), __half2float(bi[(gid + 8) * L.G + g]));
+            }
         }
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&empty[st]);
         red[((k & 1) * QG_CW + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        named_bar_sync(1, QG_CW * 32);
+        named_bar_sync(1, QG_CT);
         if (warp == k % QG_CW) {
             float v[4] = {0.f, 0.f, 0.f, 0.f};
             for (int w = 0; w < QG_CW; ++w) {
@@ -174,28 +266,76 @@ __global__ void __launch_bounds__(QG_THREADS, 1) qgemv_kernel(QgemvArgs a, int N
     }
 }
 
-}  // namespace
-
-cudaError_t launch_qgemv(const QgemvArgs &a, const LaunchCfg &c)
+template <int BITS, bool SWZ>
+cudaError_t launch_qgemv_t(const QgemvArgs &a, const LaunchCfg &c, const CUtensorMap &m)
 {
     const size_t budget = 227 * 1024;
-    const QgLayout L0 = qg_layout(a.K, a.bits, a.B, 0);
+    const QgLayout L0 = qg_layout(a.K, BITS, a.B, 0, SWZ);
     if (L0.total + 2 * L0.stage_bytes > budget)
         return cudaErrorInvalidValue;
     int NS = (int)((budget - L0.total) / L0.stage_bytes);
     NS = NS > QG_MAX_STAGES ? QG_MAX_STAGES : NS;
-    const QgLayout L = qg_layout(a.K, a.bits, a.B, NS);
+    const QgLayout L = qg_layout(a.K, BITS, a.B, NS, SWZ);
     const int n_items = (a.N + 15) / 16;
     const int grid = n_items < c.num_sms ? n_items : c.num_sms;
     cudaError_t e;
-    if (a.bits == 4) {
-        if ((e = set_smem(qgemv_kernel<4>, L.total)) != cudaSuccess)
-            return e;
-        return launch_ex(qgemv_kernel<4>, dim3(grid), dim3(QG_THREADS), L.total, c, 1, a, NS);
-    }
-    if ((e = set_smem(qgemv_kernel<8>, L.total)) != cudaSuccess)
+    if ((e = set_smem(qgemv_kernel<BITS, SWZ>, L.total)) != cudaSuccess)
         return e;
-    return launch_ex(qgemv_kernel<8>, dim3(grid), dim3(QG_THREADS), L.total, c, 1, a, NS);
+    return launch_ex(qgemv_kernel<BITS, SWZ>, dim3(grid), dim3(QG_THREADS), L.total, c, 1, a, NS,
+                     m);
+}
+
+}  // namespace
+
+// ---------------------------------------------------- host: tensor map --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            (void)cudaGetLastError();
+    }
+    return fn;
+}
+
+bool encode_codes_map(CUtensorMap *m, const uint32_t *packed, long rows, int Kw, int box_rows)
+{
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn || Kw % 32 != 0 || Kw / 32 > 256 || box_rows < 1 || box_rows > 256)
+        return false;
+    const cuuint64_t dims[3] = {32, (cuuint64_t)rows, (cuuint64_t)(Kw / 32)};
+    const cuuint64_t strides[2] = {(cuuint64_t)Kw * 4, 128};
+    const cuuint32_t box[3] = {32, (cuuint32_t)box_rows, (cuuint32_t)(Kw / 32)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t *>(packed), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+cudaError_t launch_qgemv(const QgemvArgs &a, const LaunchCfg &c)
+{
+    const int Kw = a.K * a.bits / 32;
+    CUtensorMap m;
+    memset(&m, 0, sizeof(m));
+    const bool swz = encode_codes_map(&m, a.packed, a.N, Kw, 16) &&
+                     qg_layout(a.K, a.bits, a.B, 2, true).total <= 227 * 1024;
+    if (a.bits == 4)
+        return swz ? launch_qgemv_t<4, true>(a, c, m) : launch_qgemv_t<4, false>(a, c, m);
+    return swz ? launch_qgemv_t<8, true>(a, c, m) : launch_qgemv_t<8, false>(a, c, m);
 }
 
 }  // namespace qmoe
