@@ -251,13 +251,14 @@ qmoe_status moe_group_tokens(const int32_t *idx, int32_t tokens, int32_t top_k,
  * moe_expert_qmlp, row by row):
  *   y[t] = shared(x[t]) + sum_j weights[t][j] * expert_{idx[t][j]}(x[t])
  * x: fp16 [tokens][hidden], 16-byte aligned, tokens 1..128; idx: int32 [tokens][top_k];
- * weights: fp32 [tokens][top_k]; y: fp16 [tokens][hidden].
+ * weights: fp32 [tokens][top_k]; y: fp16 [tokens][hidden], 4-byte aligned.
  * workspace: moe_prefill_workspace_bytes() bytes, 16-byte aligned; no
  * initial contents are required.
- * Every expert touched by the chunk (and the shared expert) is read from
- * memory once per call.  Returns QMOE_ERR_UNSUPPORTED when two 16-row
- * gate+up tiles (2 x 16 x hidden/2 bytes of codes plus scales and biases)
- * do not fit the kernels' shared-memory ring (hidden > ~12,000).
+ * Weights are streamed per 8-token tile of each expert: an expert with at
+ * most 8 tokens in the chunk is read once, a heavier one once per tile (the
+ * repeats served by L2).  Returns QMOE_ERR_UNSUPPORTED unless hidden is a
+ * multiple of 256 and at most 4,352 and inter is at most 2,176 (two
+ * activation tiles and two weight sub-blocks must fit shared memory).
  * ------------------------------------------------------------------------- */
 size_t moe_prefill_workspace_bytes(const qmoe_moe_layer *L, int32_t tokens, int32_t top_k);
 

@@ -466,7 +466,7 @@ qmoe_status moe_prefill_qgemm(const qmoe_moe_layer *L, const uint16_t *x, int32_
         return QMOE_ERR_INVALID_ARG;
     if (!prefill_shape_supported(L->hidden, L->inter))
         return QMOE_ERR_UNSUPPORTED;
-    if (!aligned(x, 16) || !aligned(idx, 4) || !aligned(weights, 4) || !aligned(y, 2) ||
+    if (!aligned(x, 16) || !aligned(idx, 4) || !aligned(weights, 4) || !aligned(y, 4) ||
         (status_dev && !aligned(status_dev, 4)))
         return QMOE_ERR_ALIGNMENT;
     if (!workspace)

@@ -160,18 +160,6 @@ __host__ __device__ inline size_t dn_act_bytes(const PfDims &d)
     return (size_t)TILE_T * d.hf_stride * 16 + (size_t)TILE_T * d.hs_stride * 4;
 }
 
-// this lane's 8 code bytes of row r, group g (4-bit, fragment words 2tig, 2tig+1)
-__device__ __forceinline__ uint2 tile_frag(const unsigned char *tile, const PfStage &st, int r,
-                                           int g, int tig)
-{
-    const void *p;
-    if (st.mode == TILE_SWZ)
-        p = swz128_frag<4>(tile, st.rows * 128, r, g, tig);
-    else
-        p = tile + ((size_t)r * st.S + g * 8 + 2 * tig) * 4;
-    return *reinterpret_cast<const uint2 *>(p);
-}
-
 // issue the copies of one matrix tile (rows [row0, row0 + st.rows) of a
 // row-major [.][Kw] code array) into `dst`
 __device__ __forceinline__ void issue_tile(unsigned char *dst, const PfStage &st,
@@ -282,16 +270,35 @@ __global__ void __launch_bounds__(128) prefill_prep_kernel(PrefillArgs a)
                                 a.x + (size_t)tok * d.H, d.H, threadIdx.x, 128, 1);
     }
     if (p == 0) {
-        if (threadIdx.x == 0) {
-            int n = 0;
-            for (int s = 0; s <= d.E; ++s) {
-                const int nt = (slot_count(a, s) + TILE_T - 1) / TILE_T;
-                for (int t = 0; t < nt; ++t)
-                    a.ws.tiles[n++] = (s << 4) | t;
+        // token tiles of every slot in slot order: a block-wide exclusive scan
+        // of the per-slot tile counts, 128 slots per pass
+        __shared__ int s_scan[128];
+        __shared__ int s_base;
+        if (threadIdx.x == 0)
+            s_base = 0;
+        for (int s0 = 0; s0 <= d.E; s0 += 128) {
+            const int s = s0 + threadIdx.x;
+            const int nt = s <= d.E ? (slot_count(a, s) + TILE_T - 1) / TILE_T : 0;
+            s_scan[threadIdx.x] = nt;
+            __syncthreads();
+            for (int o = 1; o < 128; o <<= 1) {   // inclusive Hillis-Steele scan
+                const int v = threadIdx.x >= o ? s_scan[threadIdx.x - o] : 0;
+                __syncthreads();
+                s_scan[threadIdx.x] += v;
+                __syncthreads();
             }
+            const int first = s_base + s_scan[threadIdx.x] - nt;
+            for (int t = 0; t < nt; ++t)
+                a.ws.tiles[first + t] = (s << 4) | t;
+            __syncthreads();
+            if (threadIdx.x == 127)
+                s_base += s_scan[127];
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) {
             a.ws.unit_ctr[0] = 0;
             a.ws.unit_ctr[1] = 0;
-            a.ws.unit_ctr[2] = n;
+            a.ws.unit_ctr[2] = s_base;
         }
         // positions of the valid pairs (ids out of range were dropped by the
         // grouping, so only offsets[E] positions hold a pair)
@@ -494,27 +501,67 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const uint4 *xr = xf + gid * d.xg_stride;
                 const float *xs0 = xsm + (2 * tig) * d.xs_stride;
                 const float *xs1 = xs0 + d.xs_stride;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
-                for (int g = 0; g < d.GH; ++g) {
-                    uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
-                    if (nvalid) {
-                        x0 = xr[(g * 2 + 0) * 4 + tig];
-                        x1 = xr[(g * 2 + 1) * 4 + tig];
-                    }
-                    float r[4];
-                    mma_group_s4(r, tile_frag(gt, st, gid, g, tig), tile_frag(utl, st, gid, g, tig),
-                                 x0, x1);
-                    const float X0 = xs0[g], X1 = xs1[g];
-                    const float sg = __half2float(gs[gid * d.GH + g]) * kSub20;
-                    const float bg = __half2float(gb[gid * d.GH + g]);
-                    const float su = __half2float(us[gid * d.GH + g]) * kSub20;
-                    const float bu = __half2float(ub[gid * d.GH + g]);
-                    acc[0] = fmaf(sg, r[0], fmaf(bg, X0, acc[0]));   // gate, token 2tig
-                    acc[1] = fmaf(sg, r[1], fmaf(bg, X1, acc[1]));   // gate, token 2tig+1
-                    acc[2] = fmaf(su, r[2], fmaf(bu, X0, acc[2]));   // up
-                    acc[3] = fmaf(su, r[3], fmaf(bu, X1, acc[3]));
+                // fragment byte offsets of row gid for the 4 groups of a step of
+                // 4 (GH % 4 == 0): step q4 adds q4 * cstride
+                int off[4], cstride;
+                if (st.mode == TILE_SWZ) {
+                    cstride = GU_ROWS * 128;   // one swizzled 128-byte chunk per 4 groups
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        off[j] = gid * 128 + (((2 * j + (tig >> 1)) ^ gid) << 4) + (tig & 1) * 8;
+                } else {
+                    cstride = 128;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        off[j] = gid * st.S * 4 + j * 32 + tig * 8;
                 }
+                // code products and folded biases accumulate apart; the
+                // subnormal factor 2^20 is applied once at the end
+                float aq[4] = {0.f, 0.f, 0.f, 0.f}, ab[4] = {0.f, 0.f, 0.f, 0.f};
+                const int nch = d.GH / 4;
+                for (int q4 = 0; q4 < nch; ++q4) {
+                    const unsigned char *gtc = gt + q4 * cstride, *utc = utl + q4 * cstride;
+                    const uint2 sgv = *reinterpret_cast<const uint2 *>(gs + gid * d.GH + 4 * q4);
+                    const uint2 bgv = *reinterpret_cast<const uint2 *>(gb + gid * d.GH + 4 * q4);
+                    const uint2 suv = *reinterpret_cast<const uint2 *>(us + gid * d.GH + 4 * q4);
+                    const uint2 buv = *reinterpret_cast<const uint2 *>(ub + gid * d.GH + 4 * q4);
+                    const float4 X0 = *reinterpret_cast<const float4 *>(xs0 + 4 * q4);
+                    const float4 X1 = *reinterpret_cast<const float4 *>(xs1 + 4 * q4);
+                    const float x0s[4] = {X0.x, X0.y, X0.z, X0.w};
+                    const float x1s[4] = {X1.x, X1.y, X1.z, X1.w};
+                    const uint32_t sgw[2] = {sgv.x, sgv.y}, bgw[2] = {bgv.x, bgv.y};
+                    const uint32_t suw[2] = {suv.x, suv.y}, buw[2] = {buv.x, buv.y};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int g = 4 * q4 + j;
+                        uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
+                        if (nvalid) {
+                            x0 = xr[(g * 2 + 0) * 4 + tig];
+                            x1 = xr[(g * 2 + 1) * 4 + tig];
+                        }
+                        float r[4];
+                        mma_group_s4(r, *reinterpret_cast<const uint2 *>(gtc + off[j]),
+                                     *reinterpret_cast<const uint2 *>(utc + off[j]), x0, x1);
+                        const float2 fsg = __half22float2(u32_as_h2(sgw[j >> 1]));
+                        const float2 fbg = __half22float2(u32_as_h2(bgw[j >> 1]));
+                        const float2 fsu = __half22float2(u32_as_h2(suw[j >> 1]));
+                        const float2 fbu = __half22float2(u32_as_h2(buw[j >> 1]));
+                        const float sg = (j & 1) ? fsg.y : fsg.x, bg = (j & 1) ? fbg.y : fbg.x;
+                        const float su = (j & 1) ? fsu.y : fsu.x, bu = (j & 1) ? fbu.y : fbu.x;
+                        aq[0] = fmaf(sg, r[0], aq[0]);   // gate, token 2tig
+                        aq[1] = fmaf(sg, r[1], aq[1]);   // gate, token 2tig+1
+                        aq[2] = fmaf(su, r[2], aq[2]);   // up
+                        aq[3] = fmaf(su, r[3], aq[3]);
+                        ab[0] = fmaf(bg, x0s[j], ab[0]);
+                        ab[1] = fmaf(bg, x1s[j], ab[1]);
+                        ab[2] = fmaf(bu, x0s[j], ab[2]);
+                        ab[3] = fmaf(bu, x1s[j], ab[3]);
+                    }
+                }
+                float acc[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    acc[i] = fmaf(aq[i], kSub20, ab[i]);
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&empty[slot]);
@@ -652,7 +699,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const uint4 *hr = hb + gid * d.hf_stride;
                 const float *hs0 = hsm + (2 * tig) * d.hs_stride;
                 const float *hs1 = hs0 + d.hs_stride;
-                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                // rows gid, gid+8, gid+16, gid+24 share (r & 7) = gid
+                const bool swz = st.mode == TILE_SWZ;
+                int rowoff[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    rowoff[i] = swz ? (gid + 8 * i) * 128 + (tig & 1) * 8
+                                    : (gid + 8 * i) * st.S * 4 + tig * 8;
+                float aq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                float ab[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                 for (int g = 0; g < d.GI; ++g) {
                     uint4 h0 = make_uint4(0, 0, 0, 0), h1 = h0, l0 = h0, l1 = h0;
                     if (nvalid) {
@@ -661,24 +716,38 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         l0 = hr[((g * 2 + 0) * 2 + 1) * 4 + tig];
                         l1 = hr[((g * 2 + 1) * 2 + 1) * 4 + tig];
                     }
-                    const float X0 = hs0[g * 2] + hs0[g * 2 + 1];
-                    const float X1 = hs1[g * 2] + hs1[g * 2 + 1];
+                    const float2 S0 = *reinterpret_cast<const float2 *>(hs0 + g * 2);
+                    const float2 S1 = *reinterpret_cast<const float2 *>(hs1 + g * 2);
+                    const float X0 = S0.x + S0.y, X1 = S1.x + S1.y;
+                    const int goff = swz ? (g >> 2) * (DN_ROWS * 128) +
+                                               (((2 * (g & 3) + (tig >> 1)) ^ gid) << 4)
+                                         : g * 32;
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         const int ra = half * 16 + gid, rb = ra + 8;
                         float r[4];
-                        mma_group_s4_hilo(r, tile_frag(wt, st, ra, g, tig),
-                                          tile_frag(wt, st, rb, g, tig), h0, h1, l0, l1);
-                        const float sa = __half2float(sc[ra * d.GI + g]) * kSub20;
+                        mma_group_s4_hilo(
+                            r, *reinterpret_cast<const uint2 *>(wt + rowoff[2 * half] + goff),
+                            *reinterpret_cast<const uint2 *>(wt + rowoff[2 * half + 1] + goff), h0,
+                            h1, l0, l1);
+                        const float sa = __half2float(sc[ra * d.GI + g]);
                         const float ba = __half2float(bi[ra * d.GI + g]);
-                        const float sb = __half2float(sc[rb * d.GI + g]) * kSub20;
+                        const float sb = __half2float(sc[rb * d.GI + g]);
                         const float bb = __half2float(bi[rb * d.GI + g]);
-                        acc[4 * half + 0] = fmaf(sa, r[0], fmaf(ba, X0, acc[4 * half + 0]));
-                        acc[4 * half + 1] = fmaf(sa, r[1], fmaf(ba, X1, acc[4 * half + 1]));
-                        acc[4 * half + 2] = fmaf(sb, r[2], fmaf(bb, X0, acc[4 * half + 2]));
-                        acc[4 * half + 3] = fmaf(sb, r[3], fmaf(bb, X1, acc[4 * half + 3]));
+                        aq[4 * half + 0] = fmaf(sa, r[0], aq[4 * half + 0]);
+                        aq[4 * half + 1] = fmaf(sa, r[1], aq[4 * half + 1]);
+                        aq[4 * half + 2] = fmaf(sb, r[2], aq[4 * half + 2]);
+                        aq[4 * half + 3] = fmaf(sb, r[3], aq[4 * half + 3]);
+                        ab[4 * half + 0] = fmaf(ba, X0, ab[4 * half + 0]);
+                        ab[4 * half + 1] = fmaf(ba, X1, ab[4 * half + 1]);
+                        ab[4 * half + 2] = fmaf(bb, X0, ab[4 * half + 2]);
+                        ab[4 * half + 3] = fmaf(bb, X1, ab[4 * half + 3]);
                     }
                 }
+                float acc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    acc[i] = fmaf(aq[i], kSub20, ab[i]);
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&empty[slot]);
@@ -704,23 +773,33 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 }
 
 // --------------------------------------------------------------- combine --
+// four consecutive outputs of one token per thread (H % 4 == 0)
 __global__ void __launch_bounds__(256) prefill_combine_kernel(PrefillArgs a)
 {
     pdl_wait();
     pdl_trigger();
     const PfDims d = pf_dims(a.E, a.H, a.I, a.T, a.top_k);
-    const int n = d.T * d.H;
+    const int H4 = d.H / 4;
+    const int n = d.T * H4;
     for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
-        const int tok = t / d.H, col = t % d.H;
-        float y = __ldcg(a.ws.r + (size_t)(d.T * d.K + tok) * d.H + col);
+        const int tok = t / H4, c4 = t - tok * H4;
+        float4 y = __ldcg(reinterpret_cast<const float4 *>(a.ws.r + (size_t)(d.T * d.K + tok) * d.H) +
+                          c4);
         for (int j = 0; j < d.K; ++j) {
             const int e = a.idx[tok * d.K + j];
             if (e < 0 || e >= d.E)
                 continue;   // flagged by the grouping kernel, contributes nothing
             const int p = a.ws.inv[tok * d.K + j];
-            y = fmaf(a.weights[tok * d.K + j], __ldcg(a.ws.r + (size_t)p * d.H + col), y);
+            const float w = a.weights[tok * d.K + j];
+            const float4 r = __ldcg(reinterpret_cast<const float4 *>(a.ws.r + (size_t)p * d.H) + c4);
+            y.x = fmaf(w, r.x, y.x);
+            y.y = fmaf(w, r.y, y.y);
+            y.z = fmaf(w, r.z, y.z);
+            y.w = fmaf(w, r.w, y.w);
         }
-        a.y[t] = __float2half_rn(y);
+        __half2 *out = reinterpret_cast<__half2 *>(a.y + (size_t)tok * d.H) + 2 * c4;
+        out[0] = __floats2half2_rn(y.x, y.y);
+        out[1] = __floats2half2_rn(y.z, y.w);
     }
 }
 
@@ -789,7 +868,7 @@ size_t prefill_workspace_layout(int E, int H, int I, int T, int top_k, void *bas
 bool prefill_shape_supported(int H, int I)
 {
     const PfDims d = pf_dims(1, H, I, 128, 16);
-    return H % DN_ROWS == 0 && I % GU_ROWS == 0 &&
+    return H % 256 == 0 && I % GU_ROWS == 0 &&
            stages_for(choose_stage(GU_ROWS, H, 2, false), gu_act_bytes(d)) >= 2 &&
            stages_for(choose_stage(DN_ROWS, I, 1, false), dn_act_bytes(d)) >= 2;
 }

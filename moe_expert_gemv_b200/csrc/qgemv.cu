@@ -170,48 +170,58 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
             const uint32_t *tile = reinterpret_cast<const uint32_t *>(stage);
             const __half *sc = reinterpret_cast<const __half *>(stage + L.codes_bytes);
             const __half *bi = reinterpret_cast<const __half *>(stage + L.codes_bytes + L.sb_bytes);
-            // one group: codes of rows gid, gid+8 -> exact integer products,
-            // then scale (and the subnormal factor) and the folded bias
-            auto group = [&](int g, float s_lo, float s_hi, float b_lo, float b_hi) {
+            // code products and folded biases accumulate apart; the subnormal
+            // factor is applied once at the end
+            float aq[4] = {0.f, 0.f, 0.f, 0.f}, ab[4] = {0.f, 0.f, 0.f, 0.f};
+            // one group from its fragment addresses (rows gid, gid+8)
+            auto group = [&](int g, const void *fa, const void *fb, float s_lo, float s_hi,
+                             float b_lo, float b_hi) {
                 uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
                 if (gid < a.B) {
                     x0 = xs[((g * 2 + 0) * a.B + gid) * 4 + tig];
                     x1 = xs[((g * 2 + 1) * a.B + gid) * 4 + tig];
                 }
                 float r[4];
-                if (BITS == 4) {
-                    uint2 wa, wb;
-                    if (SWZ) {
-                        wa = *reinterpret_cast<const uint2 *>(swz128_frag<4>(stage, 2048, gid, g, tig));
-                        wb = *reinterpret_cast<const uint2 *>(
-                            swz128_frag<4>(stage, 2048, gid + 8, g, tig));
-                    } else {
-                        wa = *reinterpret_cast<const uint2 *>(tile + gid * L.S + g * 8 + 2 * tig);
-                        wb = *reinterpret_cast<const uint2 *>(tile + (gid + 8) * L.S + g * 8 +
-                                                              2 * tig);
-                    }
-                    mma_group_s4(r, wa, wb, x0, x1);
-                } else {
-                    uint4 wa, wb;
-                    if (SWZ) {
-                        wa = *reinterpret_cast<const uint4 *>(swz128_frag<8>(stage, 2048, gid, g, tig));
-                        wb = *reinterpret_cast<const uint4 *>(
-                            swz128_frag<8>(stage, 2048, gid + 8, g, tig));
-                    } else {
-                        wa = *reinterpret_cast<const uint4 *>(tile + gid * L.S + g * 16 + 4 * tig);
-                        wb = *reinterpret_cast<const uint4 *>(tile + (gid + 8) * L.S + g * 16 +
-                                                              4 * tig);
-                    }
-                    mma_group_s8(r, wa, wb, x0, x1);
-                }
+                if (BITS == 4)
+                    mma_group_s4(r, *reinterpret_cast<const uint2 *>(fa),
+                                 *reinterpret_cast<const uint2 *>(fb), x0, x1);
+                else
+                    mma_group_s8(r, *reinterpret_cast<const uint4 *>(fa),
+                                 *reinterpret_cast<const uint4 *>(fb), x0, x1);
                 const float2 X = *reinterpret_cast<const float2 *>(xsum + g * 8 + 2 * tig);
-                acc[0] = fmaf(s_lo * kCodeScale, r[0], fmaf(b_lo, X.x, acc[0]));
-                acc[1] = fmaf(s_lo * kCodeScale, r[1], fmaf(b_lo, X.y, acc[1]));
-                acc[2] = fmaf(s_hi * kCodeScale, r[2], fmaf(b_hi, X.x, acc[2]));
-                acc[3] = fmaf(s_hi * kCodeScale, r[3], fmaf(b_hi, X.y, acc[3]));
+                aq[0] = fmaf(s_lo, r[0], aq[0]);
+                aq[1] = fmaf(s_lo, r[1], aq[1]);
+                aq[2] = fmaf(s_hi, r[2], aq[2]);
+                aq[3] = fmaf(s_hi, r[3], aq[3]);
+                ab[0] = fmaf(b_lo, X.x, ab[0]);
+                ab[1] = fmaf(b_lo, X.y, ab[1]);
+                ab[2] = fmaf(b_hi, X.x, ab[2]);
+                ab[3] = fmaf(b_hi, X.y, ab[3]);
+            };
+            // fragment address of row r, group g
+            auto frag = [&](int r, int g) -> const void * {
+                if (SWZ)
+                    return swz128_frag<BITS>(stage, 2048, r, g, tig);
+                return BITS == 4 ? (const void *)(tile + r * L.S + g * 8 + 2 * tig)
+                                 : (const void *)(tile + r * L.S + g * 16 + 4 * tig);
             };
             if (vec_sb) {
+                // 4 groups per step (g0 % 4 == 0): fragment offsets of row gid
+                // precomputed; row gid+8 is 16 rows of bytes further
+                constexpr int GPC = BITS == 4 ? 4 : 2;   // groups per 128-byte chunk
+                int off[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int jc = j % GPC;
+                    off[j] = SWZ ? gid * 128 + (j / GPC) * 2048 +
+                                       (BITS == 4 ? ((((2 * jc + (tig >> 1)) ^ gid) << 4) + (tig & 1) * 8)
+                                                  : (((4 * jc + tig) ^ gid) << 4))
+                                 : (gid * L.S + j * (BITS == 4 ? 8 : 16) + tig * (BITS == 4 ? 2 : 4)) * 4;
+                }
+                const int row8 = SWZ ? 8 * 128 : 8 * L.S * 4;
                 for (int gb = g0; gb < g1; gb += 4) {
+                    const unsigned char *base =
+                        stage + (SWZ ? (gb / GPC) * 2048 : gb * (BITS == 4 ? 32 : 64));
                     const uint2 slo = *reinterpret_cast<const uint2 *>(sc + gid * L.G + gb);
                     const uint2 shi = *reinterpret_cast<const uint2 *>(sc + (gid + 8) * L.G + gb);
                     const uint2 blo = *reinterpret_cast<const uint2 *>(bi + gid * L.G + gb);
@@ -224,15 +234,20 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                         const float2 fsh = __half22float2(u32_as_h2(sh[j >> 1]));
                         const float2 fbl = __half22float2(u32_as_h2(bl[j >> 1]));
                         const float2 fbh = __half22float2(u32_as_h2(bh[j >> 1]));
-                        group(gb + j, (j & 1) ? fsl.y : fsl.x, (j & 1) ? fsh.y : fsh.x,
-                              (j & 1) ? fbl.y : fbl.x, (j & 1) ? fbh.y : fbh.x);
+                        group(gb + j, base + off[j], base + off[j] + row8, (j & 1) ? fsl.y : fsl.x,
+                              (j & 1) ? fsh.y : fsh.x, (j & 1) ? fbl.y : fbl.x,
+                              (j & 1) ? fbh.y : fbh.x);
                     }
                 }
             } else {
                 for (int g = g0; g < g1; ++g)
-                    group(g, __half2float(sc[gid * L.G + g]), __half2float(sc[(gid + 8) * L.G + g]),
-                          __half2float(bi[gid * L.G + g]), __half2float(bi[(gid + 8) * L.G + g]));
+                    group(g, frag(gid, g), frag(gid + 8, g), __half2float(sc[gid * L.G + g]),
+                          __half2float(sc[(gid + 8) * L.G + g]), __half2float(bi[gid * L.G + g]),
+                          __half2float(bi[(gid + 8) * L.G + g]));
             }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                acc[i] = fmaf(aq[i], kCodeScale, ab[i]);
         }
         __syncwarp();
         if (lane == 0)
