@@ -319,7 +319,7 @@ def decode_config(nl, n_ranks):
         "layers": nl, "experts": E, "hidden": H, "inter": I, "top_k": TOPK,
         "bytes_per_layer": LAYER_BYTES,
         "l2": "inputs larger than L2: %.2f GB of weights, each step streams %.0f MB"
-              % (nl * LAYER_BYTES / 1e9, nl * LAYER_BYTES / 1e6),
+              % (nl * (ROUTER_BYTES + (E + 1) * EXPERT_BYTES) / 1e9, nl * LAYER_BYTES / 1e6),
         "path": "moe_decode_layers: one persistent cooperative launch per step",
         "parallelism": "replicas x%d" % n_ranks if n_ranks > 1 else "single GPU",
     }
