@@ -63,6 +63,32 @@ def qmatrix(g, rows, cols, bits=4, scale=DENSE_SCALE, bias=DENSE_BIAS, lead=()):
     return P, S, B
 
 
+FMT_ZP4, FMT_SYM8 = 1, 2
+SYM8_SCALE = (0.001, 0.004)
+
+
+def to_bf16_bits(a):
+    """fp64 values -> bf16 bit patterns (via fp32, round to nearest even)."""
+    u = np.asarray(a, dtype=np.float64).astype(np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def qmatrix_fmt(g, rows, cols, fmt):
+    """Format-variant matrix: (packed uint32 [rows][cols*bits/32], params uint32
+    [rows][cols/64] = bf16 scale | zero point << 16, signs uint32 [cols/32]).
+    ZP4: 4-bit codes, zero points uniform in 0..15, scales U(0.005, 0.02);
+    SYM8: 8-bit two's-complement codes, scales U(0.001, 0.004)."""
+    assert cols % 64 == 0 and fmt in (FMT_ZP4, FMT_SYM8)
+    bits = 4 if fmt == FMT_ZP4 else 8
+    P = random_words(g, (rows, cols * bits // 32))
+    lo, hi = DENSE_SCALE if fmt == FMT_ZP4 else SYM8_SCALE
+    S = to_bf16_bits(g.uniform(lo, hi, (rows, cols // 64))).astype(np.uint32)
+    Z = (g.integers(0, 16, (rows, cols // 64)).astype(np.uint32) if fmt == FMT_ZP4
+         else np.zeros((rows, cols // 64), np.uint32))
+    signs = random_words(g, (cols // 32,))
+    return P, S | (Z << 16), signs
+
+
 def activations(seed, rows, cols, layer=0):
     """x [rows][cols] ~ N(0,1), fp16 bits."""
     return to_f16_bits(rng(seed, layer, _TAGS["x"]).standard_normal((rows, cols)))

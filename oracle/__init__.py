@@ -55,6 +55,11 @@ def lib():
         L.or_expert.argtypes = [ctypes.POINTER(OrLayer), i64, p, p]
         L.or_moe_layer.argtypes = [ctypes.POINTER(OrLayer), p, i64, p, p, i64, p, p]
         L.or_group.argtypes = [p, i64, i64, i64, p, p, p]
+        L.or_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        L.or_bf16_to_f64.restype = ctypes.c_double
+        L.or_rht32.argtypes = [p, p, i64, i64, p]
+        L.or_dequant_fmt.argtypes = [p, p, i64, i64, ctypes.c_int, p]
+        L.or_qgemv_fmt.argtypes = [p, p, i64, i64, ctypes.c_int, p, ctypes.c_int, p, i64, p, p]
         for name in ("or_unpack", "or_pack", "or_dequant", "or_qgemv", "or_router",
                      "or_topk_from_logits", "or_expert", "or_moe_layer", "or_group"):
             getattr(L, name).restype = ctypes.c_int
@@ -133,6 +138,47 @@ def qgemv(packed, scales, biases, N, K, bits, x16):
 
 
 # -------------------------------------------------------------- router ------
+FMT_ZP4, FMT_SYM8 = 1, 2
+
+
+def bf16_to_f64(bits):
+    """bf16 bit patterns -> fp64 values (exact)."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return np.array([lib().or_bf16_to_f64(int(v)) for v in b.ravel()], dtype=np.float64).reshape(
+        b.shape)
+
+
+def rht32(x, signs, K):
+    """The block-32 random Hadamard rotation of x [B][K] (fp64 values);
+    signs: uint32 [K/32] or None (D = I)."""
+    x = _c(np.atleast_2d(x), np.float64)
+    B = x.shape[0]
+    out = np.empty((B, K), np.float64)
+    s = None if signs is None else _c(signs, np.uint32)
+    _check(lib().or_rht32(_ptr(x), None if s is None else _ptr(s), B, K, _ptr(out)), "or_rht32")
+    return out
+
+
+def dequant_fmt(packed, params, N, K, fmt):
+    W = np.empty((N, K), np.float64)
+    _check(lib().or_dequant_fmt(_ptr(_c(packed, np.uint32)), _ptr(_c(params, np.uint32)), N, K,
+                                fmt, _ptr(W)), "or_dequant_fmt")
+    return W
+
+
+def qgemv_fmt(packed, params, N, K, fmt, x16, signs=None, rotate=False):
+    """Format-variant qGEMV: returns (y64 [B][N], y16 bits [B][N])."""
+    x = _c(np.atleast_2d(x16), np.uint16)
+    B = x.shape[0]
+    y64 = np.empty((B, N), np.float64)
+    y16 = np.empty((B, N), np.uint16)
+    s = None if signs is None else _c(signs, np.uint32)
+    _check(lib().or_qgemv_fmt(_ptr(_c(packed, np.uint32)), _ptr(_c(params, np.uint32)), N, K, fmt,
+                              None if s is None else _ptr(s), int(bool(rotate)), _ptr(x), B,
+                              _ptr(y64), _ptr(y16)), "or_qgemv_fmt")
+    return y64, y16
+
+
 def router(packed, scales, biases, E, K, bits, x16, top_k):
     """Returns (logits64 [T][E], idx [T][k] int32, wt [T][k] fp64)."""
     packed, scales, biases = _c(packed, np.uint32), _c(scales, np.uint16), _c(biases, np.uint16)

@@ -225,6 +225,131 @@ int or_qgemv(const uint32_t *P, const uint16_t *S, const uint16_t *Bi,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Format variants: zero-point 4-bit and symmetric 8-bit with bf16 scales,   */
+/* and the block-32 random Hadamard rotation of the input                     */
+/* ------------------------------------------------------------------------ */
+/* uzu page (discuss.pytorch.kr), section "uzu의 모델 변환과 Mirai 양자화 형식":
+   Mirai-M is 4-bit asymmetric integer quantisation with a 4-bit zero point
+   and a bf16 scale (group 64 per the model card); Mirai-L is 8-bit symmetric;
+   both quantise after a random Hadamard transform with block size 32.
+   Readings (the page gives the formats by name only):
+     - ZP4:  w = s * (q - z), q and z unsigned 4-bit, s bf16, one (s, z) per
+             group of 64 inputs of a row;
+     - SYM8: w = s * q, q a two's-complement 8-bit code, s bf16 per group;
+     - per-group parameters are one uint32: bits 0..15 the bf16 scale,
+       bits 16..23 the zero point (0 for SYM8);
+     - rotation: the weights were quantised in the rotated basis, so the
+       product is y = W_q (R x) with R = blockdiag(H_32 D / sqrt(32)),
+       H_32[i][j] = (-1)^popcount(i & j) (Sylvester), D = diag(+-1) from one
+       sign bit per input (bit i % 32 of word i / 32; set = -1). */
+
+/* bf16 bit pattern -> value (exact: a bf16 is the top half of an fp32). */
+double or_bf16_to_f64(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static int popcount32(uint32_t v)
+{
+    int c = 0;
+    while (v) {
+        c += (int)(v & 1u);
+        v >>= 1;
+    }
+    return c;
+}
+
+/* out[b][k] = (R x)[b][k] for K inputs (K % 32 == 0); signs may be NULL
+   (NULL: D = I, so R = H_32 / sqrt(32)). */
+int or_rht32(const double *x, const uint32_t *signs, int64_t B, int64_t K, double *out)
+{
+    if (K % 32)
+        return -1;
+    const double inv = 1.0 / sqrt(32.0);
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t blk = 0; blk < K / 32; ++blk) {
+            double d[32];
+            for (int i = 0; i < 32; ++i) {
+                int neg = signs ? (int)((signs[blk] >> i) & 1u) : 0;
+                d[i] = (neg ? -1.0 : 1.0) * x[b * K + blk * 32 + i];
+            }
+            for (int i = 0; i < 32; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < 32; ++j)
+                    acc += ((popcount32((uint32_t)(i & j)) & 1) ? -1.0 : 1.0) * d[j];
+                out[b * K + blk * 32 + i] = acc * inv;
+            }
+        }
+    return 0;
+}
+
+/* Element (n, k) of a format-variant matrix (format 1 = ZP4, 2 = SYM8). */
+static double weight_fmt(const uint32_t *P, const uint32_t *params, int64_t K, int format,
+                         int64_t n, int64_t k)
+{
+    int bits = format == 1 ? 4 : 8;
+    int64_t per = 32 / bits;
+    uint32_t word = P[n * (K / per) + k / per];
+    uint32_t q = (word >> (bits * (k % per))) & ((1u << bits) - 1u);
+    uint32_t prm = params[n * (K / 64) + k / 64];
+    double s = or_bf16_to_f64((uint16_t)(prm & 0xFFFFu));
+    if (format == 1)
+        return s * ((double)q - (double)((prm >> 16) & 0xFFu));
+    int sq = q >= 128u ? (int)q - 256 : (int)q;   /* two's complement */
+    return s * (double)sq;
+}
+
+int or_dequant_fmt(const uint32_t *P, const uint32_t *params, int64_t N, int64_t K, int format,
+                   double *W)
+{
+    if ((format != 1 && format != 2) || K % 64)
+        return -1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            W[n * K + k] = weight_fmt(P, params, K, format, n, k);
+    return 0;
+}
+
+/* y = W (R x) (R omitted when signs == NULL and rotate == 0), fp64, k in
+   increasing order; y64 / y16 as or_qgemv. */
+int or_qgemv_fmt(const uint32_t *P, const uint32_t *params, int64_t N, int64_t K, int format,
+                 const uint32_t *signs, int rotate, const uint16_t *x16, int64_t B, double *y64,
+                 uint16_t *y16)
+{
+    if ((format != 1 && format != 2) || K % 64)
+        return -1;
+    double *x = (double *)malloc(sizeof(double) * (size_t)(B * K));
+    double *xr = (double *)malloc(sizeof(double) * (size_t)(B * K));
+    if (!x || !xr) {
+        free(x);
+        free(xr);
+        return -2;
+    }
+    for (int64_t i = 0; i < B * K; ++i)
+        x[i] = or_f16_to_f64(x16[i]);
+    if (rotate)
+        or_rht32(x, signs, B, K, xr);
+    else
+        memcpy(xr, x, sizeof(double) * (size_t)(B * K));
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += weight_fmt(P, params, K, format, n, k) * xr[b * K + k];
+            if (y64)
+                y64[b * N + n] = acc;
+            if (y16)
+                y16[b * N + n] = or_f64_to_f16(acc);
+        }
+    free(x);
+    free(xr);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Router: softmax, top-k, renormalisation                                   */
 /* ------------------------------------------------------------------------ */
 
