@@ -60,7 +60,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["moe_decode", "qgemv", "router", "prefill"],
+    ap.add_argument("--workload", choices=["moe_decode", "qgemv", "qgemv_fmt", "router", "prefill"],
                     default="moe_decode")
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--seed", type=int, default=0)
@@ -451,6 +451,39 @@ def main_other(args):
                 out["results"].append({"N": N, "K": K, "B": Bt, "us": round(ms * 1e3, 3),
                                        "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
                                        "rotated_copies": copies})
+    elif args.workload == "qgemv_fmt":
+        # bf16-scale formats with the block-32 rotation of x, config-1 shapes
+        for fmt, name in ((qmoe.FMT_ZP4_BF16, "zp4_bf16"), (qmoe.FMT_SYM8_BF16, "sym8_bf16")):
+            bits = 4 if fmt == qmoe.FMT_ZP4_BF16 else 8
+            for N in (14336, 4096):
+                K = 4096
+                nbytes = N * K * bits // 8 + N * (K // 64) * 4
+                copies = max(2, int(4 * 126e6 // nbytes) + 1)
+                Ws = []
+                for c in range(copies):
+                    P, prm, sg = synth.qmatrix_fmt(synth.rng(c, N, fmt), N, K, fmt)
+                    Ws.append(qmoe.QMatrixFmt.from_numpy(P, prm, sg, N, K, fmt, device=dev))
+                for Bt in (1, 8):
+                    x = torch.from_numpy(synth.activations(Bt, Bt, K).view(np.float16).copy()).to(dev)
+                    y = torch.empty(Bt, N, dtype=torch.float16, device=dev)
+
+                    def run():
+                        for W in Ws:
+                            qmoe.qgemv_fmt(W, x, y)
+                    run()
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g):
+                        run()
+                    for _ in range(3):
+                        g.replay()
+                    reps = max(10, args.steps // 10)
+                    ms = timed_replays(g.replay, reps) / (reps * copies)
+                    gbs = (nbytes + K // 8 + Bt * K * 2 + Bt * N * 2) / (ms / 1e3) / 1e9
+                    out["results"].append({"format": name, "rotation": True, "N": N, "K": K,
+                                           "B": Bt, "us": round(ms * 1e3, 3),
+                                           "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
+                                           "rotated_copies": copies})
+                del Ws
     elif args.workload == "router":
         P, S, B = synth.router(args.seed)
         R = qmoe.QMatrix.from_numpy(P, S, B, E, H, 8, dev)

@@ -115,6 +115,42 @@ qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch
                          uint16_t *y, int32_t *status_dev, void *stream);
 
 /* ---------------------------------------------------------------------------
+ * Format variants of the dense qGEMV (uzu page, discuss.pytorch.kr, section
+ * "uzu의 모델 변환과 Mirai 양자화 형식": Mirai-M is 4-bit asymmetric with a
+ * 4-bit zero point and a bf16 scale, group 64; Mirai-L is 8-bit symmetric;
+ * both quantise after a random Hadamard transform of block size 32).
+ *   QMOE_FMT_ZP4_BF16:  w = s * (q - z), q 4-bit unsigned codes (packed as
+ *                       qmoe_qmatrix, 8 per word), z the zero point 0..15
+ *   QMOE_FMT_SYM8_BF16: w = s * q, q 8-bit two's-complement codes (4 per word)
+ *   params: uint32 [rows][cols/64], 16-byte aligned: bits 0..15 the bf16
+ *           scale s, bits 16..23 the zero point z (0 for SYM8)
+ *   rht_signs: NULL, or uint32 [cols/32] (4-byte aligned): the weights were
+ *           quantised in a rotated basis and the product is
+ *             y[b] = W (R x[b]),  R = blockdiag(H_32 D / sqrt(32)),
+ *           H_32[i][j] = (-1)^popcount(i & j), D[i][i] = -1 where bit i % 32
+ *           of rht_signs[i / 32] is set.  x must then be 16-byte aligned; the
+ *           rotation runs in fp32 inside the kernel and R x enters the product
+ *           as an fp16 (hi, lo) pair (about 22 significant bits).
+ * batch 1..8; cols a multiple of 64, rows of 8; y fp16 [batch][rows].
+ * Errors as qgemv_affine (INVALID_ARG also for an unknown format).
+ * ------------------------------------------------------------------------- */
+#define QMOE_FMT_ZP4_BF16 1
+#define QMOE_FMT_SYM8_BF16 2
+
+typedef struct qmoe_qmatrix_fmt {
+    const uint32_t *packed;
+    const uint32_t *params;
+    const uint32_t *rht_signs;
+    int32_t rows;
+    int32_t cols;
+    int32_t group;
+    int32_t format;
+} qmoe_qmatrix_fmt;
+
+qmoe_status qgemv_fmt(const qmoe_qmatrix_fmt *W, const uint16_t *x, int32_t batch, uint16_t *y,
+                      int32_t *status_dev, void *stream);
+
+/* ---------------------------------------------------------------------------
  * Router + softmax + top-k + renormalisation ("내부 구조" section: the router
  * runs on resident weights and picks the top-8 experts).
  *   logits[t][e] = sum_k w_router[e][k] x[t][k]    (fp32)

@@ -190,6 +190,47 @@ qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch
     a.N = W->rows;
     a.K = W->cols;
     a.bits = W->bits;
+    a.params = nullptr;
+    a.signs = nullptr;
+    a.fmt = QG_AFFINE;
+    a.x = reinterpret_cast<const __half *>(x);
+    a.B = batch;
+    a.y = reinterpret_cast<__half *>(y);
+    a.status = status_dev ? status_dev : d->status;
+    return cuda_status(launch_qgemv(a, launch_cfg(d, stream)));
+}
+
+qmoe_status qgemv_fmt(const qmoe_qmatrix_fmt *W, const uint16_t *x, int32_t batch, uint16_t *y,
+                      int32_t *status_dev, void *stream)
+{
+    if (!W || !W->packed || !W->params || !x || !y)
+        return QMOE_ERR_INVALID_ARG;
+    if (batch < 1 || batch > 8 || W->rows <= 0 || W->cols <= 0)
+        return QMOE_ERR_INVALID_ARG;
+    if (W->format != QMOE_FMT_ZP4_BF16 && W->format != QMOE_FMT_SYM8_BF16)
+        return QMOE_ERR_INVALID_ARG;
+    if (W->group != kGroup || W->cols % kGroup != 0 || W->rows % 8 != 0)
+        return QMOE_ERR_UNSUPPORTED;
+    if (!aligned(W->packed, 16) || !aligned(W->params, 16) ||
+        (W->rht_signs && !aligned(W->rht_signs, 4)))
+        return QMOE_ERR_ALIGNMENT;
+    if (!aligned(x, W->rht_signs ? 16 : 2) || !aligned(y, 2) ||
+        (status_dev && !aligned(status_dev, 4)))
+        return QMOE_ERR_ALIGNMENT;
+    qmoe_status s;
+    DevState *d;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    QgemvArgs a;
+    a.packed = W->packed;
+    a.scales = nullptr;
+    a.biases = nullptr;
+    a.params = W->params;
+    a.signs = W->rht_signs;
+    a.N = W->rows;
+    a.K = W->cols;
+    a.fmt = W->format == QMOE_FMT_ZP4_BF16 ? QG_ZP4 : QG_SYM8;
+    a.bits = W->format == QMOE_FMT_ZP4_BF16 ? 4 : 8;
     a.x = reinterpret_cast<const __half *>(x);
     a.B = batch;
     a.y = reinterpret_cast<__half *>(y);

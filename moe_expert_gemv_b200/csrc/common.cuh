@@ -403,6 +403,56 @@ __device__ __forceinline__ void mma_group_s8(float (&r)[4], uint4 wa, uint4 wb, 
         r[i] = c[i] + d[i];
 }
 
+// The same products with an activation held as an fp16 (hi, lo) pair: the
+// codes are dequantised once and both parts accumulate, i.e. the result is
+// that of mma_group_s4 / mma_group_s8 applied to hi + lo.
+__device__ __forceinline__ void mma_group_s4_hilo(float (&r)[4], uint2 wa, uint2 wb, uint4 h0,
+                                                  uint4 h1, uint4 l0, uint4 l1)
+{
+    uint32_t pa[8], pb[8];
+    dequant4s_word(wa.x, pa);
+    dequant4s_word(wa.y, pa + 4);
+    dequant4s_word(wb.x, pb);
+    dequant4s_word(wb.y, pb + 4);
+    float c[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
+    mma_16816(c, pa[0], pb[0], pa[2], pb[2], h0.x, h0.y);
+    mma_16816(e, pa[1], pb[1], pa[3], pb[3], h1.x, h1.y);
+    mma_16816(c, pa[4], pb[4], pa[6], pb[6], h0.z, h0.w);
+    mma_16816(e, pa[5], pb[5], pa[7], pb[7], h1.z, h1.w);
+    mma_16816(c, pa[0], pb[0], pa[2], pb[2], l0.x, l0.y);
+    mma_16816(e, pa[1], pb[1], pa[3], pb[3], l1.x, l1.y);
+    mma_16816(c, pa[4], pb[4], pa[6], pb[6], l0.z, l0.w);
+    mma_16816(e, pa[5], pb[5], pa[7], pb[7], l1.z, l1.w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        r[i] = fmaf(16.f, c[i], e[i]);
+}
+__device__ __forceinline__ void mma_group_s8_hilo(float (&r)[4], uint4 wa, uint4 wb, uint4 h0,
+                                                  uint4 h1, uint4 l0, uint4 l1)
+{
+    uint32_t pa[8], pb[8];
+    dequant8s_word(wa.x, pa);
+    dequant8s_word(wb.x, pb);
+    dequant8s_word(wa.y, pa + 2);
+    dequant8s_word(wb.y, pb + 2);
+    dequant8s_word(wa.z, pa + 4);
+    dequant8s_word(wb.z, pb + 4);
+    dequant8s_word(wa.w, pa + 6);
+    dequant8s_word(wb.w, pb + 6);
+    float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
+    mma_16816(c, pa[0], pb[0], pa[1], pb[1], h0.x, h0.y);
+    mma_16816(d, pa[2], pb[2], pa[3], pb[3], h0.z, h0.w);
+    mma_16816(c, pa[4], pb[4], pa[5], pb[5], h1.x, h1.y);
+    mma_16816(d, pa[6], pb[6], pa[7], pb[7], h1.z, h1.w);
+    mma_16816(c, pa[0], pb[0], pa[1], pb[1], l0.x, l0.y);
+    mma_16816(d, pa[2], pb[2], pa[3], pb[3], l0.z, l0.w);
+    mma_16816(c, pa[4], pb[4], pa[5], pb[5], l1.x, l1.y);
+    mma_16816(d, pa[6], pb[6], pa[7], pb[7], l1.z, l1.w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        r[i] = c[i] + d[i];
+}
+
 // Smem row stride (in 32-bit words) for a tile of `cols` inputs so that the
 // fragment loads of tile_group are free of bank conflicts: the stride must be
 // 8 or 24 (mod 32) words for 4-bit (8-byte loads by 16 lanes) and 16 (mod 32)
@@ -481,38 +531,102 @@ __device__ __forceinline__ void stage_x(uint4 *xs, float *xsum, int G, int ncol,
 // All `nthreads` threads starting at `tid` take part.  The sum of (column n,
 // group g) goes to xsum[g * sum_stride + n]; with sum_stride 8 (the
 // tile_group layout) columns ncol..7 of the sums are zeroed.
-template <int KIND>
+// With ROT, each 32-input block is first rotated: x' = H_32 (D x) / sqrt(32)
+// (Sylvester Hadamard, D = diag(+-1) from bit i of signs[k / 32], set = -1),
+// computed in fp32 by the thread that owns the block, and kept as an fp16
+// pair: hi = fp16(x') in xs, lo = fp16(x' - hi) in xs_lo (same layout); the
+// sums are those of hi + lo.  (fp16 x' alone would add up to 2^-12 relative
+// error per input, far more than the products of the exact codes.)
+template <int KIND, bool ROT = false>
 __device__ __forceinline__ void stage_x_groups(uint4 *xs, float *xsum, int G, int ncol,
                                                const __half *x, int K, int tid, int nthreads,
-                                               int sum_stride = 8)
+                                               int sum_stride = 8,
+                                               const uint32_t *signs = nullptr,
+                                               uint4 *xs_lo = nullptr)
 {
     for (int t = tid; t < ncol * G; t += nthreads) {
         const int n = t / G, g = t - n * G;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)n * K + (size_t)g * kGroup);
-        uint4 raw[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            raw[i] = __ldg(src + i);
-        const __half *hv = reinterpret_cast<const __half *>(raw);
         float sum = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const float2 f = __half22float2(reinterpret_cast<const __half2 *>(raw)[i]);
-            sum += f.x + f.y;
-        }
+        for (int blk = 0; blk < 2; ++blk) {   // the group's two 32-input blocks
+            uint4 raw[4];
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+            for (int i = 0; i < 4; ++i)
+                raw[i] = __ldg(src + 4 * blk + i);
+            if (ROT) {
+                float v[32];
 #pragma unroll
-            for (int tig = 0; tig < 4; ++tig) {
-                uint32_t w[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const __half lo = hv[16 * tig + xperm(KIND, 8 * h + 2 * i)];
-                    const __half hi = hv[16 * tig + xperm(KIND, 8 * h + 2 * i + 1)];
-                    w[i] = h2_as_u32(__halves2half2(lo, hi));
+                for (int i = 0; i < 16; ++i) {
+                    const float2 f = __half22float2(reinterpret_cast<const __half2 *>(raw)[i]);
+                    v[2 * i] = f.x;
+                    v[2 * i + 1] = f.y;
                 }
-                xs[((g * 2 + h) * ncol + n) * 4 + tig] = make_uint4(w[0], w[1], w[2], w[3]);
+                const uint32_t sg = __ldg(signs + 2 * g + blk);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if ((sg >> i) & 1u)
+                        v[i] = -v[i];
+#pragma unroll
+                for (int h = 1; h < 32; h <<= 1)   // Walsh-Hadamard butterflies
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if ((i & h) == 0) {
+                            const float a = v[i], b = v[i + h];
+                            v[i] = a + b;
+                            v[i + h] = a - b;
+                        }
+                const float inv = 0.17677669529663687f;   // 1 / sqrt(32)
+                uint4 rlo[4];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float a = v[2 * i] * inv, b = v[2 * i + 1] * inv;
+                    const __half2 hh = __floats2half2_rn(a, b);
+                    const float2 back = __half22float2(hh);
+                    reinterpret_cast<__half2 *>(raw)[i] = hh;
+                    reinterpret_cast<__half2 *>(rlo)[i] = __floats2half2_rn(a - back.x, b - back.y);
+                }
+                const __half *lv = reinterpret_cast<const __half *>(rlo);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 f = __half22float2(reinterpret_cast<const __half2 *>(rlo)[i]);
+                    sum += f.x + f.y;
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int tl = 0; tl < 2; ++tl) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const __half lo = lv[16 * tl + xperm(KIND, 8 * h + 2 * i)];
+                            const __half hi = lv[16 * tl + xperm(KIND, 8 * h + 2 * i + 1)];
+                            w[i] = h2_as_u32(__halves2half2(lo, hi));
+                        }
+                        xs_lo[((g * 2 + h) * ncol + n) * 4 + 2 * blk + tl] =
+                            make_uint4(w[0], w[1], w[2], w[3]);
+                    }
             }
+            const __half *hv = reinterpret_cast<const __half *>(raw);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float2 f = __half22float2(reinterpret_cast<const __half2 *>(raw)[i]);
+                sum += f.x + f.y;
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int tl = 0; tl < 2; ++tl) {   // fragment slots tig = 2 blk + tl
+                    uint32_t w[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const __half lo = hv[16 * tl + xperm(KIND, 8 * h + 2 * i)];
+                        const __half hi = hv[16 * tl + xperm(KIND, 8 * h + 2 * i + 1)];
+                        w[i] = h2_as_u32(__halves2half2(lo, hi));
+                    }
+                    xs[((g * 2 + h) * ncol + n) * 4 + 2 * blk + tl] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+        }
         xsum[g * sum_stride + n] = sum;
     }
     if (sum_stride == 8)

@@ -18,10 +18,19 @@ struct LaunchCfg {
 };
 
 // ------------------------------------------------------------ dense qGEMV --
+// weight formats of the dense qGEMV
+enum QgemvFormat {
+    QG_AFFINE = 0,   // w = s*q + b, fp16 scale and bias per group
+    QG_ZP4 = 1,      // w = s*(q - z), bf16 scale, 4-bit zero point: params word s | z << 16
+    QG_SYM8 = 2,     // w = s*q, two's-complement 8-bit codes, bf16 scale in params
+};
+
 struct QgemvArgs {
     const uint32_t *packed;
-    const __half *scales, *biases;
-    int N, K, bits;
+    const __half *scales, *biases;   // QG_AFFINE
+    const uint32_t *params;          // QG_ZP4 / QG_SYM8: [N][K/64]
+    const uint32_t *signs;           // block-32 Hadamard rotation of x, or null
+    int N, K, bits, fmt;
     const __half *x;   // [B][K]
     int B;
     __half *y;         // [B][N]

@@ -176,30 +176,6 @@ __device__ __forceinline__ void issue_tile(unsigned char *dst, const PfStage &st
             bulk_g2s(dst + (size_t)r * st.S * 4, packed + (row0 + r) * Kw, row_bytes, bar, pol);
 }
 
-// Subnormal-code product of rows (gid, gid+8) with two activation columns
-// sets (the hi and lo fp16 parts of h) summed: 2^-20 * sum_k q (hi + lo).
-__device__ __forceinline__ void mma_group_s4_hilo(float (&r)[4], uint2 wa, uint2 wb, uint4 h0,
-                                                  uint4 h1, uint4 l0, uint4 l1)
-{
-    uint32_t pa[8], pb[8];
-    dequant4s_word(wa.x, pa);
-    dequant4s_word(wa.y, pa + 4);
-    dequant4s_word(wb.x, pb);
-    dequant4s_word(wb.y, pb + 4);
-    float c[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
-    mma_16816(c, pa[0], pb[0], pa[2], pb[2], h0.x, h0.y);
-    mma_16816(e, pa[1], pb[1], pa[3], pb[3], h1.x, h1.y);
-    mma_16816(c, pa[4], pb[4], pa[6], pb[6], h0.z, h0.w);
-    mma_16816(e, pa[5], pb[5], pa[7], pb[7], h1.z, h1.w);
-    mma_16816(c, pa[0], pb[0], pa[2], pb[2], l0.x, l0.y);
-    mma_16816(e, pa[1], pb[1], pa[3], pb[3], l1.x, l1.y);
-    mma_16816(c, pa[4], pb[4], pa[6], pb[6], l0.z, l0.w);
-    mma_16816(e, pa[5], pb[5], pa[7], pb[7], l1.z, l1.w);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        r[i] = fmaf(16.f, c[i], e[i]);
-}
-
 // h of intermediate index kidx at position pos from its gate and up values,
 // stored as fp16 (hi, lo) in the fragment order of the down projection:
 // [g][k half][column: 0 = hi, 1 = lo][tig][8], k order xperm(kPermS4, .)

@@ -36,14 +36,15 @@ constexpr int QG_MAX_STAGES = 8;
 
 struct QgLayout {
     int G, S;
-    size_t xs_off, xsum_off, red_off, bar_off, stage_off;
+    size_t xs_off, xslo_off, xsum_off, red_off, bar_off, stage_off;
     size_t codes_bytes, sb_bytes, stage_bytes, total;
 };
 
 // Offsets from a 1024-byte aligned base (the swizzled TMA destination must be
 // 1024-byte aligned); `total` includes the slack to align the dynamic
 // shared-memory window.
-__host__ __device__ inline QgLayout qg_layout(int K, int bits, int ncol, int NS, bool swz)
+__host__ __device__ inline QgLayout qg_layout(int K, int bits, int ncol, int NS, bool swz,
+                                               bool rot = false)
 {
     QgLayout L;
     L.G = K / kGroup;
@@ -51,6 +52,9 @@ __host__ __device__ inline QgLayout qg_layout(int K, int bits, int ncol, int NS,
     size_t off = 0;
     L.xs_off = off;
     off += (size_t)L.G * 2 * ncol * 4 * 16;
+    L.xslo_off = off;   // lo parts of a rotated x
+    if (rot)
+        off += (size_t)L.G * 2 * ncol * 4 * 16;
     L.xsum_off = off;
     off += (size_t)L.G * 8 * 4;
     off = (off + 15) & ~(size_t)15;
@@ -68,14 +72,24 @@ __host__ __device__ inline QgLayout qg_layout(int K, int bits, int ncol, int NS,
     return L;
 }
 
-template <int BITS, bool SWZ>
+// scale and folded-bias factor of one parameter word of the bf16 formats:
+// ZP4 w = s(q - z) -> (s, -s z); SYM8 w = s(q' - 128) with q' = q + 128 -> (s, -128 s)
+template <int FMT>
+__device__ __forceinline__ void fmt_scale_bias(uint32_t p, float &s, float &b)
+{
+    s = __uint_as_float(p << 16);
+    b = FMT == QG_ZP4 ? -s * (float)((p >> 16) & 0xFFu) : -128.f * s;
+}
+
+template <int BITS, bool SWZ, int FMT, bool ROT>
 __global__ void __launch_bounds__(QG_THREADS, 1)
     qgemv_kernel(QgemvArgs a, int NS, const __grid_constant__ CUtensorMap codes_map)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const QgLayout L = qg_layout(a.K, BITS, a.B, NS, SWZ);
+    const QgLayout L = qg_layout(a.K, BITS, a.B, NS, SWZ, ROT);
     uint4 *xs = reinterpret_cast<uint4 *>(smem + L.xs_off);
+    uint4 *xs_lo = reinterpret_cast<uint4 *>(smem + L.xslo_off);
     float *xsum = reinterpret_cast<float *>(smem + L.xsum_off);
     float4 *red = reinterpret_cast<float4 *>(smem + L.red_off);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bar_off);
@@ -125,9 +139,14 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                         bulk_g2s(stage + (size_t)r * L.S * 4, a.packed + (size_t)(r0 + r) * Kw,
                                  row_bytes, &full[st], pol);
                 }
-                bulk_g2s(stage + L.codes_bytes, a.scales + (size_t)r0 * L.G, sb, &full[st], pol);
-                bulk_g2s(stage + L.codes_bytes + L.sb_bytes, a.biases + (size_t)r0 * L.G, sb,
-                         &full[st], pol);
+                if (FMT == QG_AFFINE) {
+                    bulk_g2s(stage + L.codes_bytes, a.scales + (size_t)r0 * L.G, sb, &full[st], pol);
+                    bulk_g2s(stage + L.codes_bytes + L.sb_bytes, a.biases + (size_t)r0 * L.G, sb,
+                             &full[st], pol);
+                } else {   // one parameter word per group: the same bytes as scale + bias
+                    bulk_g2s(stage + L.codes_bytes, a.params + (size_t)r0 * L.G, 2 * sb, &full[st],
+                             pol);
+                }
                 last_use[st] = use;
             }
             // no copy may still be landing when the CTA exits
@@ -144,7 +163,9 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
     const int ctid = threadIdx.x;
     constexpr int KIND = BITS == 4 ? kPermS4 : 8;
     constexpr float kCodeScale = BITS == 4 ? kSub20 : kSub24;   // undoes the subnormal codes
-    if ((reinterpret_cast<uintptr_t>(a.x) & 15u) == 0)
+    if (ROT)
+        stage_x_groups<KIND, true>(xs, xsum, L.G, a.B, a.x, a.K, ctid, QG_CT, 8, a.signs, xs_lo);
+    else if ((reinterpret_cast<uintptr_t>(a.x) & 15u) == 0)
         stage_x_groups<KIND>(xs, xsum, L.G, a.B, a.x, a.K, ctid, QG_CT);
     else
         stage_x<KIND>(xs, xsum, L.G, a.B, 1,
@@ -176,16 +197,40 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
             // one group from its fragment addresses (rows gid, gid+8)
             auto group = [&](int g, const void *fa, const void *fb, float s_lo, float s_hi,
                              float b_lo, float b_hi) {
-                uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
+                uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0, l0 = x0, l1 = x0;
                 if (gid < a.B) {
                     x0 = xs[((g * 2 + 0) * a.B + gid) * 4 + tig];
                     x1 = xs[((g * 2 + 1) * a.B + gid) * 4 + tig];
+                    if (ROT) {
+                        l0 = xs_lo[((g * 2 + 0) * a.B + gid) * 4 + tig];
+                        l1 = xs_lo[((g * 2 + 1) * a.B + gid) * 4 + tig];
+                    }
                 }
                 float r[4];
-                if (BITS == 4)
+                if (BITS == 4 && ROT)
+                    mma_group_s4_hilo(r, *reinterpret_cast<const uint2 *>(fa),
+                                      *reinterpret_cast<const uint2 *>(fb), x0, x1, l0, l1);
+                else if (BITS == 4)
                     mma_group_s4(r, *reinterpret_cast<const uint2 *>(fa),
                                  *reinterpret_cast<const uint2 *>(fb), x0, x1);
-                else
+                else if (FMT == QG_SYM8) {
+                    // two's-complement byte q -> q + 128 = byte ^ 0x80; the
+                    // -128 s offset joins the folded bias
+                    uint4 wa = *reinterpret_cast<const uint4 *>(fa);
+                    uint4 wb = *reinterpret_cast<const uint4 *>(fb);
+                    wa.x ^= 0x80808080u;
+                    wa.y ^= 0x80808080u;
+                    wa.z ^= 0x80808080u;
+                    wa.w ^= 0x80808080u;
+                    wb.x ^= 0x80808080u;
+                    wb.y ^= 0x80808080u;
+                    wb.z ^= 0x80808080u;
+                    wb.w ^= 0x80808080u;
+                    if (ROT)
+                        mma_group_s8_hilo(r, wa, wb, x0, x1, l0, l1);
+                    else
+                        mma_group_s8(r, wa, wb, x0, x1);
+                } else
                     mma_group_s8(r, *reinterpret_cast<const uint4 *>(fa),
                                  *reinterpret_cast<const uint4 *>(fb), x0, x1);
                 const float2 X = *reinterpret_cast<const float2 *>(xsum + g * 8 + 2 * tig);
@@ -222,28 +267,51 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                 for (int gb = g0; gb < g1; gb += 4) {
                     const unsigned char *base =
                         stage + (SWZ ? (gb / GPC) * 2048 : gb * (BITS == 4 ? 32 : 64));
-                    const uint2 slo = *reinterpret_cast<const uint2 *>(sc + gid * L.G + gb);
-                    const uint2 shi = *reinterpret_cast<const uint2 *>(sc + (gid + 8) * L.G + gb);
-                    const uint2 blo = *reinterpret_cast<const uint2 *>(bi + gid * L.G + gb);
-                    const uint2 bhi = *reinterpret_cast<const uint2 *>(bi + (gid + 8) * L.G + gb);
-                    const uint32_t sl[2] = {slo.x, slo.y}, sh[2] = {shi.x, shi.y};
-                    const uint32_t bl[2] = {blo.x, blo.y}, bh[2] = {bhi.x, bhi.y};
+                    if (FMT == QG_AFFINE) {
+                        const uint2 slo = *reinterpret_cast<const uint2 *>(sc + gid * L.G + gb);
+                        const uint2 shi = *reinterpret_cast<const uint2 *>(sc + (gid + 8) * L.G + gb);
+                        const uint2 blo = *reinterpret_cast<const uint2 *>(bi + gid * L.G + gb);
+                        const uint2 bhi = *reinterpret_cast<const uint2 *>(bi + (gid + 8) * L.G + gb);
+                        const uint32_t sl[2] = {slo.x, slo.y}, sh[2] = {shi.x, shi.y};
+                        const uint32_t bl[2] = {blo.x, blo.y}, bh[2] = {bhi.x, bhi.y};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float2 fsl = __half22float2(u32_as_h2(sl[j >> 1]));
-                        const float2 fsh = __half22float2(u32_as_h2(sh[j >> 1]));
-                        const float2 fbl = __half22float2(u32_as_h2(bl[j >> 1]));
-                        const float2 fbh = __half22float2(u32_as_h2(bh[j >> 1]));
-                        group(gb + j, base + off[j], base + off[j] + row8, (j & 1) ? fsl.y : fsl.x,
-                              (j & 1) ? fsh.y : fsh.x, (j & 1) ? fbl.y : fbl.x,
-                              (j & 1) ? fbh.y : fbh.x);
+                        for (int j = 0; j < 4; ++j) {
+                            const float2 fsl = __half22float2(u32_as_h2(sl[j >> 1]));
+                            const float2 fsh = __half22float2(u32_as_h2(sh[j >> 1]));
+                            const float2 fbl = __half22float2(u32_as_h2(bl[j >> 1]));
+                            const float2 fbh = __half22float2(u32_as_h2(bh[j >> 1]));
+                            group(gb + j, base + off[j], base + off[j] + row8,
+                                  (j & 1) ? fsl.y : fsl.x, (j & 1) ? fsh.y : fsh.x,
+                                  (j & 1) ? fbl.y : fbl.x, (j & 1) ? fbh.y : fbh.x);
+                        }
+                    } else {
+                        const uint32_t *prm = reinterpret_cast<const uint32_t *>(sc);
+                        const uint4 plo = *reinterpret_cast<const uint4 *>(prm + gid * L.G + gb);
+                        const uint4 phi = *reinterpret_cast<const uint4 *>(prm + (gid + 8) * L.G + gb);
+                        const uint32_t pl[4] = {plo.x, plo.y, plo.z, plo.w};
+                        const uint32_t ph[4] = {phi.x, phi.y, phi.z, phi.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            float s_lo, s_hi, b_lo, b_hi;
+                            fmt_scale_bias<FMT>(pl[j], s_lo, b_lo);
+                            fmt_scale_bias<FMT>(ph[j], s_hi, b_hi);
+                            group(gb + j, base + off[j], base + off[j] + row8, s_lo, s_hi, b_lo, b_hi);
+                        }
                     }
                 }
-            } else {
+            } else if (FMT == QG_AFFINE) {
                 for (int g = g0; g < g1; ++g)
                     group(g, frag(gid, g), frag(gid + 8, g), __half2float(sc[gid * L.G + g]),
                           __half2float(sc[(gid + 8) * L.G + g]), __half2float(bi[gid * L.G + g]),
                           __half2float(bi[(gid + 8) * L.G + g]));
+            } else {
+                const uint32_t *prm = reinterpret_cast<const uint32_t *>(sc);
+                for (int g = g0; g < g1; ++g) {
+                    float s_lo, s_hi, b_lo, b_hi;
+                    fmt_scale_bias<FMT>(prm[gid * L.G + g], s_lo, b_lo);
+                    fmt_scale_bias<FMT>(prm[(gid + 8) * L.G + g], s_hi, b_hi);
+                    group(g, frag(gid, g), frag(gid + 8, g), s_lo, s_hi, b_lo, b_hi);
+                }
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -281,23 +349,43 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
     }
 }
 
-template <int BITS, bool SWZ>
+template <int BITS, bool SWZ, int FMT, bool ROT>
 cudaError_t launch_qgemv_t(const QgemvArgs &a, const LaunchCfg &c, const CUtensorMap &m)
 {
     const size_t budget = 227 * 1024;
-    const QgLayout L0 = qg_layout(a.K, BITS, a.B, 0, SWZ);
-    if (L0.total + 2 * L0.stage_bytes > budget)
+    const QgLayout L0 = qg_layout(a.K, BITS, a.B, 0, SWZ, ROT);
+    // one stage still works (copy and compute then alternate); it is only
+    // needed by the largest rotated 8-bit rows at batch 8
+    if (L0.total + L0.stage_bytes > budget)
         return cudaErrorInvalidValue;
     int NS = (int)((budget - L0.total) / L0.stage_bytes);
     NS = NS > QG_MAX_STAGES ? QG_MAX_STAGES : NS;
-    const QgLayout L = qg_layout(a.K, BITS, a.B, NS, SWZ);
+    const QgLayout L = qg_layout(a.K, BITS, a.B, NS, SWZ, ROT);
     const int n_items = (a.N + 15) / 16;
     const int grid = n_items < c.num_sms ? n_items : c.num_sms;
     cudaError_t e;
-    if ((e = set_smem(qgemv_kernel<BITS, SWZ>, L.total)) != cudaSuccess)
+    if ((e = set_smem(qgemv_kernel<BITS, SWZ, FMT, ROT>, L.total)) != cudaSuccess)
         return e;
-    return launch_ex(qgemv_kernel<BITS, SWZ>, dim3(grid), dim3(QG_THREADS), L.total, c, 1, a, NS,
-                     m);
+    return launch_ex(qgemv_kernel<BITS, SWZ, FMT, ROT>, dim3(grid), dim3(QG_THREADS), L.total, c, 1,
+                     a, NS, m);
+}
+
+template <bool SWZ>
+cudaError_t launch_qgemv_fmt(const QgemvArgs &a, const LaunchCfg &c, const CUtensorMap &m)
+{
+    const bool rot = a.signs != nullptr;
+    switch (a.fmt) {
+    case QG_AFFINE:
+        return a.bits == 4 ? launch_qgemv_t<4, SWZ, QG_AFFINE, false>(a, c, m)
+                           : launch_qgemv_t<8, SWZ, QG_AFFINE, false>(a, c, m);
+    case QG_ZP4:
+        return rot ? launch_qgemv_t<4, SWZ, QG_ZP4, true>(a, c, m)
+                   : launch_qgemv_t<4, SWZ, QG_ZP4, false>(a, c, m);
+    case QG_SYM8:
+        return rot ? launch_qgemv_t<8, SWZ, QG_SYM8, true>(a, c, m)
+                   : launch_qgemv_t<8, SWZ, QG_SYM8, false>(a, c, m);
+    }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -347,10 +435,8 @@ cudaError_t launch_qgemv(const QgemvArgs &a, const LaunchCfg &c)
     CUtensorMap m;
     memset(&m, 0, sizeof(m));
     const bool swz = encode_codes_map(&m, a.packed, a.N, Kw, 16) &&
-                     qg_layout(a.K, a.bits, a.B, 2, true).total <= 227 * 1024;
-    if (a.bits == 4)
-        return swz ? launch_qgemv_t<4, true>(a, c, m) : launch_qgemv_t<4, false>(a, c, m);
-    return swz ? launch_qgemv_t<8, true>(a, c, m) : launch_qgemv_t<8, false>(a, c, m);
+                     qg_layout(a.K, a.bits, a.B, 1, true, a.signs != nullptr).total <= 227 * 1024;
+    return swz ? launch_qgemv_fmt<true>(a, c, m) : launch_qgemv_fmt<false>(a, c, m);
 }
 
 }  // namespace qmoe

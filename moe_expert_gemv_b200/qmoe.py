@@ -10,6 +10,7 @@ is missing or the device is not an sm_100 GPU the calls fail loudly.
 import ctypes
 import os
 
+import numpy as np
 import torch
 
 from . import build as _build
@@ -51,6 +52,7 @@ def lib():
         p, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
         sig = {
             "qgemv_affine": [p, p, i32, p, p, p],
+            "qgemv_fmt": [p, p, i32, p, p, p],
             "moe_router_topk": [p, p, i32, i32, p, p, p, p, p],
             "moe_expert_workspace_bytes": [p, i32],
             "moe_expert_qmlp": [p, p, p, p, i32, p, p, sz, p, p],
@@ -144,6 +146,42 @@ class QMatrix:
         return cls(packed, scales, biases, rows, cols, bits, stack)
 
 
+FMT_ZP4_BF16, FMT_SYM8_BF16 = 1, 2
+
+
+class CQMatrixFmt(ctypes.Structure):
+    _fields_ = [("packed", ctypes.c_void_p), ("params", ctypes.c_void_p),
+                ("rht_signs", ctypes.c_void_p), ("rows", ctypes.c_int32),
+                ("cols", ctypes.c_int32), ("group", ctypes.c_int32), ("format", ctypes.c_int32)]
+
+
+class QMatrixFmt:
+    """A bf16-scale format-variant matrix on the GPU (zero-point 4-bit or
+    symmetric 8-bit), optionally with the block-32 Hadamard rotation signs.
+
+    packed: int32 [rows, cols*bits/32]; params: int32 [rows, cols/64];
+    signs: int32 [cols/32] or None."""
+
+    def __init__(self, packed, params, signs, rows, cols, fmt):
+        if fmt not in (FMT_ZP4_BF16, FMT_SYM8_BF16):
+            raise ValueError("unknown format %r" % (fmt,))
+        bits = 4 if fmt == FMT_ZP4_BF16 else 8
+        _need(packed, torch.int32, "packed", (rows, cols * bits // 32))
+        _need(params, torch.int32, "params", (rows, cols // 64))
+        if signs is not None:
+            _need(signs, torch.int32, "signs", (cols // 32,))
+        self.packed, self.params, self.signs = packed, params, signs
+        self.rows, self.cols, self.fmt, self.bits = rows, cols, fmt, bits
+        self.c = CQMatrixFmt(packed.data_ptr(), params.data_ptr(),
+                             signs.data_ptr() if signs is not None else None, rows, cols, 64, fmt)
+
+    @classmethod
+    def from_numpy(cls, P, params, signs, rows, cols, fmt, rotate=True, device="cuda"):
+        """From uint32 numpy arrays; `rotate` False drops the rotation."""
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.uint32).view("int32").copy()).to(device)
+        return cls(t(P), t(params), t(signs) if rotate else None, rows, cols, fmt)
+
+
 class MoELayer:
     """Routed experts (stacked gate/up/down) + shared expert (+ optional router)."""
 
@@ -180,6 +218,19 @@ def qgemv_affine(W, x, y=None, status=None):
     _need(y, torch.float16, "y", (x2.shape[0], W.rows))
     _check(lib().qgemv_affine(ctypes.byref(W.c), _ptr(x2), x2.shape[0], _ptr(y), _ptr(status),
                               _stream()), "qgemv_affine")
+    return y
+
+
+def qgemv_fmt(W, x, y=None, status=None):
+    """y[b] = W (R x[b]) (R the rotation when W has signs) for x [B][K]
+    float16 (B <= 8), W a QMatrixFmt.  Returns y [B][N] float16."""
+    x = _need(x, torch.float16, "x")
+    x2 = x.reshape(-1, W.cols)
+    if y is None:
+        y = torch.empty(x2.shape[0], W.rows, dtype=torch.float16, device=x.device)
+    _need(y, torch.float16, "y", (x2.shape[0], W.rows))
+    _check(lib().qgemv_fmt(ctypes.byref(W.c), _ptr(x2), x2.shape[0], _ptr(y), _ptr(status),
+                           _stream()), "qgemv_fmt")
     return y
 
 
