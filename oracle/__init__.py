@@ -60,6 +60,8 @@ def lib():
         L.or_rht32.argtypes = [p, p, i64, i64, p]
         L.or_dequant_fmt.argtypes = [p, p, i64, i64, ctypes.c_int, p]
         L.or_qgemv_fmt.argtypes = [p, p, i64, i64, ctypes.c_int, p, ctypes.c_int, p, i64, p, p]
+        L.or_lfu_step.argtypes = [i64, p, p, p, i64, p, p, p]
+        L.or_lfu_step.restype = i64
         for name in ("or_unpack", "or_pack", "or_dequant", "or_qgemv", "or_router",
                      "or_topk_from_logits", "or_expert", "or_moe_layer", "or_group"):
             getattr(L, name).restype = ctypes.c_int
@@ -254,3 +256,26 @@ def group(idx, E):
     pairs = np.empty(T * k, dtype=np.int32)
     _check(lib().or_group(_ptr(idx), T, k, E, _ptr(counts), _ptr(offsets), _ptr(pairs)), "group")
     return counts, offsets, pairs
+
+
+class LfuCache:
+    """The per-layer LFU expert cache plan (see or_lfu_step in oracle.c)."""
+
+    def __init__(self, nslots=16):
+        self.nslots = nslots
+        self.expert = np.full(nslots, -1, np.int32)
+        self.count = np.zeros(nslots, np.int64)
+
+    def step(self, ids):
+        """-> (slot_of [k], misses [(expert, slot), ...])."""
+        ids = _c(np.asarray(ids, np.int32), np.int32)
+        k = ids.size
+        slot_of = np.empty(k, np.int32)
+        me = np.empty(max(k, 1), np.int32)
+        ms = np.empty(max(k, 1), np.int32)
+        nm = lib().or_lfu_step(self.nslots, _ptr(self.expert), _ptr(self.count), _ptr(ids), k,
+                               _ptr(slot_of), _ptr(me), _ptr(ms))
+        if nm < 0:
+            raise ValueError("k > nslots or repeated ids")
+        return slot_of, list(zip(me[:nm].tolist(), ms[:nm].tolist()))
+

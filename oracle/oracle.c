@@ -556,3 +556,67 @@ int or_group(const int32_t *idx, int64_t T, int64_t k, int64_t E,
     free(fill);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Expert cache: the per-layer 16-slot LFU plan                               */
+/* ------------------------------------------------------------------------ */
+/* TurboFieldfare article, section "내부 구조가 진짜 흥미로운 부분": the CPU
+   takes the router's top-8 expert ids and plans the misses against the
+   layer's 16-slot LFU cache; missed experts are read into the cache before
+   the routed experts run.
+   Readings (the page names the policy only):
+     - a slot holds one expert and a use count; a hit adds one to the count;
+       an expert loaded on a miss starts at one; an evicted expert's count is
+       forgotten;
+     - the token's hits are found first (they stay), then its misses are
+       placed in the order the ids are given: into the lowest-index empty
+       slot, else into the unpinned slot with the smallest count, ties to the
+       lowest index (slots holding an expert of this token are pinned).
+   One step: slot_of[j] = slot of ids[j]; misses listed in order as
+   (expert, slot) pairs; returns the number of misses, or -1 if k > nslots
+   or the ids repeat. */
+int64_t or_lfu_step(int64_t nslots, int32_t *slot_expert, int64_t *slot_count,
+                    const int32_t *ids, int64_t k, int32_t *slot_of, int32_t *miss_expert,
+                    int32_t *miss_slot)
+{
+    if (k > nslots)
+        return -1;
+    for (int64_t a = 0; a < k; ++a)
+        for (int64_t b = a + 1; b < k; ++b)
+            if (ids[a] == ids[b])
+                return -1;
+    int pinned[256];
+    for (int64_t s = 0; s < nslots; ++s)
+        pinned[s] = 0;
+    for (int64_t j = 0; j < k; ++j) {
+        slot_of[j] = -1;
+        for (int64_t s = 0; s < nslots; ++s)
+            if (slot_expert[s] == ids[j]) {
+                slot_of[j] = (int32_t)s;
+                slot_count[s] += 1;
+                pinned[s] = 1;
+            }
+    }
+    int64_t nm = 0;
+    for (int64_t j = 0; j < k; ++j) {
+        if (slot_of[j] >= 0)
+            continue;
+        int64_t v = -1;
+        for (int64_t s = 0; s < nslots && v < 0; ++s)
+            if (slot_expert[s] < 0 && !pinned[s])
+                v = s;
+        if (v < 0)
+            for (int64_t s = 0; s < nslots; ++s)
+                if (!pinned[s] && (v < 0 || slot_count[s] < slot_count[v]))
+                    v = s;
+        slot_expert[v] = ids[j];
+        slot_count[v] = 1;
+        pinned[v] = 1;
+        slot_of[j] = (int32_t)v;
+        miss_expert[nm] = ids[j];
+        miss_slot[nm] = (int32_t)v;
+        ++nm;
+    }
+    return nm;
+}
+
