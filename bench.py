@@ -60,7 +60,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["moe_decode", "qgemv", "qgemv_fmt", "router", "prefill"],
+    ap.add_argument("--workload", choices=["moe_decode", "qgemv", "qgemv_fmt", "router", "prefill",
+                                           "expert_cache"],
                     default="moe_decode")
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--seed", type=int, default=0)
@@ -484,6 +485,34 @@ def main_other(args):
                                            "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
                                            "rotated_copies": copies})
                 del Ws
+    elif args.workload == "expert_cache":
+        # one config-3 layer with its routed experts in pinned host memory and
+        # 16 device slots; decode tokens whose routing locality is set by rho
+        m = synth.moe_layer(args.seed, 0)
+        for rho in (0.0, 0.9, 0.99):
+            layer = qmoe.ExpertCacheLayer(m, E, H, I, nslots=16, device=dev)
+            T = 48
+            x16 = synth.correlated_tokens(args.seed, T, H, rho)
+            xs = torch.from_numpy(x16.view(np.float16).copy()).to(dev)
+            y = torch.empty(H, dtype=torch.float16, device=dev)
+            for t in range(8):   # warm-up: fills the cache
+                layer.forward(xs[t], TOPK, y)
+            h0, m0, b0, _ = layer.stats()
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            for t in range(8, T):
+                layer.forward(xs[t], TOPK, y)
+            torch.cuda.synchronize()
+            el = time.perf_counter() - t0
+            h1, m1, b1, _ = layer.stats()
+            n = T - 8
+            out["results"].append({
+                "rho": rho, "tokens": n, "us_per_layer": round(el / n * 1e6, 1),
+                "layers_per_s": round(n / el, 1),
+                "hit_rate": round((h1 - h0) / max(1, (h1 - h0) + (m1 - m0)), 4),
+                "misses_per_layer": round((m1 - m0) / n, 2),
+                "h2d_GB/s": round((b1 - b0) / el / 1e9, 2)})
+            del layer
     elif args.workload == "router":
         P, S, B = synth.router(args.seed)
         R = qmoe.QMatrix.from_numpy(P, S, B, E, H, 8, dev)

@@ -269,6 +269,60 @@ qmoe_status moe_decode_layers(const void *const *packed_layers, int32_t n_layers
                               size_t workspace_bytes, int32_t *status_dev, void *stream);
 
 /* ---------------------------------------------------------------------------
+ * Host-memory expert streaming through a per-layer LFU cache (TurboFieldfare
+ * article, "내부 구조" section: the CPU takes the router's top-8 ids, plans
+ * the misses against the layer's 16-slot LFU cache and fills the missed
+ * experts into device-visible memory before the routed experts run).
+ *
+ * Plan, per token (readings; the page names the policy only): the token's
+ * hits first -- the slot's use count grows by one and the slot is pinned for
+ * this token -- then its misses in id order: the lowest-index empty slot,
+ * else the unpinned slot with the smallest count (ties: lowest index); a
+ * loaded expert starts at count 1; an evicted expert's count is forgotten.
+ *
+ * qmoe_lfu_*: the plan alone, host memory only (no GPU needed).
+ *   qmoe_lfu_plan returns the number of misses (listed in order as
+ *   miss_expert[i] -> miss_slot[i]) and fills slot_of[j] for ids[j]; -1 if
+ *   k > nslots, k > 16 or the ids repeat (the state is then unchanged).
+ *
+ * qmoe_cache_create: `host` holds the layer's routed experts (gate, up, down
+ * stacked over num_experts) in PINNED HOST memory; `slots` the same three
+ * stacks over nslots = slots->num_experts in device memory, plus the resident
+ * shared expert (device).  The cache starts empty.  Allocates its own small
+ * pinned and device buffers and an event; qmoe_cache_destroy frees them.
+ *
+ * moe_cache_layer: one decode token through the layer:
+ *   router (resident, device) -> the host reads the top_k ids (this call
+ *   SYNCHRONISES `stream` once; every other entry point never does) -> plan
+ *   -> each missed expert's nine arrays host -> device on `copy_stream`
+ *   (NULL: `stream`) -> the routed experts wait for the copies -> y =
+ *   shared(x) + sum_j weights[j] * expert_{idx[j]}(x) from the slots (as
+ *   moe_expert_qmlp; same zero-filled workspace).  idx_out / weights_out
+ *   (device, optional) receive the router's choice.  Returns
+ *   QMOE_ERR_DEVICE_STATUS if the router produced an id outside [0, E).
+ * qmoe_cache_stats: cumulative hits, misses, bytes copied; the expert held by
+ * each slot (-1: empty).
+ * ------------------------------------------------------------------------- */
+typedef struct qmoe_lfu qmoe_lfu;
+typedef struct qmoe_expert_cache qmoe_expert_cache;
+
+qmoe_status qmoe_lfu_create(int32_t nslots, qmoe_lfu **out);
+void qmoe_lfu_destroy(qmoe_lfu *h);
+int32_t qmoe_lfu_plan(qmoe_lfu *h, const int32_t *ids, int32_t k, int32_t *slot_of,
+                      int32_t *miss_expert, int32_t *miss_slot);
+qmoe_status qmoe_lfu_slots(const qmoe_lfu *h, int32_t *expert, int64_t *count);
+
+qmoe_status qmoe_cache_create(const qmoe_moe_layer *host, const qmoe_moe_layer *slots,
+                              qmoe_expert_cache **out);
+void qmoe_cache_destroy(qmoe_expert_cache *c);
+qmoe_status moe_cache_layer(qmoe_expert_cache *c, const qmoe_qmatrix *router, const uint16_t *x,
+                            int32_t top_k, uint16_t *y, int32_t *idx_out, float *weights_out,
+                            void *workspace, size_t workspace_bytes, int32_t *status_dev,
+                            void *stream, void *copy_stream);
+qmoe_status qmoe_cache_stats(const qmoe_expert_cache *c, int64_t *hits, int64_t *misses,
+                             int64_t *bytes_copied, int32_t *slot_expert);
+
+/* ---------------------------------------------------------------------------
  * Prefill grouping ("내부 구조" section: a chunk's tokens are gathered per
  * expert so one fetched expert serves many rows).
  *   counts[e]  = number of (token, slot) pairs with idx == e

@@ -71,6 +71,14 @@ def lib():
             "qmoe_status_string": [ctypes.c_int],
             "qmoe_set_dependent_launch": [i32],
             "qmoe_version": [],
+            "qmoe_lfu_create": [i32, p],
+            "qmoe_lfu_destroy": [p],
+            "qmoe_lfu_plan": [p, p, i32, p, p, p],
+            "qmoe_lfu_slots": [p, p, p],
+            "qmoe_cache_create": [p, p, p],
+            "qmoe_cache_destroy": [p],
+            "moe_cache_layer": [p, p, p, i32, p, p, p, p, sz, p, p, p],
+            "qmoe_cache_stats": [p, p, p, p, p],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -83,6 +91,9 @@ def lib():
         L.qmoe_status_string.restype = ctypes.c_char_p
         L.qmoe_version.restype = i32
         L.qmoe_set_dependent_launch.restype = i32
+        L.qmoe_lfu_destroy.restype = None
+        L.qmoe_cache_destroy.restype = None
+        L.qmoe_lfu_plan.restype = i32
         _lib = L
     return _lib
 
@@ -206,6 +217,107 @@ class MoELayer:
             router = QMatrix.from_numpy(*m["router"], E, H, 8, device)
         return cls(q["gate"], q["up"], q["down"], q["sh_gate"], q["sh_up"], q["sh_down"], E, H,
                    I, router)
+
+
+# ------------------------------------------------------- expert streaming --
+class LfuPlan:
+    """The library's per-layer LFU expert-cache plan alone (host memory only,
+    no GPU): step(ids) -> (slot_of [k], [(expert, slot), ...] misses)."""
+
+    def __init__(self, nslots=16):
+        h = ctypes.c_void_p()
+        _check(lib().qmoe_lfu_create(nslots, ctypes.byref(h)), "qmoe_lfu_create")
+        self.h, self.nslots = h, nslots
+
+    def step(self, ids):
+        ids = np.ascontiguousarray(ids, np.int32)
+        k = ids.size
+        slot_of = np.empty(max(k, 1), np.int32)
+        me = np.empty(max(k, 1), np.int32)
+        ms = np.empty(max(k, 1), np.int32)
+        v = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+        n = lib().qmoe_lfu_plan(self.h, v(ids), k, v(slot_of), v(me), v(ms))
+        if n < 0:
+            raise ValueError("k > nslots, k > 16 or repeated ids")
+        return slot_of[:k], list(zip(me[:n].tolist(), ms[:n].tolist()))
+
+    def slots(self):
+        e = np.empty(self.nslots, np.int32)
+        c = np.empty(self.nslots, np.int64)
+        _check(lib().qmoe_lfu_slots(self.h, e.ctypes.data_as(ctypes.c_void_p),
+                                    c.ctypes.data_as(ctypes.c_void_p)), "qmoe_lfu_slots")
+        return e, c
+
+    def __del__(self):
+        if getattr(self, "h", None) and _lib is not None:
+            _lib.qmoe_lfu_destroy(self.h)
+            self.h = None
+
+
+class ExpertCacheLayer:
+    """One MoE layer whose routed experts live in pinned host memory and are
+    streamed into `nslots` device slots through the library's LFU plan; the
+    router and the shared expert stay on the device."""
+
+    def __init__(self, m, E, H, I, nslots=16, device="cuda"):
+        self.E, self.H, self.I, self.nslots = E, H, I, nslots
+        pin = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a).view(dt).copy()).pin_memory()
+        self.host = {}
+        for name in ("gate", "up", "down"):
+            P, S, B = m[name]
+            self.host[name] = (pin(P, np.int32), pin(S, np.float16), pin(B, np.float16))
+        dims = {"gate": (I, H), "up": (I, H), "down": (H, I)}
+        hq = {n: CQMatrix(t[0].data_ptr(), t[1].data_ptr(), t[2].data_ptr(), dims[n][0],
+                          dims[n][1], 4, 64) for n, t in self.host.items()}
+        dev_layer = MoELayer.from_numpy(m, E, H, I, device)   # router + shared expert on device
+        self.router = dev_layer.router
+        self.shared = {n: dev_layer.mats[n] for n in ("sh_gate", "sh_up", "sh_down")}
+        self.slot = {}
+        for n, (rows, cols) in dims.items():
+            self.slot[n] = QMatrix(
+                torch.zeros(nslots * rows * cols // 8, dtype=torch.int32, device=device),
+                torch.zeros(nslots * rows * (cols // 64), dtype=torch.float16, device=device),
+                torch.zeros(nslots * rows * (cols // 64), dtype=torch.float16, device=device),
+                rows, cols, 4, nslots)
+        sh = self.shared
+        self.c_host = CMoeLayer(hq["gate"], hq["up"], hq["down"], sh["sh_gate"].c, sh["sh_up"].c,
+                                sh["sh_down"].c, E, H, I)
+        self.slot_layer = MoELayer(self.slot["gate"], self.slot["up"], self.slot["down"],
+                                   sh["sh_gate"], sh["sh_up"], sh["sh_down"], nslots, H, I)
+        h = ctypes.c_void_p()
+        _check(lib().qmoe_cache_create(ctypes.byref(self.c_host), ctypes.byref(self.slot_layer.c),
+                                       ctypes.byref(h)), "qmoe_cache_create")
+        self.h = h
+        self.workspace = {}
+        self.copy_stream = torch.cuda.Stream(device=device)
+
+    def forward(self, x, top_k=8, y=None, idx=None, weights=None, status=None):
+        """One decode token x [H] float16 through the layer; returns y [H]."""
+        x = _need(x, torch.float16, "x").reshape(-1)
+        if y is None:
+            y = torch.empty(self.H, dtype=torch.float16, device=x.device)
+        ws = self.workspace.get(top_k)
+        if ws is None:
+            ws = self.workspace[top_k] = expert_workspace(self.slot_layer, top_k, x.device)
+        _check(lib().moe_cache_layer(self.h, ctypes.byref(self.router.c), _ptr(x), top_k, _ptr(y),
+                                     _ptr(idx), _ptr(weights), _ptr(ws), ws.numel(), _ptr(status),
+                                     _stream(), ctypes.c_void_p(self.copy_stream.cuda_stream)),
+               "moe_cache_layer")
+        return y
+
+    def stats(self):
+        """(hits, misses, bytes copied, expert held by each slot)."""
+        hits, misses, nbytes = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+        slots = np.empty(self.nslots, np.int32)
+        _check(lib().qmoe_cache_stats(self.h, ctypes.byref(hits), ctypes.byref(misses),
+                                      ctypes.byref(nbytes),
+                                      slots.ctypes.data_as(ctypes.c_void_p)), "qmoe_cache_stats")
+        return hits.value, misses.value, nbytes.value, slots
+
+    def __del__(self):
+        if getattr(self, "h", None) and _lib is not None:
+            _lib.qmoe_cache_destroy(self.h)
+            self.h = None
 
 
 # ------------------------------------------------------------- operations --

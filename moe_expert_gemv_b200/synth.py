@@ -94,6 +94,18 @@ def activations(seed, rows, cols, layer=0):
     return to_f16_bits(rng(seed, layer, _TAGS["x"]).standard_normal((rows, cols)))
 
 
+def correlated_tokens(seed, T, cols, rho, layer=0):
+    """fp16 bits [T][cols]: x_0 ~ N(0,1), x_t = rho x_{t-1} + sqrt(1 - rho^2) n_t
+    (each row stays N(0,1)); rho near 1 gives consecutive tokens similar
+    routing, rho = 0 independent tokens."""
+    g = rng(seed, layer, 17)
+    x = np.empty((T, cols))
+    x[0] = g.standard_normal(cols)
+    for t in range(1, T):
+        x[t] = rho * x[t - 1] + np.sqrt(1.0 - rho * rho) * g.standard_normal(cols)
+    return to_f16_bits(x)
+
+
 def dense(seed, N, K, bits=4, layer=0):
     """One dense affine-quantized matrix with the dense-GEMV value ranges."""
     return qmatrix(rng(seed, layer, _TAGS["dense"]), N, K, bits)
