@@ -10,7 +10,8 @@
 // On B200 the whole model fits HBM, so this path exists for models that do
 // not: the routed experts of a layer live in pinned host memory, the cache is
 // `nslots` device slots laid out as a stacked expert array, and a miss is one
-// host-to-device copy per array of the expert on a copy stream.  Host code
+// host-to-device copy per array of the expert, spread over four copy
+// streams (bounded parallel copies).  Host code
 // only (no kernels): the router and the experts run the library's kernels.
 //
 // Plan (host, per token and layer): hits first -- the slot's count grows by
@@ -30,6 +31,7 @@ namespace {
 
 constexpr int kMaxSlots = 256;
 constexpr int kMaxTopK = 16;
+constexpr int kCopyStreams = 4;   // misses copied in parallel (bounded, as the pages' reads)
 
 struct Lfu {
     int nslots;
@@ -158,7 +160,8 @@ struct qmoe_expert_cache {
     int32_t *idx_dev;       // device [kMaxTopK]
     float *wt_dev;          // device [kMaxTopK]
     int32_t *slot_dev;      // device [kMaxTopK]
-    cudaEvent_t copied;
+    cudaStream_t copy[kCopyStreams];   // the cache's own copy streams
+    cudaEvent_t copied[kCopyStreams];
     int64_t hits, misses, bytes;
 };
 
@@ -228,8 +231,11 @@ qmoe_status qmoe_cache_create(const qmoe_moe_layer *host, const qmoe_moe_layer *
         e = cudaMalloc(&c->wt_dev, kMaxTopK * sizeof(float));
     if (e == cudaSuccess)
         e = cudaMalloc(&c->slot_dev, kMaxTopK * sizeof(int32_t));
-    if (e == cudaSuccess)
-        e = cudaEventCreateWithFlags(&c->copied, cudaEventDisableTiming);
+    for (int i = 0; i < kCopyStreams && e == cudaSuccess; ++i) {
+        e = cudaStreamCreateWithFlags(&c->copy[i], cudaStreamNonBlocking);
+        if (e == cudaSuccess)
+            e = cudaEventCreateWithFlags(&c->copied[i], cudaEventDisableTiming);
+    }
     if (e != cudaSuccess) {
         qmoe_cache_destroy(c);
         return QMOE_ERR_CUDA;
@@ -252,8 +258,12 @@ void qmoe_cache_destroy(qmoe_expert_cache *c)
         cudaFree(c->wt_dev);
     if (c->slot_dev)
         cudaFree(c->slot_dev);
-    if (c->copied)
-        cudaEventDestroy(c->copied);
+    for (int i = 0; i < kCopyStreams; ++i) {
+        if (c->copied[i])
+            cudaEventDestroy(c->copied[i]);
+        if (c->copy[i])
+            cudaStreamDestroy(c->copy[i]);
+    }
     free(c);
 }
 
@@ -268,7 +278,15 @@ qmoe_status moe_cache_layer(qmoe_expert_cache *c, const qmoe_qmatrix *router, co
         router->rows != c->host.num_experts)
         return QMOE_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaStream_t cs = copy_stream ? static_cast<cudaStream_t>(copy_stream) : st;
+    // copy streams: the caller's (if any) first, then the cache's own
+    cudaStream_t cs[kCopyStreams];
+    cudaEvent_t ev[kCopyStreams];
+    for (int i = 0; i < kCopyStreams; ++i) {
+        cs[i] = c->copy[i];
+        ev[i] = c->copied[i];
+    }
+    if (copy_stream)
+        cs[0] = static_cast<cudaStream_t>(copy_stream);
     // 1. router on resident weights
     qmoe_status s = moe_router_topk(router, x, 1, top_k, c->idx_dev, c->wt_dev, nullptr,
                                     status_dev, stream);
@@ -290,13 +308,25 @@ qmoe_status moe_cache_layer(qmoe_expert_cache *c, const qmoe_qmatrix *router, co
     const int nm = lfu_plan(&c->plan.c, ids, top_k, c->slot_host, miss_e, miss_s);
     if (nm < 0)
         return QMOE_ERR_INVALID_ARG;
-    // 4. the missed experts' arrays, host -> device, one copy each
+    // 4. the missed experts' arrays, host -> device, one copy each; expert m
+    //    on copy stream m % kCopyStreams.  A slot must not be overwritten
+    //    while an earlier token's experts read it: the synchronisation above
+    //    already ordered everything enqueued on `stream` before this point,
+    //    and the copy streams also wait on an event of `stream`.
+    const int nstreams = nm < kCopyStreams ? nm : kCopyStreams;
+    if (nstreams > 0) {
+        if (cudaEventRecord(ev[0], st) != cudaSuccess)
+            return QMOE_ERR_CUDA;
+        for (int i = 0; i < nstreams; ++i)
+            if (cudaStreamWaitEvent(cs[i], ev[0], 0) != cudaSuccess)
+                return QMOE_ERR_CUDA;
+    }
     for (int m = 0; m < nm; ++m) {
         ArrayPart parts[9];
         const int np = expert_parts(c->host, c->slots, miss_e[m], miss_s[m], parts);
         for (int i = 0; i < np; ++i) {
             if (cudaMemcpyAsync(parts[i].dst, parts[i].src, parts[i].bytes,
-                                cudaMemcpyHostToDevice, cs) != cudaSuccess)
+                                cudaMemcpyHostToDevice, cs[m % kCopyStreams]) != cudaSuccess)
                 return QMOE_ERR_CUDA;
             c->bytes += (int64_t)parts[i].bytes;
         }
@@ -304,9 +334,10 @@ qmoe_status moe_cache_layer(qmoe_expert_cache *c, const qmoe_qmatrix *router, co
     c->hits += top_k - nm;
     c->misses += nm;
     // 5. the routed experts wait for the copies; the slot ids follow the plan
-    if (cs != st && (cudaEventRecord(c->copied, cs) != cudaSuccess ||
-                     cudaStreamWaitEvent(st, c->copied, 0) != cudaSuccess))
-        return QMOE_ERR_CUDA;
+    for (int i = 0; i < nstreams; ++i)
+        if (cudaEventRecord(ev[i], cs[i]) != cudaSuccess ||
+            cudaStreamWaitEvent(st, ev[i], 0) != cudaSuccess)
+            return QMOE_ERR_CUDA;
     if (cudaMemcpyAsync(c->slot_dev, c->slot_host, top_k * sizeof(int32_t),
                         cudaMemcpyHostToDevice, st) != cudaSuccess)
         return QMOE_ERR_CUDA;
