@@ -38,3 +38,14 @@ def f16_values(bits):
 def to_dev_f16(bits, device="cuda"):
     import torch
     return torch.from_numpy(np.ascontiguousarray(bits, dtype=np.uint16).view(np.float16).copy()).to(device)
+
+
+def assert_close_rows(y, ref, tol=REL_TOL, what=""):
+    """assert_close over the whole output and over each row (batch element,
+    token) on its own scale."""
+    y = np.atleast_2d(np.asarray(y))
+    ref = np.atleast_2d(np.asarray(ref))
+    assert_close(y, ref, tol, what)
+    for i in range(y.shape[0]):
+        assert_close(y[i], ref[i], tol, "%s, row %d" % (what, i))
+

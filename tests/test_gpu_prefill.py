@@ -53,6 +53,8 @@ def test_small_chunks_full_compare(cuda_dev, E, H, I, T, k):
     assert flags == 0
     y64, _ = oracle.Layer(m, E, H, I).moe(x16, idx, wt.astype(np.float64))
     assert_close(y.view(np.float16), y64, what="prefill %s" % ((E, H, I, T, k),))
+    for t in range(T):   # each token on its own scale
+        assert_close(y.view(np.float16)[t], y64[t], what="prefill %s token %d" % ((E, H, I, T, k), t))
 
 
 @pytest.fixture(scope="module")
