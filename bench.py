@@ -433,7 +433,7 @@ def main_other(args):
                 P, S, B = synth.dense(c, N, K)
                 Ws.append(qmoe.QMatrix.from_numpy(P, S, B, N, K, 4, dev))
             nbytes = N * K // 2 + 2 * N * (K // 64) * 2
-            for Bt in (1, 4, 8):
+            for Bt in (1, 4, 8, 16, 32):
                 x = torch.from_numpy(synth.activations(Bt, Bt, K).view(np.float16).copy()).to(dev)
                 y = torch.empty(Bt, N, dtype=torch.float16, device=dev)
 
@@ -453,7 +453,7 @@ def main_other(args):
                                        "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
                                        "rotated_copies": copies})
     elif args.workload == "qgemv_fmt":
-        # bf16-scale formats with the block-32 rotation of x, config-1 shapes
+        # bf16-scale formats with the block-32 rotation of x, the K=4096 dense shapes
         for fmt, name in ((qmoe.FMT_ZP4_BF16, "zp4_bf16"), (qmoe.FMT_SYM8_BF16, "sym8_bf16")):
             bits = 4 if fmt == qmoe.FMT_ZP4_BF16 else 8
             for N in (14336, 4096):
@@ -464,7 +464,7 @@ def main_other(args):
                 for c in range(copies):
                     P, prm, sg = synth.qmatrix_fmt(synth.rng(c, N, fmt), N, K, fmt)
                     Ws.append(qmoe.QMatrixFmt.from_numpy(P, prm, sg, N, K, fmt, device=dev))
-                for Bt in (1, 8):
+                for Bt in (1, 8, 32):
                     x = torch.from_numpy(synth.activations(Bt, Bt, K).view(np.float16).copy()).to(dev)
                     y = torch.empty(Bt, N, dtype=torch.float16, device=dev)
 
@@ -486,7 +486,7 @@ def main_other(args):
                                            "rotated_copies": copies})
                 del Ws
     elif args.workload == "expert_cache":
-        # one config-3 layer with its routed experts in pinned host memory and
+        # one 128-expert H=2816 layer with its routed experts in pinned host memory and
         # 16 device slots; decode tokens whose routing locality is set by rho
         m = synth.moe_layer(args.seed, 0)
         for rho in (0.0, 0.9, 0.99):

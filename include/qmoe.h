@@ -108,7 +108,11 @@ typedef struct qmoe_moe_layer {
  * "기술 맥락" section, format of the "성능과 제약" section).
  *   y[b][n] = sum_k w[n][k] * x[b][k]     fp32 accumulate, fp16 output
  *   W: bits 4 or 8; x: fp16 [batch][W->cols]; y: fp16 [batch][W->rows].
- * Errors: INVALID_ARG (NULL, batch outside 1..8, shape), ALIGNMENT,
+ * batch 1..32: up to 8 rows of x per kernel launch (tensor-core N = 8); a
+ * larger batch (e.g. the 16-32 draft tokens a speculative-decoding step
+ * verifies) runs one launch per 8 rows, the later ones reading a matrix
+ * that fits L2 from L2.
+ * Errors: INVALID_ARG (NULL, batch outside 1..32, shape), ALIGNMENT,
  * UNSUPPORTED (group != 64, cols % 64, rows % 8), CUDA.
  * ------------------------------------------------------------------------- */
 qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch,
@@ -131,8 +135,9 @@ qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch
  *           of rht_signs[i / 32] is set.  x must then be 16-byte aligned; the
  *           rotation runs in fp32 inside the kernel and R x enters the product
  *           as an fp16 (hi, lo) pair (about 22 significant bits).
- * batch 1..8; cols a multiple of 64, rows of 8; y fp16 [batch][rows].
- * Errors as qgemv_affine (INVALID_ARG also for an unknown format).
+ * batch 1..32 (as qgemv_affine); cols a multiple of 64, rows of 8;
+ * y fp16 [batch][rows].  Errors as qgemv_affine (INVALID_ARG also for an
+ * unknown format).
  * ------------------------------------------------------------------------- */
 #define QMOE_FMT_ZP4_BF16 1
 #define QMOE_FMT_SYM8_BF16 2

@@ -173,7 +173,7 @@ qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch
 {
     if (!W || !x || !y)
         return QMOE_ERR_INVALID_ARG;
-    if (batch < 1 || batch > 8)
+    if (batch < 1 || batch > kMaxQgemvBatch)
         return QMOE_ERR_INVALID_ARG;
     qmoe_status s = check_qmatrix(W, W->rows, W->cols, 0);
     if (s != QMOE_OK)
@@ -197,7 +197,7 @@ qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch
     a.B = batch;
     a.y = reinterpret_cast<__half *>(y);
     a.status = status_dev ? status_dev : d->status;
-    return cuda_status(launch_qgemv(a, launch_cfg(d, stream)));
+    return cuda_status(launch_qgemv_batched(a, launch_cfg(d, stream)));
 }
 
 qmoe_status qgemv_fmt(const qmoe_qmatrix_fmt *W, const uint16_t *x, int32_t batch, uint16_t *y,
@@ -205,7 +205,7 @@ qmoe_status qgemv_fmt(const qmoe_qmatrix_fmt *W, const uint16_t *x, int32_t batc
 {
     if (!W || !W->packed || !W->params || !x || !y)
         return QMOE_ERR_INVALID_ARG;
-    if (batch < 1 || batch > 8 || W->rows <= 0 || W->cols <= 0)
+    if (batch < 1 || batch > kMaxQgemvBatch || W->rows <= 0 || W->cols <= 0)
         return QMOE_ERR_INVALID_ARG;
     if (W->format != QMOE_FMT_ZP4_BF16 && W->format != QMOE_FMT_SYM8_BF16)
         return QMOE_ERR_INVALID_ARG;
@@ -235,7 +235,7 @@ qmoe_status qgemv_fmt(const qmoe_qmatrix_fmt *W, const uint16_t *x, int32_t batc
     a.B = batch;
     a.y = reinterpret_cast<__half *>(y);
     a.status = status_dev ? status_dev : d->status;
-    return cuda_status(launch_qgemv(a, launch_cfg(d, stream)));
+    return cuda_status(launch_qgemv_batched(a, launch_cfg(d, stream)));
 }
 
 qmoe_status moe_router_topk(const qmoe_qmatrix *router, const uint16_t *x, int32_t tokens,

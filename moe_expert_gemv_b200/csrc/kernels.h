@@ -37,6 +37,10 @@ struct QgemvArgs {
     int32_t *status;
 };
 cudaError_t launch_qgemv(const QgemvArgs &a, const LaunchCfg &c);
+// batch up to kMaxQgemvBatch: one launch per slice of 8 rows of x / y (the
+// slices after the first read a matrix that fits L2 from L2)
+constexpr int kMaxQgemvBatch = 32;
+cudaError_t launch_qgemv_batched(const QgemvArgs &a, const LaunchCfg &c);
 
 // Tensor map over the 4/8-bit codes of a row-major [rows][Kw words] matrix
 // (Kw % 32 == 0) as a 3-D tensor [Kw/32 chunks][rows][32 words]: one copy

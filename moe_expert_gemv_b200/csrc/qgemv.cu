@@ -439,4 +439,18 @@ cudaError_t launch_qgemv(const QgemvArgs &a, const LaunchCfg &c)
     return swz ? launch_qgemv_fmt<true>(a, c, m) : launch_qgemv_fmt<false>(a, c, m);
 }
 
+cudaError_t launch_qgemv_batched(const QgemvArgs &a, const LaunchCfg &c)
+{
+    for (int b0 = 0; b0 < a.B; b0 += 8) {
+        QgemvArgs s = a;
+        s.x = a.x + (size_t)b0 * a.K;
+        s.y = a.y + (size_t)b0 * a.N;
+        s.B = a.B - b0 < 8 ? a.B - b0 : 8;
+        const cudaError_t e = launch_qgemv(s, c);
+        if (e != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
+}
+
 }  // namespace qmoe

@@ -322,7 +322,7 @@ class ExpertCacheLayer:
 
 # ------------------------------------------------------------- operations --
 def qgemv_affine(W, x, y=None, status=None):
-    """y[b] = W x[b] for x [B][K] float16 (B <= 8).  Returns y [B][N] float16."""
+    """y[b] = W x[b] for x [B][K] float16 (B <= 32).  Returns y [B][N] float16."""
     x = _need(x, torch.float16, "x")
     x2 = x.reshape(-1, W.cols)
     if y is None:
@@ -335,7 +335,7 @@ def qgemv_affine(W, x, y=None, status=None):
 
 def qgemv_fmt(W, x, y=None, status=None):
     """y[b] = W (R x[b]) (R the rotation when W has signs) for x [B][K]
-    float16 (B <= 8), W a QMatrixFmt.  Returns y [B][N] float16."""
+    float16 (B <= 32), W a QMatrixFmt.  Returns y [B][N] float16."""
     x = _need(x, torch.float16, "x")
     x2 = x.reshape(-1, W.cols)
     if y is None:

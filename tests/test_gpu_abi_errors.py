@@ -33,7 +33,7 @@ def test_qgemv_argument_errors(cuda_dev):
     assert call_qgemv(good, x.data_ptr(), 1, y.data_ptr()) == 0
     assert call_qgemv(good, None, 1, y.data_ptr()) == INVALID
     assert call_qgemv(good, x.data_ptr(), 0, y.data_ptr()) == INVALID
-    assert call_qgemv(good, x.data_ptr(), 9, y.data_ptr()) == INVALID
+    assert call_qgemv(good, x.data_ptr(), 33, y.data_ptr()) == INVALID
     assert call_qgemv(good, x.data_ptr() + 1, 1, y.data_ptr()) == ALIGN
     bad, k2 = mat(64, 256, off=4)
     assert call_qgemv(bad, x.data_ptr(), 1, y.data_ptr()) == ALIGN

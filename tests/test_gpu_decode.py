@@ -53,7 +53,7 @@ def test_small_stacks(cuda_dev, E, H, I, k, n):
     check_layers(ms, E, H, I, k, x16, y, idx, wt, lg)
 
 
-def test_config3_three_layers_and_repeat(cuda_dev):
+def test_moe_e128_three_layers_and_repeat(cuda_dev):
     E, H, I, k = synth.MOE_E, synth.MOE_H, synth.MOE_I, synth.MOE_TOPK
     ms, stack = make_stack(3, 3, E, H, I, k)
     x16 = np.concatenate([synth.activations(3, 1, H, layer=l) for l in range(3)])
@@ -84,7 +84,7 @@ def test_matches_unfused_path(cuda_dev):
 
 
 @pytest.mark.slow
-def test_config3_thirty_layers_sampled(cuda_dev):
+def test_moe_e128_thirty_layers_sampled(cuda_dev):
     """The full decode step: 30 layers, 12.96 GB of weights; every layer's
     routing is checked, outputs of a sample of layers against the oracle."""
     E, H, I, k, n = synth.MOE_E, synth.MOE_H, synth.MOE_I, synth.MOE_TOPK, synth.MOE_LAYERS

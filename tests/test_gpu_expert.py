@@ -26,7 +26,7 @@ def gpu_layer(G, x16, idx, wt, ws=None):
     return y
 
 
-def test_config3_layer_oracle_routing(cuda_dev, layer_full):
+def test_moe_layer_e128_oracle_routing(cuda_dev, layer_full):
     """Full-size layer; routing from the oracle's router (fp64), weights passed
     to both sides as the same fp32 values."""
     m, G, L = layer_full
@@ -36,10 +36,10 @@ def test_config3_layer_oracle_routing(cuda_dev, layer_full):
     y = gpu_layer(G, x16, idx[0], wt32[0])
     assert qmoe.qmoe_check_status() == 0
     y64, _ = L.moe(x16, idx, wt32.astype(np.float64))
-    assert_close(f16_bits(y).view(np.float16), y64[0], what="config 3 layer")
+    assert_close(f16_bits(y).view(np.float16), y64[0], what="E128 H2816 I704 layer")
 
 
-def test_config3_router_then_experts(cuda_dev, layer_full):
+def test_moe_layer_e128_router_then_experts(cuda_dev, layer_full):
     """The device path end to end: GPU router ids feed the GPU experts."""
     m, G, L = layer_full
     for seed in range(3):

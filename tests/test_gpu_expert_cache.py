@@ -51,7 +51,7 @@ def test_small_layer_token_stream(cuda_dev, rho):
 
 
 @pytest.mark.slow
-def test_config3_layer_token_stream(cuda_dev):
+def test_moe_e128_layer_token_stream(cuda_dev):
     E, H, I, k = synth.MOE_E, synth.MOE_H, synth.MOE_I, synth.MOE_TOPK
     m = synth.moe_layer(22, 0)
     x16 = synth.correlated_tokens(22, 10, H, 0.9)

@@ -58,7 +58,7 @@ def test_small_chunks_full_compare(cuda_dev, E, H, I, T, k):
 
 
 @pytest.fixture(scope="module")
-def config4():
+def chunk128():
     E, H, I = synth.MOE_E, synth.MOE_H, synth.MOE_I
     m = synth.moe_layer(4, 0)
     G = qmoe.MoELayer.from_numpy(m, E, H, I)
@@ -68,22 +68,22 @@ def config4():
 
 
 @pytest.mark.slow
-def test_config4_chunk_sampled_tokens(cuda_dev, config4):
+def test_chunk128_chunk_sampled_tokens(cuda_dev, chunk128):
     """The 128-token chunk with Zipf(1.1) routing; every output of a sample of
     32 tokens (spread over the chunk) against the oracle."""
-    m, G, idx, wt, x16 = config4
+    m, G, idx, wt, x16 = chunk128
     E, H, I = synth.MOE_E, synth.MOE_H, synth.MOE_I
     y, flags = run_prefill(G, x16, idx, wt)
     assert flags == 0
     rows = np.unique(np.concatenate([np.arange(0, 128, 5), [127]]))[:32]
     y64, _ = oracle.Layer(m, E, H, I).moe(x16[rows], idx[rows], wt[rows].astype(np.float64))
-    assert_close(y.view(np.float16)[rows], y64, what="config 4 sampled tokens")
+    assert_close(y.view(np.float16)[rows], y64, what="128-token chunk sampled tokens")
 
 
-def test_config4_rows_equal_decode_layer(cuda_dev, config4):
+def test_chunk128_rows_equal_decode_layer(cuda_dev, chunk128):
     """Row t of the chunk = the decode layer on token t with the same routing
     (two independent device paths)."""
-    m, G, idx, wt, x16 = config4
+    m, G, idx, wt, x16 = chunk128
     y, _ = run_prefill(G, x16, idx, wt)
     for t in (0, 63, 127):
         yd = qmoe.moe_expert_qmlp(G, dev(x16[t].view(np.float16), np.float16), dev(idx[t], np.int32),
@@ -110,8 +110,8 @@ def test_bad_expert_ids_flagged(cuda_dev):
     assert_close(y.view(np.float16), y64, what="bad ids dropped")
 
 
-def test_repeat_calls_bitwise_identical(cuda_dev, config4):
-    m, G, idx, wt, x16 = config4
+def test_repeat_calls_bitwise_identical(cuda_dev, chunk128):
+    m, G, idx, wt, x16 = chunk128
     a, _ = run_prefill(G, x16, idx, wt)
     b, _ = run_prefill(G, x16, idx, wt)
     assert np.array_equal(a, b)

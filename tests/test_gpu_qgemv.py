@@ -34,27 +34,27 @@ def test_pack_unpack_bit_exact(cuda_dev, bits):
         assert np.array_equal(un.cpu().numpy(), oracle.unpack(words, rows, cols, bits))
 
 
-def test_config0_single_qgemv(cuda_dev):
+def test_small_dense_single_qgemv(cuda_dev):
     """N=512, K=1024, batch 1 (the small dense case)."""
     N, K = 512, 1024
     P, S, B = synth.dense(0, N, K)
     x16 = synth.activations(0, 1, K)
     y = run_qgemv(P, S, B, N, K, 4, x16)
     y64, _ = oracle.qgemv(P, S, B, N, K, 4, x16)
-    assert_close(y.view(np.float16), y64, what="config 0")
+    assert_close(y.view(np.float16), y64, what="N=512 K=1024")
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("N", [14336, 4096])
 @pytest.mark.parametrize("Bt", [1, 4, 8])
-def test_config1_decode_sweep(cuda_dev, N, Bt):
+def test_k4096_decode_sweep(cuda_dev, N, Bt):
     """K=4096, N in {14336, 4096}, batch 1/4/8, full output against the oracle."""
     K = 4096
     P, S, B = synth.dense(1, N, K)
     x16 = synth.activations(1 + Bt, Bt, K)
     y = run_qgemv(P, S, B, N, K, 4, x16)
     y64, _ = oracle.qgemv(P, S, B, N, K, 4, x16)
-    assert_close_rows(y.view(np.float16), y64, what="config 1 N=%d B=%d" % (N, Bt))
+    assert_close_rows(y.view(np.float16), y64, what="K=4096 N=%d B=%d" % (N, Bt))
 
 
 @pytest.mark.parametrize("bits", [4, 8])
@@ -81,6 +81,19 @@ def test_tensor_copy_tiles_with_row_tail(cuda_dev, bits, N, K):
         y = run_qgemv(P, S, B, N, K, bits, x16)
         y64, _ = oracle.qgemv(P, S, B, N, K, bits, x16)
         assert_close(y.view(np.float16), y64, what="N=%d K=%d B=%d bits=%d" % (N, K, Bt, bits))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("N,K", [(512, 1024), (1000, 4096), (136, 192)])
+def test_small_m_batches(cuda_dev, bits, N, K):
+    """Batches of 9-32 rows (e.g. the draft tokens a speculative-decoding step
+    verifies), including ragged last slices of 8."""
+    P, S, B = synth.qmatrix(synth.rng(N, K, bits, 11), N, K, bits)
+    for Bt in (9, 16, 29, 32):
+        x16 = synth.activations(N + 3 * Bt, Bt, K)
+        y = run_qgemv(P, S, B, N, K, bits, x16)
+        y64, _ = oracle.qgemv(P, S, B, N, K, bits, x16)
+        assert_close_rows(y.view(np.float16), y64, what="N=%d K=%d B=%d bits=%d" % (N, K, Bt, bits))
 
 
 def test_zero_input_positive_zero(cuda_dev):

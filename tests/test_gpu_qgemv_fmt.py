@@ -33,9 +33,20 @@ def test_formats_against_oracle(cuda_dev, fmt, rotate, N, K):
                           what="fmt %d rot %d N=%d K=%d B=%d" % (fmt, rotate, N, K, Bt))
 
 
+@pytest.mark.parametrize("fmt", [qmoe.FMT_ZP4_BF16, qmoe.FMT_SYM8_BF16])
+def test_small_m_batches(cuda_dev, fmt):
+    N, K = 200, 1024
+    P, params, signs = synth.qmatrix_fmt(synth.rng(N, K, fmt, 12), N, K, fmt)
+    for Bt in (13, 32):
+        x16 = synth.activations(N + Bt + 5 * fmt, Bt, K)
+        y = run(P, params, signs, N, K, fmt, True, x16)
+        y64, _ = oracle.qgemv_fmt(P, params, N, K, fmt, x16, signs, True)
+        assert_close_rows(y.view(np.float16), y64, what="fmt %d B=%d" % (fmt, Bt))
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("fmt", [qmoe.FMT_ZP4_BF16, qmoe.FMT_SYM8_BF16])
-def test_config1_shape_sampled_rows(cuda_dev, fmt):
+def test_k4096_shapes_sampled_rows(cuda_dev, fmt):
     """N=14336, K=4096, batch 8 with the rotation: every output of 256
     sampled rows against the oracle (the oracle runs on those rows only)."""
     N, K, Bt = 14336, 4096, 8
@@ -45,7 +56,7 @@ def test_config1_shape_sampled_rows(cuda_dev, fmt):
     rows = np.random.default_rng(fmt).choice(N, 256, replace=False)
     rows.sort()
     y64, _ = oracle.qgemv_fmt(P[rows], params[rows], len(rows), K, fmt, x16, signs, True)
-    assert_close_rows(y[:, rows], y64, what="config-1 shape fmt %d" % fmt)
+    assert_close_rows(y[:, rows], y64, what="K=4096 shape fmt %d" % fmt)
 
 
 def test_zero_input_and_zero_codes(cuda_dev):

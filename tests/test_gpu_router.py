@@ -47,7 +47,7 @@ def check_against_oracle(P, S, B, E, K, bits, x16, k):
 
 
 @pytest.mark.parametrize("T", [1, 2, 4, 8, 16, 32, 64, 128])
-def test_config2_router(cuda_dev, T):
+def test_router_e128_k2816(cuda_dev, T):
     E, K = 128, 2816
     P, S, B = synth.router(2, E, K)
     x16 = synth.activations(20 + T, T, K)
