@@ -64,6 +64,8 @@ def parse():
                                            "expert_cache"],
                     default="moe_decode")
     ap.add_argument("--layers", type=int, default=LAYERS)
+    ap.add_argument("--qgemv-batch", default="1,4,8,16,32",
+                    help="batch sizes of the qgemv workload (comma-separated)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="time budget of the CPU-oracle baseline sample")
@@ -433,7 +435,7 @@ def main_other(args):
                 P, S, B = synth.dense(c, N, K)
                 Ws.append(qmoe.QMatrix.from_numpy(P, S, B, N, K, 4, dev))
             nbytes = N * K // 2 + 2 * N * (K // 64) * 2
-            for Bt in (1, 4, 8, 16, 32):
+            for Bt in [int(b) for b in args.qgemv_batch.split(",")]:
                 x = torch.from_numpy(synth.activations(Bt, Bt, K).view(np.float16).copy()).to(dev)
                 y = torch.empty(Bt, N, dtype=torch.float16, device=dev)
 

@@ -104,7 +104,7 @@ typedef struct qmoe_moe_layer {
 } qmoe_moe_layer;
 
 /* ---------------------------------------------------------------------------
- * Dense affine qGEMV, batch 1..8 (decode projection; quantized GEMV of the
+ * Dense affine qGEMV, batch 1..32 (decode projection; quantized GEMV of the
  * "기술 맥락" section, format of the "성능과 제약" section).
  *   y[b][n] = sum_k w[n][k] * x[b][k]     fp32 accumulate, fp16 output
  *   W: bits 4 or 8; x: fp16 [batch][W->cols]; y: fp16 [batch][W->rows].
@@ -113,10 +113,43 @@ typedef struct qmoe_moe_layer {
  * verifies) runs one launch per 8 rows, the later ones reading a matrix
  * that fits L2 from L2.
  * Errors: INVALID_ARG (NULL, batch outside 1..32, shape), ALIGNMENT,
- * UNSUPPORTED (group != 64, cols % 64, rows % 8), CUDA.
+ * UNSUPPORTED (group != 64, cols % 64, rows % 8, or x of up to 8 rows plus
+ * one 16-row tile over shared memory: e.g. 8-bit cols 8192 at batch 8;
+ * qgemv_affine_ws takes such rows from batch 9 on), CUDA.
  * ------------------------------------------------------------------------- */
 qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch,
                          uint16_t *y, int32_t *status_dev, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * The same product for batch 9..32 in ONE pass over the weights (the
+ * verification step of speculative decoding multiplies every projection by
+ * the 16-32 draft tokens at once; uzu page, discuss.pytorch.kr, section "uzu의
+ * 모델 변환과 Mirai 양자화 형식", lists speculative decoding among the runtime's
+ * features).  The K range is split into S slices whose x fits on chip; CTAs
+ * of different slices write fp32 partial tiles to `workspace` and the last
+ * one to finish a tile adds them in slice order (results do not depend on
+ * the order in which CTAs finish; they differ from qgemv_affine's only by
+ * fp32 rounding).
+ * qgemv_affine_workspace_bytes(rows, cols, bits, batch): bytes of workspace a
+ *   call of that shape needs; 0 when it needs none (batch <= 8, one slice,
+ *   or a shape the one-pass kernel does not take: then qgemv_affine_ws runs
+ *   qgemv_affine's path).  The one-pass kernel takes rows of whole 128-byte
+ *   code chunks (cols % 256 == 0 at 4 bits, % 128 at 8 bits), slices of a
+ *   multiple of 512 inputs, and scales / biases 16-byte aligned (otherwise
+ *   it runs qgemv_affine's path even where a workspace was asked for).
+ * workspace: device memory, 16-byte aligned, at least that many bytes,
+ *   zero-filled once before its first use.  Its first 64 KB hold per-tile
+ *   arrival counters that every call returns to zero, the rest fp32 partial
+ *   tiles, so one workspace serves calls of any shape in turn; it must not
+ *   be used by two calls that can run at the same time.  May be NULL when
+ *   the size is 0.
+ * Errors: as qgemv_affine; INVALID_ARG also for a missing or short workspace,
+ * ALIGNMENT for a workspace not 16-byte aligned.
+ * ------------------------------------------------------------------------- */
+size_t qgemv_affine_workspace_bytes(int32_t rows, int32_t cols, int32_t bits, int32_t batch);
+qmoe_status qgemv_affine_ws(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch, uint16_t *y,
+                            void *workspace, size_t workspace_bytes, int32_t *status_dev,
+                            void *stream);
 
 /* ---------------------------------------------------------------------------
  * Format variants of the dense qGEMV (uzu page, discuss.pytorch.kr, section

@@ -200,6 +200,52 @@ qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch
     return cuda_status(launch_qgemv_batched(a, launch_cfg(d, stream)));
 }
 
+size_t qgemv_affine_workspace_bytes(int32_t rows, int32_t cols, int32_t bits, int32_t batch)
+{
+    if (rows <= 0 || cols <= 0 || (bits != 4 && bits != 8) || batch < 1 || batch > kMaxQgemvBatch)
+        return 0;
+    return qgemm_small_workspace_bytes(rows, cols, bits, batch);
+}
+
+qmoe_status qgemv_affine_ws(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch, uint16_t *y,
+                            void *workspace, size_t workspace_bytes, int32_t *status_dev, void *stream)
+{
+    if (!W || !x || !y)
+        return QMOE_ERR_INVALID_ARG;
+    if (batch < 1 || batch > kMaxQgemvBatch)
+        return QMOE_ERR_INVALID_ARG;
+    qmoe_status s = check_qmatrix(W, W->rows, W->cols, 0);
+    if (s != QMOE_OK)
+        return s;
+    if (!aligned(x, 2) || !aligned(y, 2) || (status_dev && !aligned(status_dev, 4)) ||
+        (workspace && !aligned(workspace, 16)))
+        return QMOE_ERR_ALIGNMENT;
+    const size_t need = qgemm_small_workspace_bytes(W->rows, W->cols, W->bits, batch);
+    if (need > 0 && (!workspace || workspace_bytes < need))
+        return QMOE_ERR_INVALID_ARG;
+    DevState *d;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    QgemvArgs a;
+    a.packed = W->packed;
+    a.scales = reinterpret_cast<const __half *>(W->scales);
+    a.biases = reinterpret_cast<const __half *>(W->biases);
+    a.N = W->rows;
+    a.K = W->cols;
+    a.bits = W->bits;
+    a.params = nullptr;
+    a.signs = nullptr;
+    a.fmt = QG_AFFINE;
+    a.x = reinterpret_cast<const __half *>(x);
+    a.B = batch;
+    a.y = reinterpret_cast<__half *>(y);
+    a.status = status_dev ? status_dev : d->status;
+    if (batch <= 8)
+        return cuda_status(launch_qgemv(a, launch_cfg(d, stream)));
+    bool used = false;
+    return cuda_status(launch_qgemm_small(a, workspace, workspace_bytes, launch_cfg(d, stream), &used));
+}
+
 qmoe_status qgemv_fmt(const qmoe_qmatrix_fmt *W, const uint16_t *x, int32_t batch, uint16_t *y,
                       int32_t *status_dev, void *stream)
 {

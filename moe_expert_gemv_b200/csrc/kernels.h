@@ -41,14 +41,30 @@ cudaError_t launch_qgemv(const QgemvArgs &a, const LaunchCfg &c);
 // slices after the first read a matrix that fits L2 from L2)
 constexpr int kMaxQgemvBatch = 32;
 cudaError_t launch_qgemv_batched(const QgemvArgs &a, const LaunchCfg &c);
+// One pass over the weights for batch 9..32 (qgemm_small.cu): the workspace
+// (a 64 KB region of arrival counters, then fp32 partial tiles; zero-filled
+// before first use, reusable across shapes) a
+// call needs, 0 if the shape runs without one; the launch falls back to
+// launch_qgemv_batched where the shape or alignment rule it out.  *used_ws
+// reports whether the workspace was used.
+size_t qgemm_small_workspace_bytes(int N, int K, int bits, int B);
+cudaError_t launch_qgemm_small(const QgemvArgs &a, void *ws, size_t ws_bytes, const LaunchCfg &c,
+                               bool *used_ws);
 
 // Tensor map over the 4/8-bit codes of a row-major [rows][Kw words] matrix
 // (Kw % 32 == 0) as a 3-D tensor [Kw/32 chunks][rows][32 words]: one copy
-// brings `box_rows` whole rows, 128-byte swizzled (16-byte unit u of row r,
-// chunk c at byte c*box_rows*128 + r*128 + 16*(u ^ (r & 7)) of a 1024-byte
+// brings `box_chunks` 128-byte chunks (0: all, i.e. whole rows) of
+// `box_rows` rows, 128-byte swizzled (16-byte unit u of row r, chunk c of
+// the box at byte c*box_rows*128 + r*128 + 16*(u ^ (r & 7)) of a 1024-byte
 // aligned destination).  False when the driver entry point is unavailable
 // or refuses the shape.
-bool encode_codes_map(CUtensorMap *m, const uint32_t *packed, long rows, int Kw, int box_rows);
+bool encode_codes_map(CUtensorMap *m, const uint32_t *packed, long rows, int Kw, int box_rows,
+                      int box_chunks = 0);
+// 2-D map of a row-major 16-bit array [rows][cols] (no swizzle), boxes of
+// box_cols x box_rows; false if the address, the row stride or the box width
+// is not a multiple of 16 bytes.
+bool encode_u16_map_2d(CUtensorMap *m, const void *base, long rows, int cols, int box_cols,
+                       int box_rows);
 
 // ------------------------------------------------------------------ router --
 struct RouterArgs {

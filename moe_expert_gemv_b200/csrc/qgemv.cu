@@ -414,19 +414,39 @@ static EncodeTiledFn encode_tiled_fn()
     return fn;
 }
 
-bool encode_codes_map(CUtensorMap *m, const uint32_t *packed, long rows, int Kw, int box_rows)
+bool encode_codes_map(CUtensorMap *m, const uint32_t *packed, long rows, int Kw, int box_rows,
+                      int box_chunks)
 {
     EncodeTiledFn fn = encode_tiled_fn();
-    if (!fn || Kw % 32 != 0 || Kw / 32 > 256 || box_rows < 1 || box_rows > 256)
+    if (box_chunks <= 0)
+        box_chunks = Kw / 32;
+    if (!fn || Kw % 32 != 0 || box_chunks > 256 || box_chunks > Kw / 32 || box_rows < 1 ||
+        box_rows > 256)
         return false;
     const cuuint64_t dims[3] = {32, (cuuint64_t)rows, (cuuint64_t)(Kw / 32)};
     const cuuint64_t strides[2] = {(cuuint64_t)Kw * 4, 128};
-    const cuuint32_t box[3] = {32, (cuuint32_t)box_rows, (cuuint32_t)(Kw / 32)};
+    const cuuint32_t box[3] = {32, (cuuint32_t)box_rows, (cuuint32_t)box_chunks};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t *>(packed), dims, strides,
               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
+}
+
+bool encode_u16_map_2d(CUtensorMap *m, const void *base, long rows, int cols, int box_cols,
+                       int box_rows)
+{
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn || (reinterpret_cast<uintptr_t>(base) & 15u) || (cols * 2) % 16 || (box_cols * 2) % 16 ||
+        box_cols < 1 || box_cols > 256 || box_cols > cols || box_rows < 1 || box_rows > 256)
+        return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 cudaError_t launch_qgemv(const QgemvArgs &a, const LaunchCfg &c)

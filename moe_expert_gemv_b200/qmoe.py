@@ -52,6 +52,8 @@ def lib():
         p, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
         sig = {
             "qgemv_affine": [p, p, i32, p, p, p],
+            "qgemv_affine_workspace_bytes": [i32, i32, i32, i32],
+            "qgemv_affine_ws": [p, p, i32, p, p, sz, p, p],
             "qgemv_fmt": [p, p, i32, p, p, p],
             "moe_router_topk": [p, p, i32, i32, p, p, p, p, p],
             "moe_expert_workspace_bytes": [p, i32],
@@ -85,6 +87,7 @@ def lib():
             fn.argtypes = args
             fn.restype = ctypes.c_int
         L.moe_expert_workspace_bytes.restype = sz
+        L.qgemv_affine_workspace_bytes.restype = sz
         L.moe_prefill_workspace_bytes.restype = sz
         L.moe_decode_workspace_bytes.restype = sz
         L.moe_decode_pack_bytes.restype = sz
@@ -321,15 +324,54 @@ class ExpertCacheLayer:
 
 
 # ------------------------------------------------------------- operations --
-def qgemv_affine(W, x, y=None, status=None):
-    """y[b] = W x[b] for x [B][K] float16 (B <= 32).  Returns y [B][N] float16."""
+# zero-filled workspace of qgemv_affine_ws, one per device (allocated by the
+# first call that needs it, so a CUDA graph captured after a first call
+# reuses it); calls that can run at the same time on different streams must
+# pass their own workspace
+_qgemv_ws = {}
+
+
+def qgemv_workspace(W, batch, device=None):
+    """A zero-filled workspace for qgemv_affine_ws calls on W at this batch
+    (None when none is needed)."""
+    need = lib().qgemv_affine_workspace_bytes(W.rows, W.cols, W.bits, batch)
+    if not need:
+        return None
+    return torch.zeros(need, dtype=torch.uint8, device=device or torch.device("cuda"))
+
+
+def _shared_workspace(nbytes, device):
+    ws = _qgemv_ws.get(device.index)
+    if ws is None or ws.numel() < nbytes:
+        if torch.cuda.is_current_stream_capturing():
+            raise RuntimeError("qgemv_affine: no workspace of %d bytes yet on this device; call it "
+                               "once before capturing, or pass workspace=" % nbytes)
+        ws = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _qgemv_ws[device.index] = ws
+    return ws
+
+
+def qgemv_affine(W, x, y=None, status=None, one_pass=True, workspace=None):
+    """y[b] = W x[b] for x [B][K] float16 (B <= 32).  Returns y [B][N] float16.
+    A batch of 9..32 runs in one pass over the weights (qgemv_affine_ws) where
+    the shape allows it, with `workspace` (a zero-filled uint8 tensor, see
+    qgemv_workspace) or else one kept per device; one_pass=False runs one
+    qGEMV launch per 8 rows (qgemv_affine)."""
     x = _need(x, torch.float16, "x")
     x2 = x.reshape(-1, W.cols)
+    B = x2.shape[0]
     if y is None:
-        y = torch.empty(x2.shape[0], W.rows, dtype=torch.float16, device=x.device)
-    _need(y, torch.float16, "y", (x2.shape[0], W.rows))
-    _check(lib().qgemv_affine(ctypes.byref(W.c), _ptr(x2), x2.shape[0], _ptr(y), _ptr(status),
-                              _stream()), "qgemv_affine")
+        y = torch.empty(B, W.rows, dtype=torch.float16, device=x.device)
+    _need(y, torch.float16, "y", (B, W.rows))
+    need = lib().qgemv_affine_workspace_bytes(W.rows, W.cols, W.bits, B) if one_pass and B > 8 else 0
+    if need:
+        ws = workspace if workspace is not None else _shared_workspace(need, x.device)
+        _check(lib().qgemv_affine_ws(ctypes.byref(W.c), _ptr(x2), B, _ptr(y), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _ptr(status), _stream()),
+               "qgemv_affine_ws")
+    else:
+        _check(lib().qgemv_affine(ctypes.byref(W.c), _ptr(x2), B, _ptr(y), _ptr(status),
+                                  _stream()), "qgemv_affine")
     return y
 
 

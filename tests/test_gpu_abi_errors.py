@@ -26,6 +26,31 @@ def call_qgemv(c, x, batch, y):
                                    None, None)
 
 
+def call_qgemv_ws(c, x, batch, y, ws, nbytes):
+    return qmoe.lib().qgemv_affine_ws(ctypes.byref(c), ctypes.c_void_p(x), batch, ctypes.c_void_p(y),
+                                      ctypes.c_void_p(ws), nbytes, None, None)
+
+
+def test_qgemv_ws_argument_errors(cuda_dev):
+    rows, cols = 64, 4096
+    x = torch.zeros(32 * cols, dtype=torch.float16, device="cuda")
+    y = torch.zeros(32 * rows, dtype=torch.float16, device="cuda")
+    good, k1 = mat(rows, cols)
+    need = qmoe.lib().qgemv_affine_workspace_bytes(rows, cols, 4, 32)
+    assert need > 0
+    ws = torch.zeros(need + 64, dtype=torch.uint8, device="cuda")
+    assert call_qgemv_ws(good, x.data_ptr(), 32, y.data_ptr(), ws.data_ptr(), need) == 0
+    assert call_qgemv_ws(good, x.data_ptr(), 32, y.data_ptr(), None, 0) == INVALID
+    assert call_qgemv_ws(good, x.data_ptr(), 32, y.data_ptr(), ws.data_ptr(), need - 16) == INVALID
+    assert call_qgemv_ws(good, x.data_ptr(), 32, y.data_ptr(), ws.data_ptr() + 8, need) == ALIGN
+    assert call_qgemv_ws(good, x.data_ptr(), 33, y.data_ptr(), ws.data_ptr(), need) == INVALID
+    # batch <= 8 needs no workspace
+    assert call_qgemv_ws(good, x.data_ptr(), 8, y.data_ptr(), None, 0) == 0
+    assert qmoe.lib().qgemv_affine_workspace_bytes(rows, cols, 3, 32) == 0
+    assert qmoe.lib().qgemv_affine_workspace_bytes(rows, cols, 4, 0) == 0
+    torch.cuda.synchronize()
+
+
 def test_qgemv_argument_errors(cuda_dev):
     x = torch.zeros(8 * 256, dtype=torch.float16, device="cuda")
     y = torch.zeros(8 * 64, dtype=torch.float16, device="cuda")

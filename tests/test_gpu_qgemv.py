@@ -83,17 +83,85 @@ def test_tensor_copy_tiles_with_row_tail(cuda_dev, bits, N, K):
         assert_close(y.view(np.float16), y64, what="N=%d K=%d B=%d bits=%d" % (N, K, Bt, bits))
 
 
+@pytest.mark.parametrize("one_pass", [True, False])
 @pytest.mark.parametrize("bits", [4, 8])
-@pytest.mark.parametrize("N,K", [(512, 1024), (1000, 4096), (136, 192)])
-def test_small_m_batches(cuda_dev, bits, N, K):
+@pytest.mark.parametrize("N,K", [(512, 1024), (1000, 4096), (136, 192), (256, 8192)])
+def test_small_m_batches(cuda_dev, bits, N, K, one_pass):
     """Batches of 9-32 rows (e.g. the draft tokens a speculative-decoding step
-    verifies), including ragged last slices of 8."""
+    verifies): the one-pass product (K split into 1, 2, 4 or 8 slices by batch
+    and K, ragged last tiles at N=1000; K=192 is a shape it does not take and
+    runs the slices) and one launch per 8 rows (ragged last slices)."""
+    if not one_pass and bits == 8 and K == 8192:
+        pytest.skip("x of 8 rows and a 16-row tile of 8192-wide 8-bit rows exceed shared memory")
     P, S, B = synth.qmatrix(synth.rng(N, K, bits, 11), N, K, bits)
+    W = qmoe.QMatrix.from_numpy(P, S, B, N, K, bits)
     for Bt in (9, 16, 29, 32):
         x16 = synth.activations(N + 3 * Bt, Bt, K)
-        y = run_qgemv(P, S, B, N, K, bits, x16)
+        y = f16_bits(qmoe.qgemv_affine(W, to_dev_f16(x16), one_pass=one_pass))
+        assert qmoe.qmoe_check_status() == 0
         y64, _ = oracle.qgemv(P, S, B, N, K, bits, x16)
-        assert_close_rows(y.view(np.float16), y64, what="N=%d K=%d B=%d bits=%d" % (N, K, Bt, bits))
+        assert_close_rows(y.view(np.float16), y64,
+                          what="N=%d K=%d B=%d bits=%d one_pass=%s" % (N, K, Bt, bits, one_pass))
+
+
+def test_small_m_workspace_plan(cuda_dev):
+    """Workspace sizes of the one-pass product: none for batch <= 8, for one
+    slice or for a shape it does not take; partial tiles + counters otherwise."""
+    ws = qmoe.lib().qgemv_affine_workspace_bytes
+    assert ws(14336, 4096, 4, 8) == 0
+    assert ws(512, 1024, 4, 32) == 0          # x of 32 x 1024 fits: one slice
+    assert ws(136, 192, 4, 32) == 0           # rows of 96 bytes: not taken
+    # K=4096, batch 32: 4 slices of 1024, 64-row tiles, 4 n-tiles
+    tiles = 14336 // 64
+    assert ws(14336, 4096, 4, 32) == 65536 + tiles * 4 * (4 * 4 * 32) * 16
+    assert ws(14336, 4096, 4, 16) > 0
+
+
+def test_small_m_workspace_shared_across_shapes(cuda_dev):
+    """One workspace serving calls of different shapes in turn (the binding
+    keeps one per stream): counters live in a fixed region that every call
+    leaves at zero, so a shape never reads another's partial tiles as
+    counters."""
+    cases = [(1000, 4096, 4, 32), (1000, 4096, 8, 9), (256, 8192, 4, 29), (1000, 4096, 8, 32),
+             (1000, 4096, 4, 16), (256, 8192, 8, 16)]
+    mats = {}
+    for rnd in range(2):
+        for N, K, bits, Bt in cases:
+            if (N, K, bits) not in mats:
+                P, S, B = synth.qmatrix(synth.rng(N, K, bits, 21), N, K, bits)
+                mats[(N, K, bits)] = (P, S, B, qmoe.QMatrix.from_numpy(P, S, B, N, K, bits))
+            P, S, B, W = mats[(N, K, bits)]
+            x16 = synth.activations(N + Bt + rnd, Bt, K)
+            y = f16_bits(qmoe.qgemv_affine(W, to_dev_f16(x16)))
+            y64, _ = oracle.qgemv(P, S, B, N, K, bits, x16)
+            assert_close_rows(y.view(np.float16), y64, what="%s round %d" % ((N, K, bits, Bt), rnd))
+    assert qmoe.qmoe_check_status() == 0
+
+
+def test_small_m_repeat_bitwise_identical(cuda_dev):
+    """The partial tiles are added in slice order whichever CTA finishes last:
+    repeated calls give the same bits (and leave the counters at zero)."""
+    N, K = 14336, 4096
+    P, S, B = synth.dense(1, N, K)
+    W = qmoe.QMatrix.from_numpy(P, S, B, N, K, 4)
+    x = to_dev_f16(synth.activations(5, 32, K))
+    y0 = f16_bits(qmoe.qgemv_affine(W, x))
+    for _ in range(5):
+        assert np.array_equal(f16_bits(qmoe.qgemv_affine(W, x)), y0)
+    assert qmoe.qmoe_check_status() == 0
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("Bt", [16, 32])
+def test_k4096_small_m_full(cuda_dev, Bt):
+    """K=4096, N=14336 (the decode sweep's large matrix) at batch 16 and 32,
+    every output against the oracle, row by row."""
+    N, K = 14336, 4096
+    P, S, B = synth.dense(1, N, K)
+    x16 = synth.activations(40 + Bt, Bt, K)
+    y = run_qgemv(P, S, B, N, K, 4, x16)
+    y64, _ = oracle.qgemv(P, S, B, N, K, 4, x16)
+    assert_close_rows(y.view(np.float16), y64, what="K=4096 N=%d B=%d" % (N, Bt))
 
 
 def test_zero_input_positive_zero(cuda_dev):
