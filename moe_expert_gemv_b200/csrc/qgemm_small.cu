@@ -252,33 +252,36 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
                 const float s_hi = __half2float(sc[r_hi * L.GS + g]) * kCodeScale;
                 const float b_lo = __half2float(bi[r_lo * L.GS + g]);
                 const float b_hi = __half2float(bi[r_hi * L.GS + g]);
-                // every n-tile's first mma before the dependent ones
+                // one mma per accumulator first, then the dependent ones
                 float c[NT][4], d[NT][4];
-                uint4 x1[NT];
+                uint4 x0[NT], x1[NT];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const int n = nt * 8 + gid;
-                    uint4 x0 = make_uint4(0, 0, 0, 0);
-                    x1[nt] = x0;
+                    x0[nt] = make_uint4(0, 0, 0, 0);
+                    x1[nt] = x0[nt];
                     if (n < a.B) {
-                        x0 = xs[((g * 2 + 0) * a.B + n) * 4 + tig];
+                        x0[nt] = xs[((g * 2 + 0) * a.B + n) * 4 + tig];
                         x1[nt] = xs[((g * 2 + 1) * a.B + n) * 4 + tig];
                     }
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
                         c[nt][i] = d[nt][i] = 0.f;
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
                     if (BITS == 4) {
-                        mma_16816(c[nt], pa[0], pb[0], pa[2], pb[2], x0.x, x0.y);
-                        mma_16816(c[nt], pa[4], pb[4], pa[6], pb[6], x0.z, x0.w);
+                        mma_16816(c[nt], pa[0], pb[0], pa[2], pb[2], x0[nt].x, x0[nt].y);
+                        mma_16816(d[nt], pa[1], pb[1], pa[3], pb[3], x1[nt].x, x1[nt].y);
                     } else {
-                        mma_16816(c[nt], pa[0], pb[0], pa[1], pb[1], x0.x, x0.y);
-                        mma_16816(d[nt], pa[2], pb[2], pa[3], pb[3], x0.z, x0.w);
+                        mma_16816(c[nt], pa[0], pb[0], pa[1], pb[1], x0[nt].x, x0[nt].y);
+                        mma_16816(d[nt], pa[2], pb[2], pa[3], pb[3], x0[nt].z, x0[nt].w);
                     }
                 }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     if (BITS == 4) {
-                        mma_16816(d[nt], pa[1], pb[1], pa[3], pb[3], x1[nt].x, x1[nt].y);
+                        mma_16816(c[nt], pa[4], pb[4], pa[6], pb[6], x0[nt].z, x0[nt].w);
                         mma_16816(d[nt], pa[5], pb[5], pa[7], pb[7], x1[nt].z, x1[nt].w);
                     } else {
                         mma_16816(c[nt], pa[4], pb[4], pa[5], pb[5], x1[nt].x, x1[nt].y);
