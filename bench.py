@@ -61,7 +61,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["moe_decode", "qgemv", "qgemv_fmt", "router", "prefill",
-                                           "expert_cache"],
+                                           "expert_cache", "expert_parallel"],
                     default="moe_decode")
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--qgemv-batch", default="1,4,8,16,32",
@@ -487,6 +487,44 @@ def main_other(args):
                                            "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
                                            "rotated_copies": copies})
                 del Ws
+    elif args.workload == "expert_parallel":
+        # one 128-expert layer split over `world` ranks: every rank's share
+        # (moe_expert_qmlp_ep) timed on this GPU, rotating over 8 layers so the
+        # weights come from HBM; the all-reduce of the 11 KB partial is not
+        # included (it needs the other GPUs)
+        nl = 8
+        ms_l = [synth.moe_layer(args.seed, l) for l in range(nl)]
+        xs = [torch.from_numpy(synth.activations(args.seed, 1, H, layer=l).view(np.float16).copy())
+              .to(dev).reshape(-1) for l in range(nl)]
+        routed = []
+        for l in range(nl):
+            G = qmoe.MoELayer.from_numpy(ms_l[l], E, H, I, device=dev)
+            idx, wt, _ = qmoe.moe_router_topk(G.router, xs[l].reshape(1, -1), TOPK)
+            routed.append((idx.reshape(-1), wt.reshape(-1)))
+            del G
+        for world in (1, 2, 4, 8):
+            times = []
+            for r in range(world):
+                Gs = [qmoe.MoELayer.from_numpy(ms_l[l], E, H, I, device=dev, rank=r, world=world)
+                      for l in range(nl)]
+                ws = qmoe.expert_workspace(Gs[0], TOPK, dev)
+                yp = torch.empty(H, dtype=torch.float32, device=dev)
+
+                def run():
+                    for l in range(nl):
+                        qmoe.moe_expert_qmlp_ep(Gs[l], xs[l], routed[l][0], routed[l][1], r, world,
+                                                yp, ws)
+                run()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    run()
+                for _ in range(3):
+                    g.replay()
+                reps = max(10, args.steps // 10)
+                times.append(timed_replays(g.replay, reps) / (reps * nl) * 1e3)
+                del Gs, g
+            out["results"].append({"world": world, "us_per_rank": [round(t, 2) for t in times],
+                                   "us_max_rank": round(max(times), 2)})
     elif args.workload == "expert_cache":
         # one 128-expert H=2816 layer with its routed experts in pinned host memory and
         # 16 device slots; decode tokens whose routing locality is set by rho

@@ -228,6 +228,31 @@ qmoe_status moe_expert_qmlp(const qmoe_moe_layer *L, const uint16_t *x, const in
                             const float *weights, int32_t top_k, uint16_t *y, void *workspace,
                             size_t workspace_bytes, int32_t *status_dev, void *stream);
 
+/* ---------------------------------------------------------------------------
+ * Expert-parallel share of the same layer: with the experts split over
+ * `world` ranks (rank r holds experts r*E/world .. (r+1)*E/world - 1) and the
+ * router replicated, rank `rank` computes only the routed slots whose expert
+ * it holds, plus the shared expert on rank 0.  L->num_experts is the global
+ * E; L->gate, up and down stack only the E/world experts this rank holds
+ * (local expert i is global expert rank*E/world + i):
+ *   y_partial = [rank == 0] shared(x) + sum_{j: idx[j] held here} weights[j] expert_{idx[j]}(x)
+ * in fp32, so that the sum over ranks (one all-reduce of [hidden] fp32) is
+ * the layer output before its rounding to fp16 (qmoe_f32_to_f16).  Only the
+ * weights of the held experts are read.  A rank that holds none of the
+ * chosen experts (and is not rank 0) gets zeros.  An invalid id belongs to
+ * no rank.  world divides num_experts; rank in 0..world-1.  y_partial: fp32
+ * [hidden], 4-byte aligned.  Workspace and errors as moe_expert_qmlp.
+ * (Page: the routed experts of a token are independent products added
+ * together, TurboFieldfare article, section "내부 구조가 진짜 흥미로운 부분".)
+ * ------------------------------------------------------------------------- */
+qmoe_status moe_expert_qmlp_ep(const qmoe_moe_layer *L, const uint16_t *x, const int32_t *idx,
+                               const float *weights, int32_t top_k, int32_t rank, int32_t world,
+                               float *y_partial, void *workspace, size_t workspace_bytes,
+                               int32_t *status_dev, void *stream);
+
+/* fp32 [n] -> fp16 [n], round to nearest even, on `stream`. */
+qmoe_status qmoe_f32_to_f16(const float *src, uint16_t *dst, int64_t n, void *stream);
+
 /* moe_expert_qmlp for callers that cannot allocate device memory.  The pages
  * have no counterpart: this exists for callers with no way to obtain a
  * workspace -- a plugin or embedded runtime handed only a stream and tensor

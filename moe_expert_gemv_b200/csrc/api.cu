@@ -397,6 +397,49 @@ qmoe_status moe_expert_qmlp(const qmoe_moe_layer *L, const uint16_t *x, const in
     return cuda_status(launch_expert_down(a, c));
 }
 
+qmoe_status moe_expert_qmlp_ep(const qmoe_moe_layer *L, const uint16_t *x, const int32_t *idx,
+                               const float *weights, int32_t top_k, int32_t rank, int32_t world,
+                               float *y_partial, void *workspace, size_t workspace_bytes,
+                               int32_t *status_dev, void *stream)
+{
+    qmoe_status s = check_expert_common(L, top_k);
+    if (s != QMOE_OK)
+        return s;
+    if (!x || !idx || !weights || !y_partial || world < 1 || rank < 0 || rank >= world ||
+        L->num_experts % world)
+        return QMOE_ERR_INVALID_ARG;
+    if (!aligned(x, 2) || !aligned(idx, 4) || !aligned(weights, 4) || !aligned(y_partial, 4) ||
+        (status_dev && !aligned(status_dev, 4)))
+        return QMOE_ERR_ALIGNMENT;
+    DevState *d;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    ExpertArgs a;
+    if ((s = expert_args(L, x, idx, weights, top_k, nullptr, workspace, workspace_bytes,
+                         status_dev ? status_dev : d->status, &a)) != QMOE_OK)
+        return s;
+    a.ep_rank = rank;
+    a.ep_world = world;
+    a.ep_first = rank * (L->num_experts / world);
+    a.y_part = y_partial;
+    const LaunchCfg c = launch_cfg(d, stream);
+    if ((s = cuda_status(launch_expert_gateup(a, c))) != QMOE_OK)
+        return s;
+    return cuda_status(launch_expert_down(a, c));
+}
+
+qmoe_status qmoe_f32_to_f16(const float *src, uint16_t *dst, int64_t n, void *stream)
+{
+    if (!src || !dst || n < 0)
+        return QMOE_ERR_INVALID_ARG;
+    if (!aligned(src, 4) || !aligned(dst, 2))
+        return QMOE_ERR_ALIGNMENT;
+    if (n == 0)
+        return QMOE_OK;
+    return cuda_status(launch_f32_to_f16(src, reinterpret_cast<__half *>(dst), (long)n,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 size_t moe_decode_pack_bytes(const qmoe_moe_layer *L)
 {
     if (!L || L->num_experts < 1 || L->hidden < 256 || L->inter < 64)

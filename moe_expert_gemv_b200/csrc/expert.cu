@@ -21,6 +21,10 @@
 //           that the combining warp resets), so the output is deterministic.
 // Weights of the shared expert are streamed before the previous kernel of
 // the stream has completed; routed weights follow once the ids are visible.
+// Expert parallelism (EP = true, a separate instantiation so the one-GPU
+// kernels carry no ownership test): a rank skips the slots whose expert it
+// does not hold, before the copy and before the compute, and adds only its
+// own slots into an fp32 partial.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -89,6 +93,23 @@ __device__ __forceinline__ int routed_expert(const ExpertArgs &a, int j, bool *v
     return *valid ? e : 0;
 }
 
+// The slots this rank holds, as bits: bit 0 the shared expert (rank 0),
+// bit j + 1 routed slot j when its expert e has e / (E / ep_world) ==
+// ep_rank (an invalid id belongs to no rank).  One load per id, made once
+// per thread after the ids are complete (top_k <= 16).
+__device__ __forceinline__ uint32_t owned_slots(const ExpertArgs &a)
+{
+    uint32_t m = a.ep_rank == 0 ? 1u : 0u;
+    const int per = a.E / a.ep_world;
+    for (int j = 0; j < a.top_k; ++j) {
+        const int e = __ldcg(a.idx + j);
+        if (e >= 0 && e < a.E && e / per == a.ep_rank)
+            m |= 1u << (j + 1);
+    }
+    return m;
+}
+
+template <bool EP>
 __global__ void __launch_bounds__(GU_THREADS, 1) expert_gateup_kernel(ExpertArgs a)
 {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -119,21 +140,26 @@ __global__ void __launch_bounds__(GU_THREADS, 1) expert_gateup_kernel(ExpertArgs
             bool waited = false, bad = false;
             int last_use[GU_STAGES] = {-1, -1, -1};
             int k = 0;
-            for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
+            uint32_t mine = a.ep_rank == 0 ? 1u : 0u;   // before the ids: the shared slot only
+            for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
                 const int so = item / octs, oct = item % octs;
                 QMat g = a.sh_gate, u = a.sh_up;
                 size_t mat_off = 0;   // in rows
+                if (so > 0 && !waited) {
+                    pdl_wait();   // the ids come from the previous kernel
+                    waited = true;
+                    if (EP)
+                        mine = owned_slots(a);
+                }
+                if (EP && !((mine >> so) & 1u))
+                    continue;
                 if (so > 0) {
-                    if (!waited) {
-                        pdl_wait();   // the ids come from the previous kernel
-                        waited = true;
-                    }
                     bool valid;
                     const int e = routed_expert(a, so - 1, &valid);
                     bad |= !valid;
                     g = a.gate;
                     u = a.up;
-                    mat_off = (size_t)e * a.I;
+                    mat_off = (size_t)(e - a.ep_first) * a.I;   // held slots only: e >= ep_first
                 }
                 const int st = k % GU_STAGES, use = k / GU_STAGES;
                 if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, a.status))
@@ -155,6 +181,7 @@ __global__ void __launch_bounds__(GU_THREADS, 1) expert_gateup_kernel(ExpertArgs
                 bulk_g2s(bi, g.biases + r0 * L.G, sb8, &full[st], pol);
                 bulk_g2s(bi + sb8, u.biases + r0 * L.G, sb8, &full[st], pol);
                 last_use[st] = use;
+                ++k;
             }
             if (bad)
                 flag_status(a.status, QMOE_DEV_BAD_EXPERT);
@@ -174,9 +201,13 @@ __global__ void __launch_bounds__(GU_THREADS, 1) expert_gateup_kernel(ExpertArgs
     named_bar_sync(1, GU_CW * 32);
 
     const int gid = lane >> 2, tig = lane & 3;
+    const uint32_t mine = EP ? owned_slots(a) : ~0u;   // after the wait above
     bool failed = false;
-    int k = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
+    int k = -1;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        if (EP && !((mine >> (item / octs)) & 1u))
+            continue;
+        ++k;
         const int st = k % GU_STAGES, use = k / GU_STAGES;
         if (!failed && !mbar_wait(&full[st], use & 1, a.status))
             failed = true;
@@ -247,6 +278,7 @@ __host__ __device__ inline DnLayout dn_layout(int I, int top_k, int NS)
     return L;
 }
 
+template <bool EP>
 __global__ void __launch_bounds__(DN_THREADS, 1) expert_down_kernel(ExpertArgs a, int NS)
 {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -280,14 +312,17 @@ __global__ void __launch_bounds__(DN_THREADS, 1) expert_down_kernel(ExpertArgs a
             for (int s = 0; s < DN_MAX_STAGES; ++s)
                 last_use[s] = -1;
             int k = 0;
-            for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
+            const uint32_t mine = EP ? owned_slots(a) : ~0u;
+            for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
                 const int so = item / tiles, tile = item % tiles;
+                if (EP && !((mine >> so) & 1u))
+                    continue;
                 QMat d = a.sh_down;
                 size_t mat_off = 0;
                 if (so > 0) {
                     const int e = __ldcg(a.idx + (so - 1));
                     d = a.down;
-                    mat_off = (size_t)((e >= 0 && e < a.E) ? e : 0) * a.H;
+                    mat_off = (size_t)((e >= 0 && e < a.E) ? e - a.ep_first : 0) * a.H;
                 }
                 const int st = k % NS, use = k / NS;
                 if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, a.status))
@@ -307,6 +342,7 @@ __global__ void __launch_bounds__(DN_THREADS, 1) expert_down_kernel(ExpertArgs a
                 bulk_g2s(stage + L.codes_bytes, d.scales + r0 * L.G, sb, &full[st], pol);
                 bulk_g2s(stage + L.codes_bytes + L.sb_bytes, d.biases + r0 * L.G, sb, &full[st], pol);
                 last_use[st] = use;
+                ++k;
             }
             for (int s = 0; s < NS; ++s)
                 if (last_use[s] >= 0)
@@ -330,10 +366,22 @@ __global__ void __launch_bounds__(DN_THREADS, 1) expert_down_kernel(ExpertArgs a
                threadIdx.x, DN_CW * 32);
     named_bar_sync(1, DN_CW * 32);
 
+    // slots of this rank: each tile is complete after that many arrivals
+    const uint32_t mine = EP ? owned_slots(a) : ~0u;
+    const int n_owned = EP ? __popc(mine) : nslot;
+    if (n_owned == 0) {   // nothing to add here: this rank's share is zero
+        if (a.y_part)
+            for (int row = blockIdx.x * DN_CW * 32 + threadIdx.x; row < a.H; row += gridDim.x * DN_CW * 32)
+                a.y_part[row] = 0.f;
+        return;
+    }
     const int gid = lane >> 2, tig = lane & 3;
     bool failed = false;
-    int k = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
+    int k = -1;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        if (EP && !((mine >> (item / tiles)) & 1u))
+            continue;
+        ++k;
         if (k % DN_CW != warp)
             continue;
         const int st = k % NS, use = k / NS;
@@ -366,17 +414,20 @@ __global__ void __launch_bounds__(DN_THREADS, 1) expert_down_kernel(ExpertArgs a
         if (lane == 0)
             old = atomicAdd(reinterpret_cast<int *>(a.ws.counters + tile), 1);
         old = __shfl_sync(0xffffffffu, old, 0);
-        if (old == nslot - 1) {
+        if (old == n_owned - 1) {
             __threadfence();
             if (lane < 16) {
                 const int row = r0 + lane;
-                float v = __ldcg(a.ws.part + (size_t)a.top_k * a.H + row);
+                float v = (mine & 1u) ? __ldcg(a.ws.part + (size_t)a.top_k * a.H + row) : 0.f;
                 for (int j = 0; j < a.top_k; ++j) {
                     const int e = __ldcg(a.idx + j);
-                    if (e >= 0 && e < a.E)
+                    if (e >= 0 && e < a.E && ((mine >> (j + 1)) & 1u))
                         v = fmaf(__ldcg(a.weights + j), __ldcg(a.ws.part + (size_t)j * a.H + row), v);
                 }
-                a.y[row] = __float2half_rn(v);
+                if (a.y_part)
+                    a.y_part[row] = v;
+                else
+                    a.y[row] = __float2half_rn(v);
             }
             if (lane == 0)
                 a.ws.counters[tile] = 0;
@@ -393,10 +444,12 @@ cudaError_t launch_expert_gateup(const ExpertArgs &a, const LaunchCfg &c)
         return cudaErrorInvalidValue;
     const int n_items = (a.top_k + 1) * (a.I / 8);
     const int grid = n_items < c.num_sms ? n_items : c.num_sms;
-    cudaError_t e = set_smem(expert_gateup_kernel, L.total);
+    const bool ep = a.ep_world > 1;
+    cudaError_t e = ep ? set_smem(expert_gateup_kernel<true>, L.total) : set_smem(expert_gateup_kernel<false>, L.total);
     if (e != cudaSuccess)
         return e;
-    return launch_ex(expert_gateup_kernel, dim3(grid), dim3(GU_THREADS), L.total, c, 1, a);
+    return ep ? launch_ex(expert_gateup_kernel<true>, dim3(grid), dim3(GU_THREADS), L.total, c, 1, a)
+              : launch_ex(expert_gateup_kernel<false>, dim3(grid), dim3(GU_THREADS), L.total, c, 1, a);
 }
 
 cudaError_t launch_expert_down(const ExpertArgs &a, const LaunchCfg &c)
@@ -411,10 +464,12 @@ cudaError_t launch_expert_down(const ExpertArgs &a, const LaunchCfg &c)
     const DnLayout L = dn_layout(a.I, a.top_k, NS);
     const int n_items = (a.top_k + 1) * (a.H / 16);
     const int grid = n_items < c.num_sms ? n_items : c.num_sms;
-    cudaError_t e = set_smem(expert_down_kernel, L.total);
+    const bool ep = a.ep_world > 1;
+    cudaError_t e = ep ? set_smem(expert_down_kernel<true>, L.total) : set_smem(expert_down_kernel<false>, L.total);
     if (e != cudaSuccess)
         return e;
-    return launch_ex(expert_down_kernel, dim3(grid), dim3(DN_THREADS), L.total, c, 1, a, NS);
+    return ep ? launch_ex(expert_down_kernel<true>, dim3(grid), dim3(DN_THREADS), L.total, c, 1, a, NS)
+              : launch_ex(expert_down_kernel<false>, dim3(grid), dim3(DN_THREADS), L.total, c, 1, a, NS);
 }
 
 }  // namespace qmoe

@@ -102,9 +102,16 @@ struct ExpertArgs {
     __half *y;              // [H]
     ExpertWorkspace ws;
     int32_t *status;
+    // expert parallelism: this rank computes the routed slots whose expert
+    // e has e / (E / ep_world) == ep_rank, and the shared expert on rank 0;
+    // gate/up/down stack only its experts, from expert ep_first on; with
+    // y_part set, the sum of its slots goes there in fp32 instead of y
+    int ep_rank = 0, ep_world = 1, ep_first = 0;
+    float *y_part = nullptr;   // [H]
 };
 cudaError_t launch_expert_gateup(const ExpertArgs &a, const LaunchCfg &c);
 cudaError_t launch_expert_down(const ExpertArgs &a, const LaunchCfg &c);
+cudaError_t launch_f32_to_f16(const float *src, __half *dst, long n, cudaStream_t s);
 
 // ------------------------------------------------ fused multi-layer decode --
 constexpr int kDecodeMaxLayers = 32;

@@ -145,4 +145,21 @@ cudaError_t launch_group(const GroupArgs &a, const LaunchCfg &c)
     return launch_ex(group_kernel, dim3(1), dim3(GR_THREADS), smem, c, 1, a);
 }
 
+// fp32 -> fp16, round to nearest even (the last step of an expert-parallel
+// layer: the all-reduced fp32 partials become the fp16 layer output)
+namespace {
+__global__ void f32_to_f16_kernel(const float *src, __half *dst, long n)
+{
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
+        dst[i] = __float2half_rn(src[i]);
+}
+}  // namespace
+
+cudaError_t launch_f32_to_f16(const float *src, __half *dst, long n, cudaStream_t s)
+{
+    const long blocks = (n + 255) / 256;
+    f32_to_f16_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, s>>>(src, dst, n);
+    return cudaGetLastError();
+}
+
 }  // namespace qmoe

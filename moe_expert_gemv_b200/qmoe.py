@@ -54,6 +54,8 @@ def lib():
             "qgemv_affine": [p, p, i32, p, p, p],
             "qgemv_affine_workspace_bytes": [i32, i32, i32, i32],
             "qgemv_affine_ws": [p, p, i32, p, p, sz, p, p],
+            "moe_expert_qmlp_ep": [p, p, p, p, i32, i32, i32, p, p, sz, p, p],
+            "qmoe_f32_to_f16": [p, p, ctypes.c_int64, p],
             "qgemv_fmt": [p, p, i32, p, p, p],
             "moe_router_topk": [p, p, i32, i32, p, p, p, p, p],
             "moe_expert_workspace_bytes": [p, i32],
@@ -209,17 +211,70 @@ class MoELayer:
                            hidden, inter)
 
     @classmethod
-    def from_numpy(cls, m, E, H, I, device="cuda"):
-        """From a dict like moe_expert_gemv_b200.synth.moe_layer() returns."""
+    def from_numpy(cls, m, E, H, I, device="cuda", rank=0, world=1):
+        """From a dict like moe_expert_gemv_b200.synth.moe_layer() returns.
+        With world > 1, the routed gate/up/down keep only the E/world experts
+        rank `rank` holds (for moe_expert_qmlp_ep); shared expert and router
+        are whole on every rank."""
+        if E % world or not 0 <= rank < world:
+            raise ValueError("world must divide E and 0 <= rank < world")
+        lo, hi = rank * (E // world), (rank + 1) * (E // world)
         q = {}
         for name, rows, cols in (("gate", I, H), ("up", I, H), ("down", H, I),
                                  ("sh_gate", I, H), ("sh_up", I, H), ("sh_down", H, I)):
-            q[name] = QMatrix.from_numpy(*m[name], rows, cols, 4, device)
+            arrs = m[name]
+            if world > 1 and not name.startswith("sh_"):
+                arrs = tuple(a[lo:hi] for a in arrs)
+            q[name] = QMatrix.from_numpy(*arrs, rows, cols, 4, device)
         router = None
         if "router" in m:
             router = QMatrix.from_numpy(*m["router"], E, H, 8, device)
         return cls(q["gate"], q["up"], q["down"], q["sh_gate"], q["sh_up"], q["sh_down"], E, H,
                    I, router)
+
+
+def expert_owner(e, E, world):
+    """Rank that holds expert e when E experts are split over `world` ranks."""
+    return e // (E // world)
+
+
+def moe_expert_qmlp_ep(G, x, idx, weights, rank, world, y_partial=None, workspace=None,
+                       status=None):
+    """This rank's share of an expert-parallel MoE layer (G from
+    MoELayer.from_numpy(..., rank=rank, world=world)): fp32 [H] partial,
+    shared expert on rank 0.  The partials of all ranks sum to the layer
+    output before its rounding to fp16."""
+    x = _need(x, torch.float16, "x")
+    top_k = idx.numel()
+    if y_partial is None:
+        y_partial = torch.empty(G.hidden, dtype=torch.float32, device=x.device)
+    _need(y_partial, torch.float32, "y_partial", (G.hidden,))
+    ws = workspace if workspace is not None else expert_workspace(G, top_k, x.device)
+    _check(lib().moe_expert_qmlp_ep(ctypes.byref(G.c), _ptr(x), _ptr(idx), _ptr(weights), top_k,
+                                    rank, world, _ptr(y_partial), _ptr(ws), ws.numel(), _ptr(status),
+                                    _stream()), "moe_expert_qmlp_ep")
+    return y_partial
+
+
+def f32_to_f16(src, dst=None):
+    """fp32 -> fp16 (round to nearest even) in the library's kernel."""
+    src = _need(src, torch.float32, "src")
+    if dst is None:
+        dst = torch.empty(src.shape, dtype=torch.float16, device=src.device)
+    _check(lib().qmoe_f32_to_f16(_ptr(src), _ptr(dst), src.numel(), _stream()), "qmoe_f32_to_f16")
+    return dst
+
+
+def moe_layer_ep(G, x, idx, weights, group=None, workspace=None):
+    """One expert-parallel MoE layer on this rank of `group` (torch.distributed,
+    NCCL on GPUs): the rank's partial, one all-reduce of the [H] fp32
+    partials, then fp16.  Every rank passes the same x, idx and weights (the
+    router is replicated)."""
+    import torch.distributed as dist
+    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    yp = moe_expert_qmlp_ep(G, x, idx, weights, rank, world, workspace=workspace)
+    dist.all_reduce(yp, group=group)
+    return f32_to_f16(yp)
 
 
 # ------------------------------------------------------- expert streaming --
