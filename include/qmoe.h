@@ -124,8 +124,7 @@ qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch
  * The same product for batch 9..32 in ONE pass over the weights (the
  * verification step of speculative decoding multiplies every projection by
  * the 16-32 draft tokens at once; uzu page, discuss.pytorch.kr, section "uzu의
- * 모델 변환과 Mirai 양자화 형식", lists speculative decoding among the runtime's
- * features).  The K range is split into S slices whose x fits on chip; CTAs
+ * 추측 디코딩 구조").  The K range is split into S slices whose x fits on chip; CTAs
  * of different slices write fp32 partial tiles to `workspace` and the last
  * one to finish a tile adds them in slice order (results do not depend on
  * the order in which CTAs finish; they differ from qgemv_affine's only by

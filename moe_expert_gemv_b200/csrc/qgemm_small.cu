@@ -1,9 +1,9 @@
 // qgemm_small.cu -- dense affine-quantized product for a batch of 9..32 rows
 // of x in ONE pass over the weights: the small-M verification product of a
 // speculative-decoding step (the uzu page, discuss.pytorch.kr, section "uzu의
-// 모델 변환과 Mirai 양자화 형식", lists speculative decoding among the
-// runtime's features; its verification step multiplies every projection by
-// the 16-32 draft tokens at once).  Format: MLX affine 4-bit (8-bit) group 64
+// 추측 디코딩 구조": a draft model proposes 16-32 tokens and the main model
+// checks them in one forward pass, so every projection multiplies 16-32
+// rows of activations at once).  Format: MLX affine 4-bit (8-bit) group 64
 // (TurboFieldfare article, jeff.news, section "성능과 제약").
 //
 //   y[b][n] = sum_g s[n][g] * (sum_{k in g} q[n][k] x[b][k]) + b[n][g] * X[b][g]

@@ -34,3 +34,30 @@ def test_status_strings_without_gpu():
     lib.qmoe_status_string.restype = ctypes.c_char_p
     for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert lib.qmoe_status_string(code).startswith(b"QMOE_")
+
+
+def test_one_pass_workspace_sizes_without_gpu():
+    """qgemv_affine_workspace_bytes is host arithmetic: the one-pass plan for
+    batch 9..32 (K slices whose x fits 64 KB of shared memory, ~32 KB weight
+    tiles) and its workspace (64 KB of tile counters + fp32 partial tiles)."""
+    lib = ctypes.CDLL(build.build())
+    f = lib.qgemv_affine_workspace_bytes
+    f.restype = ctypes.c_size_t
+    f.argtypes = [ctypes.c_int32] * 4
+    # batch <= 8, an unsupported width (rows of 96 bytes) or bad arguments: none
+    assert f(14336, 4096, 4, 8) == 0
+    assert f(136, 192, 4, 32) == 0
+    assert f(14336, 4096, 3, 32) == 0 and f(14336, 4096, 4, 33) == 0 and f(0, 4096, 4, 16) == 0
+    # x of 32 x 1024 fp16 = 64 KB: one slice, no workspace
+    assert f(512, 1024, 4, 32) == 0
+    # K=4096, batch 32: 4 slices of 1024, 64-row tiles, 4 n-tiles of 8 columns
+    tiles = 14336 // 64
+    assert f(14336, 4096, 4, 32) == 65536 + tiles * 4 * (4 * 4 * 32) * 16
+    # batch 16: 2 slices of 2048 (64 KB of x), 32-row tiles (1 KB of codes a row), 2 n-tiles
+    tiles = 14336 // 32
+    assert f(14336, 4096, 4, 16) == 65536 + tiles * 2 * (2 * 2 * 32) * 16
+    # batch 9 rounds up to 2 n-tiles; 8-bit rows of 2048 codes: 16-row tiles
+    tiles = (1000 + 15) // 16
+    assert f(1000, 4096, 8, 9) == 65536 + tiles * 2 * (1 * 2 * 32) * 16
+    # K=8192 at batch 32: 8 slices of 1024
+    assert f(256, 8192, 4, 32) == 65536 + (256 // 64) * 8 * (4 * 4 * 32) * 16
