@@ -134,7 +134,7 @@ qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch
  *   or a shape the one-pass kernel does not take: then qgemv_affine_ws runs
  *   qgemv_affine's path).  The one-pass kernel takes rows of whole 128-byte
  *   code chunks (cols % 256 == 0 at 4 bits, % 128 at 8 bits), slices of a
- *   multiple of 512 inputs, and scales / biases 16-byte aligned (otherwise
+ *   multiple of 512 inputs, x and scales / biases 16-byte aligned (otherwise
  *   it runs qgemv_affine's path even where a workspace was asked for).
  * workspace: device memory, 16-byte aligned, at least that many bytes,
  *   zero-filled once before its first use.  Its first 64 KB hold per-tile

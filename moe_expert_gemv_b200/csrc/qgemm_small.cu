@@ -446,9 +446,12 @@ cudaError_t launch_qgemm_small(const QgemvArgs &a, void *ws, size_t ws_bytes, co
 {
     *used_ws = false;
     const SmPlan p = plan_small(a.N, a.K, a.bits, a.B);
-    const bool sb_ok = ((reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases)) & 15u) == 0 &&
-                       (a.K / kGroup * 2) % 16 == 0;
-    if (!p.ok || !sb_ok || a.fmt != QG_AFFINE || a.signs)
+    // x is read with 16-byte loads; scales and biases by 2-D tensor copies
+    const bool align_ok =
+        ((reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.scales) |
+          reinterpret_cast<uintptr_t>(a.biases)) & 15u) == 0 &&
+        (a.K / kGroup * 2) % 16 == 0;
+    if (!p.ok || !align_ok || a.fmt != QG_AFFINE || a.signs)
         return launch_qgemv_batched(a, c);
     const int per = c.num_sms / p.S, n_tiles = (a.N + p.TM - 1) / p.TM;
     if (per < 1 || (n_tiles + per - 1) / per > SM_MAX_CTA_TILES)

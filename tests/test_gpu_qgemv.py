@@ -138,6 +138,25 @@ def test_small_m_workspace_shared_across_shapes(cuda_dev):
     assert qmoe.qmoe_check_status() == 0
 
 
+@pytest.mark.parametrize("Bt", [4, 16, 32])
+def test_x_only_2_byte_aligned(cuda_dev, Bt):
+    """x may start at any fp16 element: a view one element into its buffer
+    (the one-pass product, which loads x 16 bytes at a time, takes the slice
+    path for it; the slices stage such an x element by element)."""
+    N, K = 1000, 4096
+    P, S, B = synth.dense(7, N, K)
+    W = qmoe.QMatrix.from_numpy(P, S, B, N, K, 4)
+    x16 = synth.activations(70 + Bt, Bt, K)
+    buf = torch.empty(Bt * K + 1, dtype=torch.float16, device="cuda")
+    buf[1:] = to_dev_f16(x16).reshape(-1)
+    x = buf[1:].view(Bt, K)
+    assert x.data_ptr() % 16 == 2
+    y = f16_bits(qmoe.qgemv_affine(W, x))
+    assert qmoe.qmoe_check_status() == 0
+    y64, _ = oracle.qgemv(P, S, B, N, K, 4, x16)
+    assert_close_rows(y.view(np.float16), y64, what="x at +2 bytes, B=%d" % Bt)
+
+
 def test_small_m_repeat_bitwise_identical(cuda_dev):
     """The partial tiles are added in slice order whichever CTA finishes last:
     repeated calls give the same bits (and leave the counters at zero)."""
