@@ -306,9 +306,10 @@ qmoe_status moe_expert_down(const qmoe_moe_layer *L, const int32_t *idx, const f
  * accumulation of exact products).  Layer l+1 starts after layer l has
  * finished, as it would if it consumed y[l]; the weights of later layers
  * that do not depend on the routing are streamed ahead of time.
- * x, y: fp16 [n_layers][hidden]; idx: int32 [n_layers][top_k], weights: fp32
- * [n_layers][top_k], logits: fp32 [n_layers][num_experts]; idx, weights and
- * logits may be NULL.  top_k 1..16.
+ * x, y: fp16 [n_layers][hidden], x 16-byte aligned (it is read 16 bytes at a
+ * time); idx: int32 [n_layers][top_k], weights: fp32 [n_layers][top_k],
+ * logits: fp32 [n_layers][num_experts]; idx, weights and logits may be
+ * NULL.  top_k 1..16.
  * workspace: moe_decode_workspace_bytes() bytes, 16-byte aligned, ZERO-FILLED
  * before first use; each successful call leaves it zero-filled again.  Calls
  * sharing a workspace must not overlap in time.  Stacks of more than 32

@@ -507,7 +507,9 @@ qmoe_status moe_decode_layers(const void *const *packed_layers, int32_t n_layers
         if (!aligned(packed_layers[l], 16))
             return QMOE_ERR_ALIGNMENT;
     }
-    if (!aligned(x, 2) || !aligned(y, 2) || (idx && !aligned(idx, 4)) ||
+    // each layer's x is read with 16-byte loads (hidden % 256 keeps every
+    // layer's row 16-byte aligned once the first is)
+    if (!aligned(x, 16) || !aligned(y, 2) || (idx && !aligned(idx, 4)) ||
         (weights && !aligned(weights, 4)) || (logits && !aligned(logits, 4)) ||
         (status_dev && !aligned(status_dev, 4)))
         return QMOE_ERR_ALIGNMENT;

@@ -180,3 +180,21 @@ def test_fp16_overflow_matches_oracle_rounding(cuda_dev):
         fin = np.isfinite(want)
         den = np.maximum(np.abs(y64[0][fin]), 1e-2 * np.abs(y64[0][fin]).max())
         assert (np.abs(g[fin] - y64[0][fin]) / den).max() <= REL_TOL, what
+
+
+def test_x_alignment_rule(cuda_dev):
+    """The fused decode reads x 16 bytes at a time: an x that starts one fp16
+    element into its buffer is refused before any launch (QMOE_ERR_ALIGNMENT),
+    and the same values 16-byte aligned go through."""
+    E, H, I, k, n = 16, 256, 64, 4, 2
+    ms, stack = make_stack(5, n, E, H, I, k)
+    x16 = np.concatenate([synth.activations(9 + l, 1, H, layer=l) for l in range(n)])
+    buf = torch.empty(n * H + 8, dtype=torch.float16, device="cuda")
+    buf[1:1 + n * H] = torch.from_numpy(x16.view(np.float16).copy()).cuda().reshape(-1)
+    xbad = buf[1:1 + n * H].view(n, H)
+    assert xbad.data_ptr() % 16 == 2
+    with pytest.raises(qmoe.QmoeError) as e:
+        qmoe.moe_decode_layers(stack, xbad)
+    assert e.value.code == -2
+    y, idx, wt, lg = run(stack, x16, E, k)
+    check_layers(ms, E, H, I, k, x16, y, idx, wt, lg)
