@@ -341,7 +341,9 @@ def main_decode(args):
     step_bytes = nl * (LAYER_BYTES + 2 * H * 2)
     gbs = step_bytes / (launch_ms / 1e3) / 1e9
     trf = NCU_TRAFFIC.get("moe_decode_kernel")
-    traffic = trf["bytes"] if trf and trf["sha"] == source_sha("decode.cu") else None
+    # traffic grows in proportion to the layers a launch streams
+    traffic = (round(trf["bytes"] * nl / 30) if trf and trf["sha"] == source_sha("decode.cu")
+               else None)
     line = {
         "metric": "qGEMV/MoE-layer weight-stream GB/s vs HBM peak; MoE decode layers/s",
         "value": round(value, 1),
