@@ -75,3 +75,52 @@ def test_expert_parallel_partials_sum_to_layer(tmp_path):
     assert res[0]["owners"] == [0] * 8 + [1] * 8
     held = sorted(res[0]["held"] + res[1]["held"])
     assert held == sorted(res[0]["idx"])
+
+
+def _plumbing_main(rank, world, port, out_dir):
+    """moe_layer_ep's host side under gloo: each rank's share (a stand-in for
+    the device kernel: a vector of rank + 1), the all-reduce over the group,
+    the fp16 conversion (a stand-in for the library's kernel)."""
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+
+    from moe_expert_gemv_b200 import qmoe
+
+    dist.init_process_group("gloo", init_method="tcp://127.0.0.1:%d" % port, rank=rank,
+                            world_size=world)
+    seen = {}
+
+    def share(G, x, idx, weights, r, w, workspace=None):
+        seen["rank"], seen["world"] = r, w
+        return torch.full((8,), float(r + 1), dtype=torch.float32)
+
+    qmoe.moe_expert_qmlp_ep = share
+    qmoe.f32_to_f16 = lambda t: t.half()
+    y = qmoe.moe_layer_ep(None, None, None, None)
+    dist.barrier()
+    dist.destroy_process_group()
+    with open(os.path.join(out_dir, "p%d.json" % rank), "w") as f:
+        json.dump({"y": y.float().tolist(), "dtype": str(y.dtype), **seen}, f)
+
+
+def test_moe_layer_ep_plumbing(tmp_path):
+    import torch.multiprocessing as mp
+    world, port = 2, free_port()
+    ctx = mp.get_context("spawn")
+    procs = [ctx.Process(target=_plumbing_main, args=(r, world, port, str(tmp_path)))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+    codes = [p.exitcode for p in procs]
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert codes == [0, 0], codes
+    for r in range(world):
+        d = json.load(open(tmp_path / ("p%d.json" % r)))
+        assert d["rank"] == r and d["world"] == world
+        assert d["dtype"] == "torch.float16"
+        assert d["y"] == [3.0] * 8          # 1 + 2 summed over the two ranks
