@@ -61,3 +61,28 @@ def test_one_pass_workspace_sizes_without_gpu():
     assert f(1000, 4096, 8, 9) == 65536 + tiles * 2 * (1 * 2 * 32) * 16
     # K=8192 at batch 32: 8 slices of 1024
     assert f(256, 8192, 4, 32) == 65536 + (256 // 64) * 8 * (4 * 4 * 32) * 16
+
+
+def test_decode_pack_holds_exactly_the_row_major_bytes_without_gpu():
+    """moe_decode_pack_bytes is host arithmetic: the streaming layout is a
+    permutation of the row-major layer (8-bit router + E routed experts + the
+    shared expert, codes and fp16 scale + bias per 64 inputs), nothing added."""
+    from moe_expert_gemv_b200 import qmoe
+    lib = ctypes.CDLL(build.build())
+    f = lib.moe_decode_pack_bytes
+    f.restype = ctypes.c_size_t
+    f.argtypes = [ctypes.c_void_p]
+
+    def mat_bytes(rows, cols, bits):
+        return rows * cols * bits // 8 + 2 * rows * (cols // 64) * 2
+
+    for E, H, I in ((128, 2816, 704), (16, 256, 64), (64, 1024, 192)):
+        L = qmoe.CMoeLayer()
+        L.num_experts, L.hidden, L.inter = E, H, I
+        want = mat_bytes(E, H, 8) + (E + 1) * (2 * mat_bytes(I, H, 4) + mat_bytes(H, I, 4))
+        assert f(ctypes.addressof(L)) == want
+    # the numbers the benchmark quotes: 30 layers of the 128-expert layer
+    L = qmoe.CMoeLayer()
+    L.num_experts, L.hidden, L.inter = 128, 2816, 704
+    assert f(ctypes.addressof(L)) == 382976 + 129 * 3345408
+    assert 30 * f(ctypes.addressof(L)) == 12958218240   # "12.96 GB of weights"
