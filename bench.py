@@ -14,7 +14,14 @@ the weight-stream GB/s of the dominant kernel against the measured HBM peak
 CPU oracle timed on a bounded sample (`cpu_baseline`).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload moe_decode|qgemv|router|prefill]
+                  [--workload moe_decode|qgemv|qgemv_fmt|router|prefill|
+                              expert_cache|expert_parallel]
+                  [--layers L] [--qgemv-batch 1,4,8,16,32]
+
+The other workloads print one JSON line of per-kernel numbers each: dense
+qGEMV at batch 1..32 (one pass over the weights from batch 9 on), the
+bf16-scale formats, the router, the 128-token prefill chunk, expert streaming
+from host memory, and one rank's share of an expert-parallel layer.
 
 Under torchrun every rank runs an independent replica (weak scaling); the
 timed region is bracketed by a barrier and device synchronisation, and the
