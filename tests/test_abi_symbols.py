@@ -86,3 +86,27 @@ def test_decode_pack_holds_exactly_the_row_major_bytes_without_gpu():
     L.num_experts, L.hidden, L.inter = 128, 2816, 704
     assert f(ctypes.addressof(L)) == 382976 + 129 * 3345408
     assert 30 * f(ctypes.addressof(L)) == 12958218240   # "12.96 GB of weights"
+
+
+def test_header_is_plain_c_and_links_from_c(tmp_path):
+    """include/qmoe.h is a C header (strict C11, no C++ constructs), and a C
+    program links against the library and calls it (no GPU call)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        import pytest
+        pytest.skip("no C compiler")
+    lib = build.build()
+    src = tmp_path / "use.c"
+    src.write_text('#include "qmoe.h"\n#include <string.h>\n'
+                   'int main(void) {\n'
+                   '  if (qmoe_version() <= 0) return 1;\n'
+                   '  if (strncmp(qmoe_status_string(QMOE_OK), "QMOE_", 5)) return 2;\n'
+                   '  if (qgemv_affine_workspace_bytes(14336, 4096, 4, 8) != 0) return 3;\n'
+                   '  return 0;\n}\n')
+    exe = tmp_path / "use"
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                    os.path.join(ROOT, "include"), str(src), "-L", os.path.dirname(lib), "-lqmoe",
+                    "-Wl,-rpath," + os.path.dirname(lib), "-o", str(exe)], check=True)
+    assert subprocess.run([str(exe)]).returncode == 0
