@@ -357,12 +357,16 @@ qmoe_status moe_decode_layers(const void *const *packed_layers, int32_t n_layers
  * moe_cache_layer: one decode token through the layer:
  *   router (resident, device) -> the host reads the top_k ids (this call
  *   SYNCHRONISES `stream` once; every other entry point never does) -> plan
- *   -> each missed expert's nine arrays host -> device on `copy_stream`
- *   (NULL: `stream`) -> the routed experts wait for the copies -> y =
+ *   -> each missed expert's nine arrays host -> device, the misses spread
+ *   over four copy streams (the first is `copy_stream` when given, the
+ *   others the cache's own) -> the routed experts wait for the copies -> y =
  *   shared(x) + sum_j weights[j] * expert_{idx[j]}(x) from the slots (as
  *   moe_expert_qmlp; same zero-filled workspace).  idx_out / weights_out
  *   (device, optional) receive the router's choice.  Returns
- *   QMOE_ERR_DEVICE_STATUS if the router produced an id outside [0, E).
+ *   QMOE_ERR_DEVICE_STATUS if the router produced an id outside [0, E)
+ *   (the cache unchanged).  If a copy or launch fails after the plan, the
+ *   cache forgets every slot (all empty) so that no later token trusts a
+ *   slot whose copy may not have landed.
  * qmoe_cache_stats: cumulative hits, misses, bytes copied; the expert held by
  * each slot (-1: empty).
  * ------------------------------------------------------------------------- */

@@ -308,6 +308,13 @@ qmoe_status moe_cache_layer(qmoe_expert_cache *c, const qmoe_qmatrix *router, co
     const int nm = lfu_plan(&c->plan.c, ids, top_k, c->slot_host, miss_e, miss_s);
     if (nm < 0)
         return QMOE_ERR_INVALID_ARG;
+    // From here the plan already names the new slot contents: if any step
+    // fails, forget the whole cache (every slot empty) rather than keep a plan
+    // whose copies may not have landed; the next token copies again.
+    auto fail = [&](qmoe_status st_) {
+        lfu_reset(&c->plan.c, c->plan.c.nslots);
+        return st_;
+    };
     // 4. the missed experts' arrays, host -> device, one copy each; expert m
     //    on copy stream m % kCopyStreams.  A slot must not be overwritten
     //    while an earlier token's experts read it: the synchronisation above
@@ -316,10 +323,10 @@ qmoe_status moe_cache_layer(qmoe_expert_cache *c, const qmoe_qmatrix *router, co
     const int nstreams = nm < kCopyStreams ? nm : kCopyStreams;
     if (nstreams > 0) {
         if (cudaEventRecord(ev[0], st) != cudaSuccess)
-            return QMOE_ERR_CUDA;
+            return fail(QMOE_ERR_CUDA);
         for (int i = 0; i < nstreams; ++i)
             if (cudaStreamWaitEvent(cs[i], ev[0], 0) != cudaSuccess)
-                return QMOE_ERR_CUDA;
+                return fail(QMOE_ERR_CUDA);
     }
     for (int m = 0; m < nm; ++m) {
         ArrayPart parts[9];
@@ -327,7 +334,7 @@ qmoe_status moe_cache_layer(qmoe_expert_cache *c, const qmoe_qmatrix *router, co
         for (int i = 0; i < np; ++i) {
             if (cudaMemcpyAsync(parts[i].dst, parts[i].src, parts[i].bytes,
                                 cudaMemcpyHostToDevice, cs[m % kCopyStreams]) != cudaSuccess)
-                return QMOE_ERR_CUDA;
+                return fail(QMOE_ERR_CUDA);
             c->bytes += (int64_t)parts[i].bytes;
         }
     }
@@ -337,15 +344,15 @@ qmoe_status moe_cache_layer(qmoe_expert_cache *c, const qmoe_qmatrix *router, co
     for (int i = 0; i < nstreams; ++i)
         if (cudaEventRecord(ev[i], cs[i]) != cudaSuccess ||
             cudaStreamWaitEvent(st, ev[i], 0) != cudaSuccess)
-            return QMOE_ERR_CUDA;
+            return fail(QMOE_ERR_CUDA);
     if (cudaMemcpyAsync(c->slot_dev, c->slot_host, top_k * sizeof(int32_t),
                         cudaMemcpyHostToDevice, st) != cudaSuccess)
-        return QMOE_ERR_CUDA;
+        return fail(QMOE_ERR_CUDA);
     // 6. shared + routed experts from the slots
     s = moe_expert_qmlp(&c->slots, x, c->slot_dev, c->wt_dev, top_k, y, workspace,
                         workspace_bytes, status_dev, stream);
     if (s != QMOE_OK)
-        return s;
+        return fail(s);
     if (idx_out && cudaMemcpyAsync(idx_out, c->idx_dev, top_k * sizeof(int32_t),
                                    cudaMemcpyDeviceToDevice, st) != cudaSuccess)
         return QMOE_ERR_CUDA;
