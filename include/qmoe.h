@@ -261,11 +261,16 @@ qmoe_status qmoe_f32_to_f16(const float *src, uint16_t *dst, int64_t n, void *st
  * the library: a 1 MiB __device__ array that every GPU loading the library
  * holds until the process exits.  Requests whose workspace
  * (moe_expert_workspace_bytes) exceeds 1 MiB return QMOE_ERR_WORKSPACE.
- * It allocates and frees nothing.  The first call on each device looks up the
- * array's device address (with that device current); make that first call
- * before any stream capture.  Each call clears the buffer's counters on
- * `stream` before its kernels run.  Every call shares the one buffer, so
- * calls that overlap on the GPU (for instance on two streams) race. */
+ * It allocates and frees nothing.  Every call looks up the array's device
+ * address in the current device's context (nothing is cached, so a new
+ * context after a device reset is picked up); `stream` must belong to the
+ * current device.  The first call on a device also loads the array's module
+ * there, so make that first call before any stream capture.  A call checks
+ * all of its arguments before it enqueues anything: a rejected call leaves
+ * the stream and the buffer untouched.  An accepted call clears the buffer's
+ * counters on `stream` before its kernels run.  Every call shares the one
+ * buffer, so calls that overlap on the GPU (for instance on two streams)
+ * race. */
 qmoe_status moe_expert_qmlp_noalloc(const qmoe_moe_layer *L, const uint16_t *x,
                                     const int32_t *idx, const float *weights, int32_t top_k,
                                     uint16_t *y, int32_t *status_dev, void *stream);

@@ -162,6 +162,26 @@ qmoe_status check_expert_common(const qmoe_moe_layer *L, int32_t top_k)
 }
 
 }  // namespace
+
+// Every check moe_expert_qmlp makes before it enqueues anything: the layer's
+// shapes and formats, top_k, the pointers and their alignment, and that the
+// current device is one the library was built for.
+qmoe_status validate_expert_qmlp(const qmoe_moe_layer *L, const uint16_t *x, const int32_t *idx,
+                                 const float *weights, int32_t top_k, const uint16_t *y,
+                                 const int32_t *status_dev)
+{
+    qmoe_status s = check_expert_common(L, top_k);
+    if (s != QMOE_OK)
+        return s;
+    if (!x || !idx || !weights || !y)
+        return QMOE_ERR_INVALID_ARG;
+    if (!aligned(x, 2) || !aligned(idx, 4) || !aligned(weights, 4) || !aligned(y, 2) ||
+        (status_dev && !aligned(status_dev, 4)))
+        return QMOE_ERR_ALIGNMENT;
+    DevState *d;
+    return device_state(&d);
+}
+
 }  // namespace qmoe
 
 using namespace qmoe;
@@ -376,14 +396,9 @@ qmoe_status moe_expert_qmlp(const qmoe_moe_layer *L, const uint16_t *x, const in
                             const float *weights, int32_t top_k, uint16_t *y, void *workspace,
                             size_t workspace_bytes, int32_t *status_dev, void *stream)
 {
-    qmoe_status s = check_expert_common(L, top_k);
+    qmoe_status s = qmoe::validate_expert_qmlp(L, x, idx, weights, top_k, y, status_dev);
     if (s != QMOE_OK)
         return s;
-    if (!x || !idx || !weights || !y)
-        return QMOE_ERR_INVALID_ARG;
-    if (!aligned(x, 2) || !aligned(idx, 4) || !aligned(weights, 4) || !aligned(y, 2) ||
-        (status_dev && !aligned(status_dev, 4)))
-        return QMOE_ERR_ALIGNMENT;
     DevState *d;
     if ((s = device_state(&d)) != QMOE_OK)
         return s;

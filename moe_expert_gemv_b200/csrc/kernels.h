@@ -92,6 +92,11 @@ struct ExpertWorkspace {
     int32_t *counters; // [hidden / 16]
 };
 size_t expert_workspace_layout(int hidden, int inter, int top_k, void *base, ExpertWorkspace *ws);
+// The argument checks of moe_expert_qmlp (shapes, formats, top_k, pointers,
+// alignment, device), run before anything is enqueued.
+qmoe_status validate_expert_qmlp(const qmoe_moe_layer *L, const uint16_t *x, const int32_t *idx,
+                                 const float *weights, int32_t top_k, const uint16_t *y,
+                                 const int32_t *status_dev);
 
 struct ExpertArgs {
     QMat gate, up, down, sh_gate, sh_up, sh_down;

@@ -9,13 +9,15 @@
 // library holds until the process exits.
 //
 // The kernels see the buffer through its device address, which host code
-// obtains with cudaGetSymbolAddress once per device (the array's name in host
-// code is only a host-side stand-in).  Only the arrival counters must start at
-// zero; they are cleared on the stream before each call.  All calls share the
-// one buffer, so calls that overlap on the GPU (two streams, or two devices'
-// worth of work issued to the same device at once) race and must be avoided.
-#include <mutex>
-
+// obtains with cudaGetSymbolAddress (the array's name in host code is only a
+// host-side stand-in).  The address is looked up on every call, with the
+// device that is current at the call, so a new context (after a device reset)
+// or another current device gets its own address; nothing is cached.  Only
+// the arrival counters must start at zero; every call checks all of its
+// arguments first and only then clears them on the stream.  All calls share
+// the one buffer, so calls that overlap on the GPU (two streams, or two
+// devices' worth of work issued to the same device at once) race and must be
+// avoided.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,25 +30,13 @@ constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDev = 64;
-std::mutex g_noalloc_mu;
-void *g_noalloc_ptr[kMaxDev];
-
-// Device address of the scratch array on the current device (set up on the
-// first call made with that device current).
+// Device address of the scratch array in the current device's context.
 qmoe_status noalloc_scratch(void **out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
         return QMOE_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
-            return QMOE_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
-    }
-    *out = g_noalloc_ptr[dev];
+    *out = p;
     return QMOE_OK;
 }
 
@@ -60,16 +50,18 @@ extern "C" qmoe_status moe_expert_qmlp_noalloc(const qmoe_moe_layer *L, const ui
                                                int32_t top_k, uint16_t *y, int32_t *status_dev,
                                                void *stream)
 {
-    if (!L || !x || !idx || !weights || !y || top_k < 1 || top_k > 16)
-        return QMOE_ERR_INVALID_ARG;
+    // every argument check first: a rejected call enqueues nothing on the
+    // stream, so it cannot clear the counters of a call still in flight
+    qmoe_status s = validate_expert_qmlp(L, x, idx, weights, top_k, y, status_dev);
+    if (s != QMOE_OK)
+        return s;
     const size_t need = moe_expert_workspace_bytes(L, top_k);
     if (need == 0)
         return QMOE_ERR_INVALID_ARG;
     if (need > kNoAllocScratchBytes)
         return QMOE_ERR_WORKSPACE;   // beyond the built-in scratch: use moe_expert_qmlp
     void *scratch = nullptr;
-    qmoe_status s = noalloc_scratch(&scratch);
-    if (s != QMOE_OK)
+    if ((s = noalloc_scratch(&scratch)) != QMOE_OK)
         return s;
     ExpertWorkspace ws;
     expert_workspace_layout(L->hidden, L->inter, top_k, scratch, &ws);

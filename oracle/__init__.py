@@ -276,6 +276,6 @@ class LfuCache:
         nm = lib().or_lfu_step(self.nslots, _ptr(self.expert), _ptr(self.count), _ptr(ids), k,
                                _ptr(slot_of), _ptr(me), _ptr(ms))
         if nm < 0:
-            raise ValueError("k > nslots or repeated ids")
+            raise ValueError("k > nslots, nslots outside 1..256, or repeated ids")
         return slot_of, list(zip(me[:nm].tolist(), ms[:nm].tolist()))
 

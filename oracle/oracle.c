@@ -357,7 +357,7 @@ int or_qgemv_fmt(const uint32_t *P, const uint32_t *params, int64_t N, int64_t K
    logits (ties -> lower index first) in descending order, then the selected
    probabilities divided by their sum.  Selection is on the logits; softmax
    is monotone so this is the same set as selecting on probabilities. */
-static void select_topk(const double *l, int64_t E, int64_t k, int32_t *idx, double *wt)
+static int select_topk(const double *l, int64_t E, int64_t k, int32_t *idx, double *wt)
 {
     double m = -INFINITY;
     for (int64_t e = 0; e < E; ++e)
@@ -369,6 +369,11 @@ static void select_topk(const double *l, int64_t E, int64_t k, int32_t *idx, dou
     unsigned char *taken = (unsigned char *)calloc((size_t)E, 1);
     double psum = 0.0;
     double *p = (double *)malloc(sizeof(double) * (size_t)k);
+    if (!taken || !p) {
+        free(taken);
+        free(p);
+        return -2;
+    }
     for (int64_t j = 0; j < k; ++j) {
         int64_t best = -1;
         for (int64_t e = 0; e < E; ++e) {
@@ -386,6 +391,7 @@ static void select_topk(const double *l, int64_t E, int64_t k, int32_t *idx, dou
         wt[j] = p[j] / psum;
     free(p);
     free(taken);
+    return 0;
 }
 
 /* Full router on T tokens: 8-bit (or 4-bit) affine router matrix [E][K].
@@ -403,10 +409,11 @@ int or_router(const uint32_t *P, const uint16_t *S, const uint16_t *Bi,
     for (int64_t i = 0; i < T * K; ++i)
         x[i] = or_f16_to_f64(x16[i]);
     qmatvec_f64(P, S, Bi, E, K, bits, x, T, logits64);
-    for (int64_t t = 0; t < T; ++t)
-        select_topk(logits64 + t * E, E, k, idx + t * k, wt + t * k);
+    int rc = 0;
+    for (int64_t t = 0; t < T && rc == 0; ++t)
+        rc = select_topk(logits64 + t * E, E, k, idx + t * k, wt + t * k);
     free(x);
-    return 0;
+    return rc;
 }
 
 /* The same selection applied to given fp32 logits (e.g. a device's own). */
@@ -416,13 +423,16 @@ int or_topk_from_logits(const float *logits32, int64_t T, int64_t E, int64_t k,
     if (k < 1 || k > E)
         return -1;
     double *l = (double *)malloc(sizeof(double) * (size_t)E);
-    for (int64_t t = 0; t < T; ++t) {
+    if (!l)
+        return -2;
+    int rc = 0;
+    for (int64_t t = 0; t < T && rc == 0; ++t) {
         for (int64_t e = 0; e < E; ++e)
             l[e] = (double)logits32[t * E + e];
-        select_topk(l, E, k, idx + t * k, wt + t * k);
+        rc = select_topk(l, E, k, idx + t * k, wt + t * k);
     }
     free(l);
-    return 0;
+    return rc;
 }
 
 /* ------------------------------------------------------------------------ */
@@ -446,9 +456,9 @@ static double silu(double z) { return z / (1.0 + exp(-z)); }
 
 /* One SwiGLU expert on one token: r = down (silu(gate x) * (up x)).
    gate/up are [I][H], down is [H][I]; x has H fp64 entries; r has H. */
-static void expert_mlp(const or_mat *gate, const or_mat *up, const or_mat *down,
-                       int64_t e, int64_t H, int64_t I, int bits,
-                       const double *x, double *r)
+static int expert_mlp(const or_mat *gate, const or_mat *up, const or_mat *down,
+                      int64_t e, int64_t H, int64_t I, int bits,
+                      const double *x, double *r)
 {
     int64_t per = 32 / bits;
     const uint32_t *Pg = gate->packed + e * I * (H / per);
@@ -463,6 +473,12 @@ static void expert_mlp(const or_mat *gate, const or_mat *up, const or_mat *down,
     double *g = (double *)malloc(sizeof(double) * (size_t)I);
     double *u = (double *)malloc(sizeof(double) * (size_t)I);
     double *h = (double *)malloc(sizeof(double) * (size_t)I);
+    if (!g || !u || !h) {
+        free(g);
+        free(u);
+        free(h);
+        return -2;
+    }
     qmatvec_f64(Pg, Sg, Bg, I, H, bits, x, 1, g);
     qmatvec_f64(Pu, Su, Bu, I, H, bits, x, 1, u);
     for (int64_t i = 0; i < I; ++i)
@@ -471,6 +487,7 @@ static void expert_mlp(const or_mat *gate, const or_mat *up, const or_mat *down,
     free(g);
     free(u);
     free(h);
+    return 0;
 }
 
 /* Routed expert e of the layer on one fp16 token (exposed for composition
@@ -480,14 +497,17 @@ int or_expert(const or_layer *L, int64_t e, const uint16_t *x16, double *r)
     if (L->H % 64 || L->I % 64 || e >= L->E)
         return -1;
     double *x = (double *)malloc(sizeof(double) * (size_t)L->H);
+    if (!x)
+        return -2;
     for (int64_t i = 0; i < L->H; ++i)
         x[i] = or_f16_to_f64(x16[i]);
+    int rc;
     if (e < 0)
-        expert_mlp(&L->sh_gate, &L->sh_up, &L->sh_down, 0, L->H, L->I, (int)L->bits, x, r);
+        rc = expert_mlp(&L->sh_gate, &L->sh_up, &L->sh_down, 0, L->H, L->I, (int)L->bits, x, r);
     else
-        expert_mlp(&L->gate, &L->up, &L->down, e, L->H, L->I, (int)L->bits, x, r);
+        rc = expert_mlp(&L->gate, &L->up, &L->down, e, L->H, L->I, (int)L->bits, x, r);
     free(x);
-    return 0;
+    return rc;
 }
 
 /* MoE layer on T tokens with given routing: y[t] = shared(x_t) +
@@ -506,16 +526,18 @@ int or_moe_layer(const or_layer *L, const uint16_t *x16, int64_t T,
     double *x = (double *)malloc(sizeof(double) * (size_t)H);
     double *r = (double *)malloc(sizeof(double) * (size_t)H);
     double *y = (double *)malloc(sizeof(double) * (size_t)H);
-    for (int64_t t = 0; t < T; ++t) {
+    int rc = (x && r && y) ? 0 : -2;
+    for (int64_t t = 0; t < T && rc == 0; ++t) {
         for (int64_t i = 0; i < H; ++i)
             x[i] = or_f16_to_f64(x16[t * H + i]);
-        expert_mlp(&L->sh_gate, &L->sh_up, &L->sh_down, 0, H, L->I, (int)L->bits, x, y);
-        for (int64_t j = 0; j < k; ++j) {
-            expert_mlp(&L->gate, &L->up, &L->down, idx[t * k + j], H, L->I, (int)L->bits, x, r);
-            for (int64_t i = 0; i < H; ++i)
+        rc = expert_mlp(&L->sh_gate, &L->sh_up, &L->sh_down, 0, H, L->I, (int)L->bits, x, y);
+        for (int64_t j = 0; j < k && rc == 0; ++j) {
+            rc = expert_mlp(&L->gate, &L->up, &L->down, idx[t * k + j], H, L->I, (int)L->bits,
+                            x, r);
+            for (int64_t i = 0; i < H && rc == 0; ++i)
                 y[i] += wt[t * k + j] * r[i];
         }
-        for (int64_t i = 0; i < H; ++i) {
+        for (int64_t i = 0; i < H && rc == 0; ++i) {
             if (y64)
                 y64[t * H + i] = y[i];
             if (y16)
@@ -525,7 +547,7 @@ int or_moe_layer(const or_layer *L, const uint16_t *x16, int64_t T,
     free(x);
     free(r);
     free(y);
-    return 0;
+    return rc;
 }
 
 /* ------------------------------------------------------------------------ */
@@ -549,6 +571,8 @@ int or_group(const int32_t *idx, int64_t T, int64_t k, int64_t E,
     for (int64_t e = 0; e < E; ++e)
         offsets[e + 1] = offsets[e] + counts[e];
     int32_t *fill = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    if (!fill)
+        return -2;
     for (int64_t e = 0; e < E; ++e)
         fill[e] = offsets[e];
     for (int64_t i = 0; i < T * k; ++i)
@@ -573,13 +597,13 @@ int or_group(const int32_t *idx, int64_t T, int64_t k, int64_t E,
        slot, else into the unpinned slot with the smallest count, ties to the
        lowest index (slots holding an expert of this token are pinned).
    One step: slot_of[j] = slot of ids[j]; misses listed in order as
-   (expert, slot) pairs; returns the number of misses, or -1 if k > nslots
-   or the ids repeat. */
+   (expert, slot) pairs; returns the number of misses, or -1 if k > nslots,
+   nslots is outside 1..256, or the ids repeat. */
 int64_t or_lfu_step(int64_t nslots, int32_t *slot_expert, int64_t *slot_count,
                     const int32_t *ids, int64_t k, int32_t *slot_of, int32_t *miss_expert,
                     int32_t *miss_slot)
 {
-    if (k > nslots)
+    if (k > nslots || nslots < 1 || nslots > 256)   /* the pinned flags hold 256 slots */
         return -1;
     for (int64_t a = 0; a < k; ++a)
         for (int64_t b = a + 1; b < k; ++b)

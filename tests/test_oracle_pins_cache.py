@@ -61,3 +61,15 @@ def test_rejects_repeats_and_overflow():
         c.step([1, 1])
     with pytest.raises(ValueError):
         c.step([1, 2, 3, 4, 5])
+
+
+def test_lfu_rejects_slot_counts_beyond_its_flags():
+    """The plan keeps one pinned flag per slot for at most 256 slots; more
+    slots (or none) are refused instead of overrunning the flags."""
+    for n in (0, 257, 1000):
+        c = oracle.LfuCache(nslots=max(n, 1))
+        c.nslots = n
+        c.expert = np.full(max(n, 1), -1, np.int32)
+        c.count = np.zeros(max(n, 1), np.int64)
+        with pytest.raises(ValueError):
+            c.step([1])
