@@ -22,6 +22,17 @@ import numpy as np
 from .build import build as _build
 
 _lib = None
+_libs = {}
+_threads = False
+
+
+def use_threads(on=True):
+    """Route later oracle calls to the OpenMP build of the same source (its
+    output rows split over threads, bit-identical results); only the
+    multi-threaded CPU baseline uses it."""
+    global _threads, _lib
+    _threads = bool(on)
+    _lib = None
 
 
 class OrMat(ctypes.Structure):
@@ -38,8 +49,10 @@ class OrLayer(ctypes.Structure):
 
 def lib():
     global _lib
+    if _lib is None and _threads in _libs:
+        _lib = _libs[_threads]
     if _lib is None:
-        L = ctypes.CDLL(_build())
+        L = ctypes.CDLL(_build(threads=_threads))
         p = ctypes.c_void_p
         i64 = ctypes.c_int64
         L.or_f16_to_f64.argtypes = [ctypes.c_uint16]
@@ -65,7 +78,7 @@ def lib():
         for name in ("or_unpack", "or_pack", "or_dequant", "or_qgemv", "or_router",
                      "or_topk_from_logits", "or_expert", "or_moe_layer", "or_group"):
             getattr(L, name).restype = ctypes.c_int
-        _lib = L
+        _lib = _libs[_threads] = L
     return _lib
 
 

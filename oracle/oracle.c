@@ -179,6 +179,10 @@ static void qmatvec_f64(const uint32_t *P, const uint16_t *S, const uint16_t *Bi
     int64_t G = K / 64;
     uint32_t mask = (1u << bits) - 1u;
     for (int64_t b = 0; b < B; ++b)
+        /* rows are independent: the threaded build (-fopenmp) splits them over
+           threads; each row's sum keeps the index order, so the result is the
+           same bit for bit */
+#pragma omp parallel for schedule(static)
         for (int64_t n = 0; n < N; ++n) {
             const uint32_t *row = P + n * (K / per);
             double acc = 0.0;

@@ -357,3 +357,28 @@ def test_zipf_routing_shape():
     assert np.all(np.diff(wt, axis=1) <= 0)
     c = np.bincount(idx.ravel(), minlength=128)
     assert c.max() > 64 and (c <= 8).sum() > 64
+
+
+def test_threaded_build_is_bit_identical():
+    """The OpenMP build of the oracle (output rows split over threads, used
+    only for the multi-threaded CPU baseline) computes every output bit for
+    bit like the plain build: each row's sum keeps the index order."""
+    from moe_expert_gemv_b200 import synth
+    E, H, I = 16, 256, 128
+    m = synth.moe_layer(3, 0, E=E, H=H, I=I)
+    x16 = synth.activations(3, 5, H)
+    P, S, B = synth.dense(3, 96, 512)
+    xd = synth.activations(4, 3, 512)
+    L = oracle.Layer(m, E, H, I)
+    outs = []
+    try:
+        for threads in (False, True):
+            oracle.use_threads(threads)
+            lg, idx, wt = oracle.router(*m["router"], E, H, 8, x16, 4)
+            y, _ = L.moe(x16, idx, wt)
+            q, _ = oracle.qgemv(P, S, B, 96, 512, 4, xd)
+            outs.append((lg, idx, wt, y, q))
+    finally:
+        oracle.use_threads(False)
+    for a, b in zip(*outs):
+        assert np.array_equal(a, b)
