@@ -211,6 +211,46 @@ def timed_replays(fn, iters, dist=None):
 
 
 # ---------------------------------------------------- CPU oracle baseline --
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline_line(seconds, seed, m):
+    """The oracle on bounded samples of decode layers: the threaded build on
+    every host thread (the reported value) and the plain single-threaded
+    build beside it."""
+    import oracle
+    half = seconds / 2.0
+    d1, e1 = oracle_decode_layers(half, seed, m=m)
+    nt = host_threads()
+    oracle.use_threads(True)
+    try:
+        dn, en = oracle_decode_layers(half, seed, m=m)
+    finally:
+        oracle.use_threads(False)
+    return {"value": round(dn / en, 3), "unit": "layers/s", "cores": nt, "kind": "oracle",
+            "sample": "%d decode layers (router + shared + 8 routed experts) of layer 0's "
+                      "weights, fresh seeded tokens, %.1f s, OpenMP over output rows on %d "
+                      "threads" % (dn, en, nt),
+            "cpu_model": cpu_model(),
+            "single_thread": {"value": round(d1 / e1, 3), "unit": "layers/s", "cores": 1,
+                              "sample": "%d layers, %.1f s" % (d1, e1)}}
+
+
 def oracle_decode_layers(seconds, seed, max_layers=None, m=None):
     """Run the CPU oracle on decode layers (router + shared + 8 routed experts)
     of one layer's weights with fresh seeded tokens until `seconds` elapse.
@@ -383,12 +423,7 @@ def main_decode(args):
     if r["clk"]:
         line["clocks"] = r["clk"]
     if N == 1 and not args.no_cpu_baseline:
-        done, el = oracle_decode_layers(args.cpu_seconds, args.seed, m=r["m0"])
-        line["cpu_baseline"] = {"value": round(done / el, 3), "unit": "layers/s", "cores": 1,
-                                "kind": "oracle",
-                                "sample": "%d decode layers (router + shared + 8 routed experts) "
-                                          "of layer 0's weights, fresh seeded tokens, %.1f s, "
-                                          "single thread" % (done, el)}
+        line["cpu_baseline"] = cpu_baseline_line(args.cpu_seconds, args.seed, r["m0"])
     print(json.dumps(line), flush=True)
     dist.close()
 
@@ -402,10 +437,14 @@ def main_reference(args):
     per_layer = 0.25
     steps = max(3, min(args.steps, int(budget / per_layer)))
     warm = min(args.warmup, 2)
+    import oracle
     from moe_expert_gemv_b200 import synth
     m = synth.moe_layer(args.seed, 0)
+    nt = host_threads()
+    oracle.use_threads(True)   # the oracle's OpenMP build on every host thread
     oracle_decode_layers(0.0, args.seed, max_layers=max(1, warm), m=m)
     done, el = oracle_decode_layers(1e9, args.seed, max_layers=steps, m=m)
+    oracle.use_threads(False)
     value = done / el
     line = {
         "impl": "reference",
@@ -416,11 +455,11 @@ def main_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": dict(decode_config(args.layers, 1),
                        path="CPU oracle (fp64), one layer of the stack per step"),
-        "cpu_baseline": {"value": round(value, 3), "unit": "layers/s", "cores": 1,
-                         "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 3), "unit": "layers/s", "cores": nt,
+                         "kind": "oracle", "cpu_model": cpu_model(),
                          "sample": "%d decode layers (router + shared + 8 routed experts) "
-                                   "of layer 0's weights, fresh seeded tokens, single thread"
-                                   % done},
+                                   "of layer 0's weights, fresh seeded tokens, OpenMP over "
+                                   "output rows on %d threads" % (done, nt)},
         "e2e": {"value": round(value, 3), "unit": "layers/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -583,38 +622,53 @@ def main_other(args):
             out["results"].append({"T": T, "us": round(ms * 1e3, 3),
                                    "tokens_per_s": round(T / (ms / 1e3), 1)})
     elif args.workload == "prefill":
-        # 128-token chunk, Zipf(1.1) routing, rotating over 4 layers (1.7 GB of
-        # weights) so consecutive calls do not find their experts in L2
+        # 128-token chunk through one 128-expert layer, rotating over 4 layers
+        # (1.7 GB of weights) so consecutive calls do not find their experts in
+        # L2.  Routings: the pages' Zipf(1.1) draw, and a dense one (every token
+        # to experts 0..7: nine 128-token slots, the tensor-bound case).  Paths:
+        # streaming kernels only, and experts with >= 16 tokens on tcgen05.
         nl = 4
         Gs = [qmoe.MoELayer.from_numpy(synth.moe_layer(args.seed, l), E, H, I, dev)
               for l in range(nl)]
-        idx_np, wt_np = synth.zipf_routing(args.seed)
-        T = idx_np.shape[0]
+        idx_z, wt_z = synth.zipf_routing(args.seed)
+        T = idx_z.shape[0]
+        idx_d = np.tile(np.arange(TOPK, dtype=np.int32), (T, 1))
         x = torch.from_numpy(synth.activations(args.seed, T, H).view(np.float16).copy()).to(dev)
-        idx = torch.from_numpy(idx_np).to(dev)
-        wt = torch.from_numpy(wt_np).to(dev)
         y = torch.empty(T, H, dtype=torch.float16, device=dev)
         ws = torch.empty(qmoe.moe_prefill_workspace_bytes(Gs[0], T, TOPK), dtype=torch.uint8,
                          device=dev)
-
-        def run():
-            for G in Gs:
-                qmoe.moe_prefill_qgemm(G, x, idx, wt, y, ws)
-        run()
-        torch.cuda.synchronize()
-        assert qmoe.qmoe_check_status() == 0
-        for _ in range(3):
-            run()
-        reps = max(5, args.steps // 50)
-        ms = timed_replays(run, reps) / (reps * nl)
-        touched = int(np.unique(idx_np).size)
-        nbytes = (touched + 1) * EXPERT_BYTES
         flops = 2.0 * (T * TOPK + T) * 3 * I * H
-        gbs = nbytes / (ms / 1e3) / 1e9
-        out["results"].append({"T": T, "experts_touched": touched, "us": round(ms * 1e3, 2),
-                               "tokens_per_s": round(T / (ms / 1e3), 1),
-                               "weight_GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
-                               "useful_TFLOP/s": round(flops / (ms / 1e3) / 1e12, 2)})
+        old_min = qmoe.qmoe_set_prefill_tensor_min(0)
+        try:
+            for routing, idx_np in (("zipf1.1", idx_z), ("dense_experts_0_7", idx_d)):
+                idx = torch.from_numpy(idx_np).to(dev)
+                wt = torch.from_numpy(wt_z).to(dev)
+                for tmin in (0, qmoe.TENSOR_MIN_DEFAULT):
+                    qmoe.qmoe_set_prefill_tensor_min(tmin)
+
+                    def run():
+                        for G in Gs:
+                            qmoe.moe_prefill_qgemm(G, x, idx, wt, y, ws)
+                    run()
+                    torch.cuda.synchronize()
+                    assert qmoe.qmoe_check_status() == 0
+                    for _ in range(3):
+                        run()
+                    reps = max(5, args.steps // 50)
+                    ms = timed_replays(run, reps) / (reps * nl)
+                    counts = np.bincount(idx_np.ravel(), minlength=E)
+                    touched = int((counts > 0).sum())
+                    heavy = int((counts >= tmin).sum() + (T >= tmin)) if tmin else 0
+                    nbytes = (touched + 1) * EXPERT_BYTES
+                    gbs = nbytes / (ms / 1e3) / 1e9
+                    out["results"].append({
+                        "T": T, "routing": routing, "tensor_min_tokens": tmin,
+                        "tensor_core_slots": heavy, "experts_touched": touched,
+                        "us": round(ms * 1e3, 2), "tokens_per_s": round(T / (ms / 1e3), 1),
+                        "weight_GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                        "useful_TFLOP/s": round(flops / (ms / 1e3) / 1e12, 2)})
+        finally:
+            qmoe.qmoe_set_prefill_tensor_min(old_min)
     else:
         out["error"] = "workload not available"
     print(json.dumps(out), flush=True)

@@ -187,6 +187,19 @@ typedef struct qmoe_qmatrix_fmt {
 qmoe_status qgemv_fmt(const qmoe_qmatrix_fmt *W, const uint16_t *x, int32_t batch, uint16_t *y,
                       int32_t *status_dev, void *stream);
 
+/* The format variants for batch 9..32 in ONE pass over the weights, with the
+ * same workspace contract as qgemv_affine_workspace_bytes / qgemv_affine_ws
+ * (uzu page, "uzu의 추측 디코딩 구조": the 16-32 draft tokens of a
+ * verification step multiply every projection at once).  rotated != 0: the
+ * call will pass rht_signs (the rotated x is kept as an fp16 (hi, lo) pair,
+ * which halves the inputs of a slice).  Shapes the one-pass kernel does not
+ * take, and batch <= 8, run qgemv_fmt's path. */
+size_t qgemv_fmt_workspace_bytes(int32_t rows, int32_t cols, int32_t format, int32_t rotated,
+                                 int32_t batch);
+qmoe_status qgemv_fmt_ws(const qmoe_qmatrix_fmt *W, const uint16_t *x, int32_t batch, uint16_t *y,
+                         void *workspace, size_t workspace_bytes, int32_t *status_dev,
+                         void *stream);
+
 /* ---------------------------------------------------------------------------
  * Router + softmax + top-k + renormalisation ("내부 구조" section: the router
  * runs on resident weights and picks the top-8 experts).
@@ -310,17 +323,23 @@ qmoe_status moe_expert_down(const qmoe_moe_layer *L, const int32_t *idx, const f
  * with the arithmetic of moe_router_topk followed by moe_expert_qmlp (fp32
  * accumulation of exact products).  Layer l+1 starts after layer l has
  * finished, as it would if it consumed y[l]; the weights of later layers
- * that do not depend on the routing are streamed ahead of time.
+ * that do not depend on the routing are streamed ahead of time.  The parts
+ * of a layer output computed on different SM clusters are added with fp32
+ * atomics, so the last bits of y may differ from call to call (the routing,
+ * idx, weights and logits do not).
  * x, y: fp16 [n_layers][hidden], x 16-byte aligned (it is read 16 bytes at a
  * time); idx: int32 [n_layers][top_k], weights: fp32 [n_layers][top_k],
  * logits: fp32 [n_layers][num_experts]; idx, weights and logits may be
  * NULL.  top_k 1..16.
- * workspace: moe_decode_workspace_bytes() bytes, 16-byte aligned, ZERO-FILLED
- * before first use; each successful call leaves it zero-filled again.  Calls
- * sharing a workspace must not overlap in time.  Stacks of more than 32
- * layers are processed 32 layers per launch.  The launch is cooperative (one
- * CTA per SM, all resident); it fails with QMOE_ERR_CUDA if the GPU is busy
- * with other work that prevents co-residency.
+ * workspace: moe_decode_workspace_bytes() bytes (control words and two fp32
+ * [hidden] layer accumulators), 16-byte aligned, ZERO-FILLED before first
+ * use; each successful call leaves it zero-filled again (after a call whose
+ * status word reports a timeout, zero it again).  Calls sharing a workspace
+ * must not overlap in time.  Stacks of more than 32 layers are processed 32
+ * layers per launch.  The launch is cooperative, in clusters of 8 CTAs (one
+ * CTA per SM, as many clusters as fit at once: 15 on a 148-SM B200); it fails
+ * with QMOE_ERR_CUDA if the GPU is busy with other work that prevents
+ * co-residency.
  * ------------------------------------------------------------------------- */
 size_t moe_decode_pack_bytes(const qmoe_moe_layer *L);
 
@@ -364,8 +383,10 @@ qmoe_status moe_decode_layers(const void *const *packed_layers, int32_t n_layers
  *   SYNCHRONISES `stream` once; every other entry point never does) -> plan
  *   -> each missed expert's nine arrays host -> device, the misses spread
  *   over four copy streams (the first is `copy_stream` when given, the
- *   others the cache's own) -> the routed experts wait for the copies -> y =
- *   shared(x) + sum_j weights[j] * expert_{idx[j]}(x) from the slots (as
+ *   others the cache's own) -> meanwhile the shared expert runs on `stream`
+ *   (it needs no copy; its output is kept in fp32) -> the routed experts
+ *   wait for the copies -> y = shared(x) + sum_j weights[j] *
+ *   expert_{idx[j]}(x) from the slots, rounded once (the arithmetic of
  *   moe_expert_qmlp; same zero-filled workspace).  idx_out / weights_out
  *   (device, optional) receive the router's choice.  Returns
  *   QMOE_ERR_DEVICE_STATUS if the router produced an id outside [0, E)
@@ -451,6 +472,19 @@ const char *qmoe_status_string(qmoe_status s);
 /* Enable (1, the default) or disable (0) programmatic dependent launch for
  * all later calls in this process.  Returns the previous setting. */
 int32_t qmoe_set_dependent_launch(int32_t enable);
+
+/* Time limit of every wait inside moe_decode_layers (a wait that does not
+ * complete in time flags QMOE_DEV_TIMEOUT, stops the whole launch and lets it
+ * return), in nanoseconds; 0 restores the default of 2 s.  Applies to later
+ * calls in this process; returns the previous setting. */
+uint64_t qmoe_set_decode_wait_limit_ns(uint64_t ns);
+
+/* Experts of a prefill chunk (and the shared expert) with at least
+ * `min_tokens` tokens run on the tensor-core (tcgen05) kernels, the others on
+ * the streaming kernels; 0 sends every expert to the streaming kernels.  The
+ * default is 16.  Applies to later moe_prefill_qgemm calls in this process;
+ * returns the previous setting. */
+int32_t qmoe_set_prefill_tensor_min(int32_t min_tokens);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int32_t qmoe_version(void);

@@ -28,6 +28,8 @@ struct DevState {
 DevState g_dev[kMaxDevices];
 std::mutex g_mu;
 std::atomic<int32_t> g_pdl_enabled{1};
+std::atomic<int32_t> g_prefill_tc_min{0};
+std::atomic<unsigned long long> g_decode_wait_ns{kWaitLimitNs};
 
 qmoe_status device_state(DevState **out)
 {
@@ -182,6 +184,35 @@ qmoe_status validate_expert_qmlp(const qmoe_moe_layer *L, const uint16_t *x, con
     return device_state(&d);
 }
 
+qmoe_status expert_qmlp_slots(const qmoe_moe_layer *L, const uint16_t *x, const int32_t *idx,
+                              const float *weights, int32_t top_k, uint32_t slot_mask,
+                              float *y_part, const float *y_add, uint16_t *y, void *workspace,
+                              size_t workspace_bytes, int32_t *status_dev, void *stream)
+{
+    if (slot_mask == 0 || (slot_mask >> (top_k + 1)) != 0 || (!y_part && !y))
+        return QMOE_ERR_INVALID_ARG;
+    uint16_t *yy = y ? y : reinterpret_cast<uint16_t *>(y_part);   // alignment checks only
+    qmoe_status s = validate_expert_qmlp(L, x, idx, weights, top_k, yy, status_dev);
+    if (s != QMOE_OK)
+        return s;
+    if ((y_part && !aligned(y_part, 4)) || (y_add && !aligned(y_add, 4)))
+        return QMOE_ERR_ALIGNMENT;
+    DevState *d;
+    if ((s = device_state(&d)) != QMOE_OK)
+        return s;
+    ExpertArgs a;
+    if ((s = expert_args(L, x, idx, weights, top_k, y, workspace, workspace_bytes,
+                         status_dev ? status_dev : d->status, &a)) != QMOE_OK)
+        return s;
+    a.slot_mask = slot_mask;
+    a.y_part = y_part;
+    a.y_add = y_add;
+    const LaunchCfg c = launch_cfg(d, stream);
+    if ((s = cuda_status(launch_expert_gateup(a, c))) != QMOE_OK)
+        return s;
+    return cuda_status(launch_expert_down(a, c));
+}
+
 }  // namespace qmoe
 
 using namespace qmoe;
@@ -266,8 +297,9 @@ qmoe_status qgemv_affine_ws(const qmoe_qmatrix *W, const uint16_t *x, int32_t ba
     return cuda_status(launch_qgemm_small(a, workspace, workspace_bytes, launch_cfg(d, stream), &used));
 }
 
-qmoe_status qgemv_fmt(const qmoe_qmatrix_fmt *W, const uint16_t *x, int32_t batch, uint16_t *y,
-                      int32_t *status_dev, void *stream)
+// checks shared by qgemv_fmt and qgemv_fmt_ws; fills the launch arguments
+static qmoe_status fmt_args(const qmoe_qmatrix_fmt *W, const uint16_t *x, int32_t batch,
+                            uint16_t *y, int32_t *status_dev, DevState **d, QgemvArgs *a)
 {
     if (!W || !W->packed || !W->params || !x || !y)
         return QMOE_ERR_INVALID_ARG;
@@ -284,24 +316,62 @@ qmoe_status qgemv_fmt(const qmoe_qmatrix_fmt *W, const uint16_t *x, int32_t batc
         (status_dev && !aligned(status_dev, 4)))
         return QMOE_ERR_ALIGNMENT;
     qmoe_status s;
-    DevState *d;
-    if ((s = device_state(&d)) != QMOE_OK)
+    if ((s = device_state(d)) != QMOE_OK)
         return s;
+    a->packed = W->packed;
+    a->scales = nullptr;
+    a->biases = nullptr;
+    a->params = W->params;
+    a->signs = W->rht_signs;
+    a->N = W->rows;
+    a->K = W->cols;
+    a->fmt = W->format == QMOE_FMT_ZP4_BF16 ? QG_ZP4 : QG_SYM8;
+    a->bits = W->format == QMOE_FMT_ZP4_BF16 ? 4 : 8;
+    a->x = reinterpret_cast<const __half *>(x);
+    a->B = batch;
+    a->y = reinterpret_cast<__half *>(y);
+    a->status = status_dev ? status_dev : (*d)->status;
+    return QMOE_OK;
+}
+
+qmoe_status qgemv_fmt(const qmoe_qmatrix_fmt *W, const uint16_t *x, int32_t batch, uint16_t *y,
+                      int32_t *status_dev, void *stream)
+{
+    DevState *d;
     QgemvArgs a;
-    a.packed = W->packed;
-    a.scales = nullptr;
-    a.biases = nullptr;
-    a.params = W->params;
-    a.signs = W->rht_signs;
-    a.N = W->rows;
-    a.K = W->cols;
-    a.fmt = W->format == QMOE_FMT_ZP4_BF16 ? QG_ZP4 : QG_SYM8;
-    a.bits = W->format == QMOE_FMT_ZP4_BF16 ? 4 : 8;
-    a.x = reinterpret_cast<const __half *>(x);
-    a.B = batch;
-    a.y = reinterpret_cast<__half *>(y);
-    a.status = status_dev ? status_dev : d->status;
+    const qmoe_status s = fmt_args(W, x, batch, y, status_dev, &d, &a);
+    if (s != QMOE_OK)
+        return s;
     return cuda_status(launch_qgemv_batched(a, launch_cfg(d, stream)));
+}
+
+size_t qgemv_fmt_workspace_bytes(int32_t rows, int32_t cols, int32_t format, int32_t rotated,
+                                 int32_t batch)
+{
+    if (rows <= 0 || cols <= 0 || batch < 1 || batch > kMaxQgemvBatch ||
+        (format != QMOE_FMT_ZP4_BF16 && format != QMOE_FMT_SYM8_BF16))
+        return 0;
+    return qgemm_small_workspace_bytes(rows, cols, format == QMOE_FMT_ZP4_BF16 ? 4 : 8, batch,
+                                       rotated != 0);
+}
+
+qmoe_status qgemv_fmt_ws(const qmoe_qmatrix_fmt *W, const uint16_t *x, int32_t batch, uint16_t *y,
+                         void *workspace, size_t workspace_bytes, int32_t *status_dev,
+                         void *stream)
+{
+    DevState *d;
+    QgemvArgs a;
+    qmoe_status s = fmt_args(W, x, batch, y, status_dev, &d, &a);
+    if (s != QMOE_OK)
+        return s;
+    if (workspace && !aligned(workspace, 16))
+        return QMOE_ERR_ALIGNMENT;
+    const size_t need =
+        qgemm_small_workspace_bytes(a.N, a.K, a.bits, batch, W->rht_signs != nullptr);
+    if (need > 0 && (!workspace || workspace_bytes < need))
+        return QMOE_ERR_INVALID_ARG;
+    bool used = false;
+    return cuda_status(launch_qgemm_small(a, workspace, workspace_bytes, launch_cfg(d, stream), &used));
 }
 
 qmoe_status moe_router_topk(const qmoe_qmatrix *router, const uint16_t *x, int32_t tokens,
@@ -544,7 +614,8 @@ qmoe_status moe_decode_layers(const void *const *packed_layers, int32_t n_layers
     a.H = hidden;
     a.I = inter;
     a.top_k = top_k;
-    a.NS_r = 0;
+    a.NS = 0;
+    a.wait_ns = g_decode_wait_ns.load();
     a.status = status_dev ? status_dev : d->status;
     decode_workspace_layout(a.E, a.H, a.I, top_k, workspace, &a.ws);
     for (int l0 = 0; l0 < n_layers; l0 += kDecodeMaxLayers) {
@@ -643,6 +714,8 @@ qmoe_status moe_prefill_qgemm(const qmoe_moe_layer *L, const uint16_t *x, int32_
     a.y = reinterpret_cast<__half *>(y);
     a.status = status_dev ? status_dev : d->status;
     prefill_workspace_layout(a.E, a.H, a.I, tokens, top_k, workspace, &a.ws);
+    const int tc_min = g_prefill_tc_min.load();
+    a.tc_min = (tc_min > 0 && prefill_tc_supported(a.H, a.I)) ? tc_min : (1 << 30);
     return cuda_status(launch_prefill(a, launch_cfg(d, stream)));
 }
 
@@ -721,6 +794,16 @@ const char *qmoe_status_string(qmoe_status s)
 int32_t qmoe_set_dependent_launch(int32_t enable)
 {
     return g_pdl_enabled.exchange(enable ? 1 : 0);
+}
+
+uint64_t qmoe_set_decode_wait_limit_ns(uint64_t ns)
+{
+    return g_decode_wait_ns.exchange(ns == 0 ? kWaitLimitNs : ns);
+}
+
+int32_t qmoe_set_prefill_tensor_min(int32_t min_tokens)
+{
+    return g_prefill_tc_min.exchange(min_tokens < 0 ? 0 : min_tokens);
 }
 
 int32_t qmoe_version(void) { return 100; }

@@ -160,6 +160,7 @@ struct qmoe_expert_cache {
     int32_t *idx_dev;       // device [kMaxTopK]
     float *wt_dev;          // device [kMaxTopK]
     int32_t *slot_dev;      // device [kMaxTopK]
+    float *ysh_dev;         // device fp32 [hidden]: the shared expert's output
     cudaStream_t copy[kCopyStreams];   // the cache's own copy streams
     cudaEvent_t copied[kCopyStreams];
     int64_t hits, misses, bytes;
@@ -231,6 +232,8 @@ qmoe_status qmoe_cache_create(const qmoe_moe_layer *host, const qmoe_moe_layer *
         e = cudaMalloc(&c->wt_dev, kMaxTopK * sizeof(float));
     if (e == cudaSuccess)
         e = cudaMalloc(&c->slot_dev, kMaxTopK * sizeof(int32_t));
+    if (e == cudaSuccess)
+        e = cudaMalloc(&c->ysh_dev, (size_t)host->hidden * sizeof(float));
     for (int i = 0; i < kCopyStreams && e == cudaSuccess; ++i) {
         e = cudaStreamCreateWithFlags(&c->copy[i], cudaStreamNonBlocking);
         if (e == cudaSuccess)
@@ -258,6 +261,8 @@ void qmoe_cache_destroy(qmoe_expert_cache *c)
         cudaFree(c->wt_dev);
     if (c->slot_dev)
         cudaFree(c->slot_dev);
+    if (c->ysh_dev)
+        cudaFree(c->ysh_dev);
     for (int i = 0; i < kCopyStreams; ++i) {
         if (c->copied[i])
             cudaEventDestroy(c->copied[i]);
@@ -340,7 +345,13 @@ qmoe_status moe_cache_layer(qmoe_expert_cache *c, const qmoe_qmatrix *router, co
     }
     c->hits += top_k - nm;
     c->misses += nm;
-    // 5. the routed experts wait for the copies; the slot ids follow the plan
+    // 5. the shared expert needs no copy: it runs on `stream` while the
+    //    missed experts are in flight, its fp32 output kept for the sum
+    s = expert_qmlp_slots(&c->slots, x, c->slot_dev, c->wt_dev, top_k, 1u, c->ysh_dev, nullptr,
+                          nullptr, workspace, workspace_bytes, status_dev, stream);
+    if (s != QMOE_OK)
+        return fail(s);
+    // 6. the routed experts wait for the copies; the slot ids follow the plan
     for (int i = 0; i < nstreams; ++i)
         if (cudaEventRecord(ev[i], cs[i]) != cudaSuccess ||
             cudaStreamWaitEvent(st, ev[i], 0) != cudaSuccess)
@@ -348,9 +359,10 @@ qmoe_status moe_cache_layer(qmoe_expert_cache *c, const qmoe_qmatrix *router, co
     if (cudaMemcpyAsync(c->slot_dev, c->slot_host, top_k * sizeof(int32_t),
                         cudaMemcpyHostToDevice, st) != cudaSuccess)
         return fail(QMOE_ERR_CUDA);
-    // 6. shared + routed experts from the slots
-    s = moe_expert_qmlp(&c->slots, x, c->slot_dev, c->wt_dev, top_k, y, workspace,
-                        workspace_bytes, status_dev, stream);
+    // 7. y = shared output + sum_j weights[j] * routed expert j, from the slots
+    const uint32_t routed = ((1u << top_k) - 1u) << 1;
+    s = expert_qmlp_slots(&c->slots, x, c->slot_dev, c->wt_dev, top_k, routed, nullptr,
+                          c->ysh_dev, y, workspace, workspace_bytes, status_dev, stream);
     if (s != QMOE_OK)
         return fail(s);
     if (idx_out && cudaMemcpyAsync(idx_out, c->idx_dev, top_k * sizeof(int32_t),

@@ -99,6 +99,16 @@ __device__ __forceinline__ int routed_expert(const ExpertArgs &a, int j, bool *v
 // per thread after the ids are complete (top_k <= 16).
 __device__ __forceinline__ uint32_t owned_slots(const ExpertArgs &a)
 {
+    if (a.slot_mask) {   // an explicit choice: the routed slots among it with a valid id
+        uint32_t m = a.slot_mask & 1u;
+        for (int j = 0; j < a.top_k; ++j)
+            if ((a.slot_mask >> (j + 1)) & 1u) {
+                const int e = __ldcg(a.idx + j);
+                if (e >= 0 && e < a.E)
+                    m |= 1u << (j + 1);
+            }
+        return m;
+    }
     uint32_t m = a.ep_rank == 0 ? 1u : 0u;
     const int per = a.E / a.ep_world;
     for (int j = 0; j < a.top_k; ++j) {
@@ -140,7 +150,8 @@ __global__ void __launch_bounds__(GU_THREADS, 1) expert_gateup_kernel(ExpertArgs
             bool waited = false, bad = false;
             int last_use[GU_STAGES] = {-1, -1, -1};
             int k = 0;
-            uint32_t mine = a.ep_rank == 0 ? 1u : 0u;   // before the ids: the shared slot only
+            // before the ids are known: the shared slot only
+            uint32_t mine = a.slot_mask ? (a.slot_mask & 1u) : (a.ep_rank == 0 ? 1u : 0u);
             for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
                 const int so = item / octs, oct = item % octs;
                 QMat g = a.sh_gate, u = a.sh_up;
@@ -370,9 +381,13 @@ __global__ void __launch_bounds__(DN_THREADS, 1) expert_down_kernel(ExpertArgs a
     const uint32_t mine = EP ? owned_slots(a) : ~0u;
     const int n_owned = EP ? __popc(mine) : nslot;
     if (n_owned == 0) {   // nothing to add here: this rank's share is zero
-        if (a.y_part)
-            for (int row = blockIdx.x * DN_CW * 32 + threadIdx.x; row < a.H; row += gridDim.x * DN_CW * 32)
-                a.y_part[row] = 0.f;
+        for (int row = blockIdx.x * DN_CW * 32 + threadIdx.x; row < a.H; row += gridDim.x * DN_CW * 32) {
+            const float v = a.y_add ? __ldcg(a.y_add + row) : 0.f;
+            if (a.y_part)
+                a.y_part[row] = v;
+            else if (a.slot_mask)
+                a.y[row] = __float2half_rn(v);
+        }
         return;
     }
     const int gid = lane >> 2, tig = lane & 3;
@@ -419,6 +434,8 @@ __global__ void __launch_bounds__(DN_THREADS, 1) expert_down_kernel(ExpertArgs a
             if (lane < 16) {
                 const int row = r0 + lane;
                 float v = (mine & 1u) ? __ldcg(a.ws.part + (size_t)a.top_k * a.H + row) : 0.f;
+                if (a.y_add)
+                    v += __ldcg(a.y_add + row);
                 for (int j = 0; j < a.top_k; ++j) {
                     const int e = __ldcg(a.idx + j);
                     if (e >= 0 && e < a.E && ((mine >> (j + 1)) & 1u))
@@ -444,7 +461,7 @@ cudaError_t launch_expert_gateup(const ExpertArgs &a, const LaunchCfg &c)
         return cudaErrorInvalidValue;
     const int n_items = (a.top_k + 1) * (a.I / 8);
     const int grid = n_items < c.num_sms ? n_items : c.num_sms;
-    const bool ep = a.ep_world > 1;
+    const bool ep = a.ep_world > 1 || a.slot_mask != 0;
     cudaError_t e = ep ? set_smem(expert_gateup_kernel<true>, L.total) : set_smem(expert_gateup_kernel<false>, L.total);
     if (e != cudaSuccess)
         return e;
@@ -464,7 +481,7 @@ cudaError_t launch_expert_down(const ExpertArgs &a, const LaunchCfg &c)
     const DnLayout L = dn_layout(a.I, a.top_k, NS);
     const int n_items = (a.top_k + 1) * (a.H / 16);
     const int grid = n_items < c.num_sms ? n_items : c.num_sms;
-    const bool ep = a.ep_world > 1;
+    const bool ep = a.ep_world > 1 || a.slot_mask != 0;
     cudaError_t e = ep ? set_smem(expert_down_kernel<true>, L.total) : set_smem(expert_down_kernel<false>, L.total);
     if (e != cudaSuccess)
         return e;

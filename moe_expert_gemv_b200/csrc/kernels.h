@@ -47,7 +47,7 @@ cudaError_t launch_qgemv_batched(const QgemvArgs &a, const LaunchCfg &c);
 // call needs, 0 if the shape runs without one; the launch falls back to
 // launch_qgemv_batched where the shape or alignment rule it out.  *used_ws
 // reports whether the workspace was used.
-size_t qgemm_small_workspace_bytes(int N, int K, int bits, int B);
+size_t qgemm_small_workspace_bytes(int N, int K, int bits, int B, bool rot = false);
 cudaError_t launch_qgemm_small(const QgemvArgs &a, void *ws, size_t ws_bytes, const LaunchCfg &c,
                                bool *used_ws);
 
@@ -65,6 +65,18 @@ bool encode_codes_map(CUtensorMap *m, const uint32_t *packed, long rows, int Kw,
 // is not a multiple of 16 bytes.
 bool encode_u16_map_2d(CUtensorMap *m, const void *base, long rows, int cols, int box_cols,
                        int box_rows);
+// the same for a row-major 32-bit array (the parameter words of the formats)
+bool encode_u32_map_2d(CUtensorMap *m, const void *base, long rows, int cols, int box_cols,
+                       int box_rows);
+
+// scale and folded-bias factor of one parameter word of the bf16 formats:
+// ZP4 w = s(q - z) -> (s, -s z); SYM8 w = s(q' - 128) with q' = q + 128 -> (s, -128 s)
+template <int FMT>
+__device__ __forceinline__ void fmt_scale_bias(uint32_t p, float &s, float &b)
+{
+    s = __uint_as_float(p << 16);
+    b = FMT == QG_ZP4 ? -s * (float)((p >> 16) & 0xFFu) : -128.f * s;
+}
 
 // ------------------------------------------------------------------ router --
 struct RouterArgs {
@@ -113,8 +125,18 @@ struct ExpertArgs {
     // y_part set, the sum of its slots goes there in fp32 instead of y
     int ep_rank = 0, ep_world = 1, ep_first = 0;
     float *y_part = nullptr;   // [H]
+    // an explicit choice of slots instead (bit 0 the shared expert, bit j + 1
+    // routed slot j), and an fp32 [H] vector added to the sum of those slots
+    uint32_t slot_mask = 0;
+    const float *y_add = nullptr;
 };
 cudaError_t launch_expert_gateup(const ExpertArgs &a, const LaunchCfg &c);
+// moe_expert_qmlp restricted to the slots of slot_mask (see ExpertArgs),
+// the sum written to y_part (fp32) when given, else y_add + sum to y (fp16)
+qmoe_status expert_qmlp_slots(const qmoe_moe_layer *L, const uint16_t *x, const int32_t *idx,
+                              const float *weights, int32_t top_k, uint32_t slot_mask,
+                              float *y_part, const float *y_add, uint16_t *y, void *workspace,
+                              size_t workspace_bytes, int32_t *status_dev, void *stream);
 cudaError_t launch_expert_down(const ExpertArgs &a, const LaunchCfg &c);
 cudaError_t launch_f32_to_f16(const float *src, __half *dst, long n, cudaStream_t s);
 
@@ -129,17 +151,15 @@ size_t decode_pack_bytes(int E, int H, int I);
 cudaError_t launch_decode_pack(const DecodePackArgs &a, void *dst, cudaStream_t s);
 
 struct DecodeWorkspace {
-    unsigned *ctl;                   // control words: router / done / exit / abort counters,
-                                     // then one readiness counter per slot (zero between launches)
-    int *counters;                   // [H / 32] arrival counters (zero between launches)
-    float *logits_part;              // [2][E]
-    uint4 *hfrag;                    // [top_k + 1][I/64][2][2][4] fp16 fragments of h (hi, lo)
-    float *part;                     // [top_k + 1][H] per-expert down outputs
+    unsigned *ctl;   // control words: layer arrivals, abort, exit (zero between launches)
+    float *y_acc;    // [2][H] fp32 layer outputs being summed (zero between launches)
 };
 size_t decode_workspace_layout(int E, int H, int I, int top_k, void *base, DecodeWorkspace *ws);
 
 struct DecodeArgs {
-    int L, E, H, I, top_k, NS_r;
+    int L, E, H, I, top_k;
+    int NS;               // ring stages (set by launch_decode)
+    unsigned long long wait_ns = 2000000000ull;   // limit of every wait of the kernel (ns)
     const __half *x;      // [L][H]
     __half *y;            // [L][H]
     int32_t *idx;         // [L][top_k] or null
@@ -164,6 +184,16 @@ struct PrefillWorkspace {
     uint4 *hfrag;       // per position: h (hi, lo) fragments (+64 B pad)
     float *hsum;        // per position: group sums of h hi / lo
     float *r;           // [T * top_k + T][H] unweighted expert outputs per position
+    // the tensor-core path of the heavy slots (prefill_tc.cu); activation rows
+    // keep the k order (0,4,1,5,2,6,3,7) inside every 8 inputs
+    int32_t *heavy;     // [E + 1] heavy slots, most tokens first (count in unit_ctr[3])
+    __half *xg;         // [npos][H] x of each position's token
+    __half *xb_hi;      // [npos][64] group sums of x, fp16 (hi, lo) pair, zero-padded
+    __half *xb_lo;
+    __half *hb_hi;      // [npos][I] h, fp16 (hi, lo) pair
+    __half *hb_lo;
+    __half *hs_hi;      // [npos][64] group sums of h (hi + lo), as a pair, zero-padded
+    __half *hs_lo;
 };
 size_t prefill_workspace_layout(int E, int hidden, int inter, int T, int top_k, void *base,
                                 PrefillWorkspace *ws);
@@ -185,8 +215,13 @@ struct PrefillArgs {
     __half *y;             // [T][H]
     PrefillWorkspace ws;
     int32_t *status;
+    int tc_min = 1 << 30;  // slots with at least this many tokens take the tensor-core path
 };
 cudaError_t launch_prefill(const PrefillArgs &a, const LaunchCfg &c);
+// the heavy slots on tcgen05 (prefill_tc.cu): gate/up + SwiGLU, or down
+cudaError_t launch_prefill_tc(const PrefillArgs &a, const LaunchCfg &c, bool down);
+bool prefill_tc_supported(int hidden, int inter);
+constexpr int kTcMinTokens = 16;
 // the shared-memory ring of the grouped kernels holds at least two units
 bool prefill_shape_supported(int hidden, int inter);
 

@@ -102,6 +102,12 @@ __device__ __forceinline__ int pos_token(const PrefillArgs &a, int p)
     return p < tk ? a.ws.pairs[p] / a.top_k : p - tk;
 }
 
+// slot s goes to the tensor-core kernels (prefill_tc.cu)
+__device__ __forceinline__ bool slot_heavy(const PrefillArgs &a, int s)
+{
+    return slot_count(a, s) >= a.tc_min;
+}
+
 // ------------------------------------------------------------- stage layout --
 struct PfStage {
     int rows;           // rows per matrix tile
@@ -244,6 +250,31 @@ __global__ void __launch_bounds__(128) prefill_prep_kernel(PrefillArgs a)
         stage_x_groups<kPermS4>(a.ws.xfrag + (size_t)p * d.xg_stride,
                                 a.ws.xsum + (size_t)p * d.xs_stride, d.GH, 1,
                                 a.x + (size_t)tok * d.H, d.H, threadIdx.x, 128, 1);
+        if (a.tc_min <= a.T) {
+            // the tensor-core path's rows: x in the k order (0,4,1,5,2,6,3,7)
+            // of every 8 inputs, its group sums as an fp16 pair, and zeroed h
+            // sums (only the groups that exist are written later)
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)tok * d.H);
+            uint4 *dst = reinterpret_cast<uint4 *>(a.ws.xg + (size_t)p * d.H);
+            for (int c = threadIdx.x; c < d.H / 8; c += blockDim.x) {
+                const uint4 v = __ldg(src + c);
+                dst[c] = make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632),
+                                    __byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
+            }
+            if (threadIdx.x < 64) {
+                const int g = threadIdx.x;
+                float sum = 0.f;
+                if (g < d.GH)
+                    for (int k = 0; k < kGroup; ++k)
+                        sum += __half2float(a.x[(size_t)tok * d.H + g * kGroup + k]);
+                const __half hi = __float2half_rn(sum);
+                const int col = (g & ~7) | ((g & 3) << 1) | ((g & 7) >> 2);
+                a.ws.xb_hi[(size_t)p * 64 + col] = hi;
+                a.ws.xb_lo[(size_t)p * 64 + col] = __float2half_rn(sum - __half2float(hi));
+                a.ws.hs_hi[(size_t)p * 64 + g] = __float2half(0.f);
+                a.ws.hs_lo[(size_t)p * 64 + g] = __float2half(0.f);
+            }
+        }
     }
     if (p == 0) {
         // token tiles of every slot in slot order: a block-wide exclusive scan
@@ -254,7 +285,7 @@ __global__ void __launch_bounds__(128) prefill_prep_kernel(PrefillArgs a)
             s_base = 0;
         for (int s0 = 0; s0 <= d.E; s0 += 128) {
             const int s = s0 + threadIdx.x;
-            const int nt = s <= d.E ? (slot_count(a, s) + TILE_T - 1) / TILE_T : 0;
+            const int nt = (s <= d.E && !slot_heavy(a, s)) ? (slot_count(a, s) + TILE_T - 1) / TILE_T : 0;
             s_scan[threadIdx.x] = nt;
             __syncthreads();
             for (int o = 1; o < 128; o <<= 1) {   // inclusive Hillis-Steele scan
@@ -276,6 +307,29 @@ __global__ void __launch_bounds__(128) prefill_prep_kernel(PrefillArgs a)
             a.ws.unit_ctr[1] = 0;
             a.ws.unit_ctr[2] = s_base;
         }
+        // heavy slots, most tokens first (ties: lower slot first)
+        int nh = 0;
+        for (int s = threadIdx.x; s <= d.E; s += blockDim.x) {
+            if (!slot_heavy(a, s))
+                continue;
+            const int cs = slot_count(a, s);
+            int rank = 0;
+            for (int s2 = 0; s2 <= d.E; ++s2)
+                if (slot_heavy(a, s2)) {
+                    const int c2 = slot_count(a, s2);
+                    rank += (c2 > cs || (c2 == cs && s2 < s)) ? 1 : 0;
+                }
+            a.ws.heavy[rank] = s;
+            ++nh;
+        }
+        __shared__ int s_nh;
+        if (threadIdx.x == 0)
+            s_nh = 0;
+        __syncthreads();
+        atomicAdd(&s_nh, nh);
+        __syncthreads();
+        if (threadIdx.x == 0)
+            a.ws.unit_ctr[3] = s_nh;
         // positions of the valid pairs (ids out of range were dropped by the
         // grouping, so only offsets[E] positions hold a pair)
         for (int q = threadIdx.x; q < nvalid; q += blockDim.x)
@@ -824,6 +878,11 @@ size_t prefill_workspace_layout(int E, int H, int I, int T, int top_k, void *bas
     const size_t hfrag_off = take((size_t)d.npos * d.hf_stride * 16);
     const size_t hsum_off = take((size_t)d.npos * d.hs_stride * 4);
     const size_t r_off = take((size_t)d.npos * H * 4);
+    const size_t heavy_off = take((size_t)(E + 1) * 4);
+    const size_t xg_off = take((size_t)d.npos * H * 2);
+    const size_t xb_off = take((size_t)d.npos * 64 * 2 * 2);
+    const size_t hb_off = take((size_t)d.npos * I * 2 * 2);
+    const size_t hs_off = take((size_t)d.npos * 64 * 2 * 2);
     if (base && ws) {
         unsigned char *b = static_cast<unsigned char *>(base);
         ws->counts = reinterpret_cast<int32_t *>(b + counts_off);
@@ -837,6 +896,14 @@ size_t prefill_workspace_layout(int E, int H, int I, int T, int top_k, void *bas
         ws->hfrag = reinterpret_cast<uint4 *>(b + hfrag_off);
         ws->hsum = reinterpret_cast<float *>(b + hsum_off);
         ws->r = reinterpret_cast<float *>(b + r_off);
+        ws->heavy = reinterpret_cast<int32_t *>(b + heavy_off);
+        ws->xg = reinterpret_cast<__half *>(b + xg_off);
+        ws->xb_hi = reinterpret_cast<__half *>(b + xb_off);
+        ws->xb_lo = ws->xb_hi + (size_t)d.npos * 64;
+        ws->hb_hi = reinterpret_cast<__half *>(b + hb_off);
+        ws->hb_lo = ws->hb_hi + (size_t)d.npos * I;
+        ws->hs_hi = reinterpret_cast<__half *>(b + hs_off);
+        ws->hs_lo = ws->hs_hi + (size_t)d.npos * 64;
     }
     return off;
 }
@@ -890,6 +957,9 @@ cudaError_t launch_prefill(const PrefillArgs &a, const LaunchCfg &c)
     if ((e = launch_ex(prefill_gateup_kernel, dim3(c.num_sms), dim3(PF_THREADS), smem_gu, c, 1, a,
                        sgu, ns_gu, mg, mu, msg, msu)) != cudaSuccess)
         return e;
+    const bool tc = a.tc_min <= a.T;
+    if (tc && (e = launch_prefill_tc(a, c, false)) != cudaSuccess)
+        return e;
     if ((e = launch_ex(prefill_hsum_kernel, dim3(c.num_sms), dim3(256), 0, c, 1, a)) != cudaSuccess)
         return e;
 
@@ -908,6 +978,8 @@ cudaError_t launch_prefill(const PrefillArgs &a, const LaunchCfg &c)
         return e;
     if ((e = launch_ex(prefill_down_kernel, dim3(c.num_sms), dim3(PF_THREADS), smem_dn, c, 1, a,
                        sdn, ns_dn, md, msd)) != cudaSuccess)
+        return e;
+    if (tc && (e = launch_prefill_tc(a, c, true)) != cudaSuccess)
         return e;
     return launch_ex(prefill_combine_kernel, dim3(c.num_sms * 2), dim3(256), 0, c, 1, a);
 }

@@ -49,6 +49,7 @@ constexpr int SM_MAX_CTA_TILES = 1024;     // tiles one CTA may take (flags in s
 
 struct SmArgs {
     const __half *x;
+    const uint32_t *signs;   // rotation signs [K / 32] (formats with the rotation)
     __half *y;
     unsigned *ctr;      // [tiles] arrival counters, zero between calls
     float4 *part;       // [tiles][S][MT * NT * 32] partial tiles (S > 1)
@@ -58,17 +59,21 @@ struct SmArgs {
 
 struct SmLayout {
     int GS;
-    size_t xs_off, xsum_off, red_off, last_off, bar_off, stage_off;
+    size_t xs_off, xslo_off, xsum_off, red_off, last_off, bar_off, stage_off;
     size_t codes_bytes, sb_bytes, stage_bytes, total;
 };
 
-__host__ __device__ inline SmLayout sm_layout(int KS, int bits, int B, int TM, int NS)
+__host__ __device__ inline SmLayout sm_layout(int KS, int bits, int B, int TM, int NS,
+                                              bool rot = false)
 {
     SmLayout L;
     L.GS = KS / kGroup;
     size_t off = 0;
     L.xs_off = off;   // x fragments: uint4 per (group, half, column, quad lane)
     off += (size_t)L.GS * 2 * B * 4 * 16;
+    L.xslo_off = off;   // the lo parts of a rotated x, same layout
+    if (rot)
+        off += (size_t)L.GS * 2 * B * 4 * 16;
     L.xsum_off = off;   // group sums: [GS][32]
     off += (size_t)L.GS * 32 * 4;
     L.red_off = off;   // one float4 per (warp, n-tile, lane)
@@ -97,7 +102,9 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int c0,
         : "memory");
 }
 
-template <int BITS>
+// (XOR80: two's-complement bytes q -> q + 128 = byte ^ 0x80, the symmetric
+// 8-bit format)
+template <int BITS, bool XOR80 = false>
 __device__ __forceinline__ void dequant_frags(const void *fa, const void *fb, uint32_t (&pa)[8],
                                               uint32_t (&pb)[8])
 {
@@ -109,8 +116,18 @@ __device__ __forceinline__ void dequant_frags(const void *fa, const void *fb, ui
         dequant4s_word(wb.x, pb);
         dequant4s_word(wb.y, pb + 4);
     } else {
-        const uint4 wa = *reinterpret_cast<const uint4 *>(fa);
-        const uint4 wb = *reinterpret_cast<const uint4 *>(fb);
+        uint4 wa = *reinterpret_cast<const uint4 *>(fa);
+        uint4 wb = *reinterpret_cast<const uint4 *>(fb);
+        if (XOR80) {
+            wa.x ^= 0x80808080u;
+            wa.y ^= 0x80808080u;
+            wa.z ^= 0x80808080u;
+            wa.w ^= 0x80808080u;
+            wb.x ^= 0x80808080u;
+            wb.y ^= 0x80808080u;
+            wb.z ^= 0x80808080u;
+            wb.w ^= 0x80808080u;
+        }
         dequant8s_word(wa.x, pa);
         dequant8s_word(wa.y, pa + 2);
         dequant8s_word(wa.z, pa + 4);
@@ -143,7 +160,11 @@ __device__ __forceinline__ void store_unit(const SmArgs &a, int t, int mt, int n
     }
 }
 
-template <int BITS, int NT>
+// FMT: QG_AFFINE (fp16 scale + bias arrays: two 2-D copies per tile), or
+// QG_ZP4 / QG_SYM8 (one bf16-scale parameter word per group: one 2-D copy
+// into the same bytes); ROT: x rotated by the block-32 Hadamard transform and
+// kept as an fp16 (hi, lo) pair, both parts through the same dequantised codes
+template <int BITS, int NT, int FMT, bool ROT>
 __global__ void __launch_bounds__(SM_THREADS, 1)
     qgemm_small_kernel(SmArgs a, int NS, const __grid_constant__ CUtensorMap codes_map,
                        const __grid_constant__ CUtensorMap scales_map,
@@ -151,8 +172,9 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const SmLayout L = sm_layout(a.KS, BITS, a.B, a.TM, NS);
+    const SmLayout L = sm_layout(a.KS, BITS, a.B, a.TM, NS, ROT);
     uint4 *xs = reinterpret_cast<uint4 *>(smem + L.xs_off);
+    uint4 *xs_lo = reinterpret_cast<uint4 *>(smem + L.xslo_off);
     float *xsum = reinterpret_cast<float *>(smem + L.xsum_off);
     float4 *red = reinterpret_cast<float4 *>(smem + L.red_off);
     int *s_last = reinterpret_cast<int *>(smem + L.last_off);
@@ -180,7 +202,8 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
         if (lane == 0) {
             prefetch_tensormap(&codes_map);
             prefetch_tensormap(&scales_map);
-            prefetch_tensormap(&biases_map);
+            if (FMT == QG_AFFINE)
+                prefetch_tensormap(&biases_map);
             const uint64_t pol = l2_evict_first_policy();
             const int cps = a.KS * BITS / 32 / 32;   // 128-byte chunks per slice row
             int k = 0;
@@ -195,9 +218,12 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
                 // tensor copies deliver whole boxes (rows past N zero-filled)
                 mbar_arrive_expect_tx(&full[st], (uint32_t)(L.codes_bytes + 2 * L.sb_bytes));
                 tma_load_3d(stage, &codes_map, 0, t * a.TM, q * cps, &full[st], pol);
+                // affine: scales then biases; formats: the parameter words
+                // (4 bytes per group, the same bytes)
                 tma_load_2d(stage + L.codes_bytes, &scales_map, q * L.GS, t * a.TM, &full[st], pol);
-                tma_load_2d(stage + L.codes_bytes + L.sb_bytes, &biases_map, q * L.GS, t * a.TM,
-                            &full[st], pol);
+                if (FMT == QG_AFFINE)
+                    tma_load_2d(stage + L.codes_bytes + L.sb_bytes, &biases_map, q * L.GS, t * a.TM,
+                                &full[st], pol);
                 last_use[st] = use;
             }
             // no copy may still be landing when the CTA exits
@@ -215,7 +241,11 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
     constexpr int KIND = BITS == 4 ? kPermS4 : 8;
     constexpr float kCodeScale = BITS == 4 ? kSub20 : kSub24;
     // this slice of x: columns 0..B-1 staged, sums of columns B..31 zero
-    stage_x_groups<KIND>(xs, xsum, L.GS, a.B, a.x + (size_t)q * a.KS, a.K, ctid, SM_CT, 32);
+    if (ROT)
+        stage_x_groups<KIND, true>(xs, xsum, L.GS, a.B, a.x + (size_t)q * a.KS, a.K, ctid, SM_CT, 32,
+                                   a.signs + (size_t)q * (a.KS / 32), xs_lo);
+    else
+        stage_x_groups<KIND>(xs, xsum, L.GS, a.B, a.x + (size_t)q * a.KS, a.K, ctid, SM_CT, 32);
     for (int t = ctid; t < L.GS * 32; t += SM_CT)
         if ((t & 31) >= a.B)
             xsum[t] = 0.f;
@@ -244,14 +274,24 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
             const unsigned char *stage = smem + L.stage_off + (size_t)st * L.stage_bytes;
             const __half *sc = reinterpret_cast<const __half *>(stage + L.codes_bytes);
             const __half *bi = reinterpret_cast<const __half *>(stage + L.codes_bytes + L.sb_bytes);
+            const uint32_t *prm = reinterpret_cast<const uint32_t *>(stage + L.codes_bytes);
             for (int g = g0; g < g0 + gpw; ++g) {
                 uint32_t pa[8], pb[8];
-                dequant_frags<BITS>(swz128_frag<BITS>(stage, chunk_bytes, r_lo, g, tig),
-                                    swz128_frag<BITS>(stage, chunk_bytes, r_hi, g, tig), pa, pb);
-                const float s_lo = __half2float(sc[r_lo * L.GS + g]) * kCodeScale;
-                const float s_hi = __half2float(sc[r_hi * L.GS + g]) * kCodeScale;
-                const float b_lo = __half2float(bi[r_lo * L.GS + g]);
-                const float b_hi = __half2float(bi[r_hi * L.GS + g]);
+                dequant_frags<BITS, FMT == QG_SYM8>(swz128_frag<BITS>(stage, chunk_bytes, r_lo, g, tig),
+                                                    swz128_frag<BITS>(stage, chunk_bytes, r_hi, g, tig),
+                                                    pa, pb);
+                float s_lo, s_hi, b_lo, b_hi;
+                if (FMT == QG_AFFINE) {
+                    s_lo = __half2float(sc[r_lo * L.GS + g]);
+                    s_hi = __half2float(sc[r_hi * L.GS + g]);
+                    b_lo = __half2float(bi[r_lo * L.GS + g]);
+                    b_hi = __half2float(bi[r_hi * L.GS + g]);
+                } else {
+                    fmt_scale_bias<FMT>(prm[r_lo * L.GS + g], s_lo, b_lo);
+                    fmt_scale_bias<FMT>(prm[r_hi * L.GS + g], s_hi, b_hi);
+                }
+                s_lo *= kCodeScale;
+                s_hi *= kCodeScale;
                 // one mma per accumulator first, then the dependent ones
                 float c[NT][4], d[NT][4];
                 uint4 x0[NT], x1[NT];
@@ -286,6 +326,28 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
                     } else {
                         mma_16816(c[nt], pa[4], pb[4], pa[5], pb[5], x1[nt].x, x1[nt].y);
                         mma_16816(d[nt], pa[6], pb[6], pa[7], pb[7], x1[nt].z, x1[nt].w);
+                    }
+                }
+                if (ROT) {   // the lo part of the rotated x through the same codes
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const int n = nt * 8 + gid;
+                        uint4 l0 = make_uint4(0, 0, 0, 0), l1 = l0;
+                        if (n < a.B) {
+                            l0 = xs_lo[((g * 2 + 0) * a.B + n) * 4 + tig];
+                            l1 = xs_lo[((g * 2 + 1) * a.B + n) * 4 + tig];
+                        }
+                        if (BITS == 4) {
+                            mma_16816(c[nt], pa[0], pb[0], pa[2], pb[2], l0.x, l0.y);
+                            mma_16816(d[nt], pa[1], pb[1], pa[3], pb[3], l1.x, l1.y);
+                            mma_16816(c[nt], pa[4], pb[4], pa[6], pb[6], l0.z, l0.w);
+                            mma_16816(d[nt], pa[5], pb[5], pa[7], pb[7], l1.z, l1.w);
+                        } else {
+                            mma_16816(c[nt], pa[0], pb[0], pa[1], pb[1], l0.x, l0.y);
+                            mma_16816(d[nt], pa[2], pb[2], pa[3], pb[3], l0.z, l0.w);
+                            mma_16816(c[nt], pa[4], pb[4], pa[5], pb[5], l1.x, l1.y);
+                            mma_16816(d[nt], pa[6], pb[6], pa[7], pb[7], l1.z, l1.w);
+                        }
                     }
                 }
 #pragma unroll
@@ -371,7 +433,7 @@ struct SmPlan {
     size_t smem, ws_bytes, part_bytes;
 };
 
-SmPlan plan_small(int N, int K, int bits, int B)
+SmPlan plan_small(int N, int K, int bits, int B, bool rot = false)
 {
     SmPlan p;
     memset(&p, 0, sizeof(p));
@@ -386,7 +448,7 @@ SmPlan plan_small(int N, int K, int bits, int B)
         const int KS = K / S, GS = KS / kGroup;
         if ((Kw / 32) % S)   // whole 128-byte chunks per slice
             continue;
-        if ((size_t)KS * B * 2 > SM_X_BUDGET)
+        if ((size_t)KS * B * 2 * (rot ? 2 : 1) > SM_X_BUDGET)
             continue;
         // ~32 KB of codes per tile; 16, 32 or 64 rows
         int TM = (int)(32768 / ((size_t)KS * bits / 8));
@@ -394,7 +456,7 @@ SmPlan plan_small(int N, int K, int bits, int B)
         const int nblk = SM_CW / (TM / 16);
         if (GS % nblk || GS / nblk < 1 || GS > 256 || GS % 8 || KS * bits / 32 / 32 > 256)
             continue;
-        const SmLayout L0 = sm_layout(KS, bits, B, TM, 0);
+        const SmLayout L0 = sm_layout(KS, bits, B, TM, 0, rot);
         const size_t budget = 227 * 1024;
         if (L0.total + 2 * L0.stage_bytes > budget)
             continue;
@@ -405,7 +467,7 @@ SmPlan plan_small(int N, int K, int bits, int B)
         p.TM = TM;
         p.NT = (B + 7) / 8;
         p.NS = NS;
-        p.smem = sm_layout(KS, bits, B, TM, NS).total;
+        p.smem = sm_layout(KS, bits, B, TM, NS, rot).total;
         const size_t tiles = (size_t)(N + TM - 1) / TM;
         if (tiles > (size_t)SM_MAX_TILES)
             return p;
@@ -419,23 +481,38 @@ SmPlan plan_small(int N, int K, int bits, int B)
     return p;
 }
 
-template <int BITS, int NT>
+template <int BITS, int NT, int FMT, bool ROT>
 cudaError_t launch_small_t(const SmArgs &a, const SmPlan &p, const LaunchCfg &c, const CUtensorMap &mc,
                            const CUtensorMap &ms, const CUtensorMap &mb)
 {
     cudaError_t e;
-    if ((e = set_smem(qgemm_small_kernel<BITS, NT>, p.smem)) != cudaSuccess)
+    if ((e = set_smem(qgemm_small_kernel<BITS, NT, FMT, ROT>, p.smem)) != cudaSuccess)
         return e;
     const int grid = (c.num_sms / p.S) * p.S;
-    return launch_ex(qgemm_small_kernel<BITS, NT>, dim3(grid), dim3(SM_THREADS), p.smem, c, 1, a, p.NS,
-                     mc, ms, mb);
+    return launch_ex(qgemm_small_kernel<BITS, NT, FMT, ROT>, dim3(grid), dim3(SM_THREADS), p.smem, c,
+                     1, a, p.NS, mc, ms, mb);
+}
+
+template <int FMT, bool ROT>
+cudaError_t launch_small_nt(int bits, const SmArgs &a, const SmPlan &p, const LaunchCfg &c,
+                            const CUtensorMap &mc, const CUtensorMap &ms, const CUtensorMap &mb)
+{
+    switch (bits * 10 + p.NT) {
+    case 42: return launch_small_t<4, 2, FMT, ROT>(a, p, c, mc, ms, mb);
+    case 43: return launch_small_t<4, 3, FMT, ROT>(a, p, c, mc, ms, mb);
+    case 44: return launch_small_t<4, 4, FMT, ROT>(a, p, c, mc, ms, mb);
+    case 82: return launch_small_t<8, 2, FMT, ROT>(a, p, c, mc, ms, mb);
+    case 83: return launch_small_t<8, 3, FMT, ROT>(a, p, c, mc, ms, mb);
+    case 84: return launch_small_t<8, 4, FMT, ROT>(a, p, c, mc, ms, mb);
+    }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-size_t qgemm_small_workspace_bytes(int N, int K, int bits, int B)
+size_t qgemm_small_workspace_bytes(int N, int K, int bits, int B, bool rot)
 {
-    const SmPlan p = plan_small(N, K, bits, B);
+    const SmPlan p = plan_small(N, K, bits, B, rot);
     return p.ok ? p.ws_bytes : 0;
 }
 
@@ -445,13 +522,18 @@ cudaError_t launch_qgemm_small(const QgemvArgs &a, void *ws, size_t ws_bytes, co
                                bool *used_ws)
 {
     *used_ws = false;
-    const SmPlan p = plan_small(a.N, a.K, a.bits, a.B);
-    // x is read with 16-byte loads; scales and biases by 2-D tensor copies
-    const bool align_ok =
-        ((reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.scales) |
-          reinterpret_cast<uintptr_t>(a.biases)) & 15u) == 0 &&
-        (a.K / kGroup * 2) % 16 == 0;
-    if (!p.ok || !align_ok || a.fmt != QG_AFFINE || a.signs)
+    const bool rot = a.signs != nullptr;
+    const SmPlan p = plan_small(a.N, a.K, a.bits, a.B, rot);
+    // x is read with 16-byte loads; scales and biases (or the parameter words)
+    // by 2-D tensor copies
+    const uintptr_t sb_addr = a.fmt == QG_AFFINE
+                                  ? (reinterpret_cast<uintptr_t>(a.scales) |
+                                     reinterpret_cast<uintptr_t>(a.biases))
+                                  : reinterpret_cast<uintptr_t>(a.params);
+    const int sb_row_bytes = a.K / kGroup * (a.fmt == QG_AFFINE ? 2 : 4);
+    const bool align_ok = ((reinterpret_cast<uintptr_t>(a.x) | sb_addr) & 15u) == 0 &&
+                          sb_row_bytes % 16 == 0;
+    if (!p.ok || !align_ok)
         return launch_qgemv_batched(a, c);
     const int per = c.num_sms / p.S, n_tiles = (a.N + p.TM - 1) / p.TM;
     if (per < 1 || (n_tiles + per - 1) / per > SM_MAX_CTA_TILES)
@@ -464,12 +546,17 @@ cudaError_t launch_qgemm_small(const QgemvArgs &a, void *ws, size_t ws_bytes, co
     memset(&mb, 0, sizeof(mb));
     const int Kw = a.K * a.bits / 32;
     const int G = a.K / kGroup;
-    if (!encode_codes_map(&mc, a.packed, a.N, Kw, p.TM, p.KS * a.bits / 32 / 32) ||
-        !encode_u16_map_2d(&ms, a.scales, a.N, G, p.KS / kGroup, p.TM) ||
-        !encode_u16_map_2d(&mb, a.biases, a.N, G, p.KS / kGroup, p.TM))
+    bool maps = encode_codes_map(&mc, a.packed, a.N, Kw, p.TM, p.KS * a.bits / 32 / 32);
+    if (a.fmt == QG_AFFINE)
+        maps = maps && encode_u16_map_2d(&ms, a.scales, a.N, G, p.KS / kGroup, p.TM) &&
+               encode_u16_map_2d(&mb, a.biases, a.N, G, p.KS / kGroup, p.TM);
+    else
+        maps = maps && encode_u32_map_2d(&ms, a.params, a.N, G, p.KS / kGroup, p.TM);
+    if (!maps)
         return launch_qgemv_batched(a, c);
     SmArgs s;
     s.x = a.x;
+    s.signs = a.signs;
     s.y = a.y;
     s.status = a.status;
     s.N = a.N;
@@ -481,13 +568,15 @@ cudaError_t launch_qgemm_small(const QgemvArgs &a, void *ws, size_t ws_bytes, co
     s.ctr = p.S > 1 ? static_cast<unsigned *>(ws) : nullptr;
     s.part = p.S > 1 ? reinterpret_cast<float4 *>(static_cast<unsigned char *>(ws) + SM_CTR_BYTES) : nullptr;
     *used_ws = p.S > 1;
-    switch (a.bits * 10 + p.NT) {
-    case 42: return launch_small_t<4, 2>(s, p, c, mc, ms, mb);
-    case 43: return launch_small_t<4, 3>(s, p, c, mc, ms, mb);
-    case 44: return launch_small_t<4, 4>(s, p, c, mc, ms, mb);
-    case 82: return launch_small_t<8, 2>(s, p, c, mc, ms, mb);
-    case 83: return launch_small_t<8, 3>(s, p, c, mc, ms, mb);
-    case 84: return launch_small_t<8, 4>(s, p, c, mc, ms, mb);
+    switch (a.fmt) {
+    case QG_AFFINE:
+        return launch_small_nt<QG_AFFINE, false>(a.bits, s, p, c, mc, ms, mb);
+    case QG_ZP4:
+        return rot ? launch_small_nt<QG_ZP4, true>(4, s, p, c, mc, ms, mb)
+                   : launch_small_nt<QG_ZP4, false>(4, s, p, c, mc, ms, mb);
+    case QG_SYM8:
+        return rot ? launch_small_nt<QG_SYM8, true>(8, s, p, c, mc, ms, mb)
+                   : launch_small_nt<QG_SYM8, false>(8, s, p, c, mc, ms, mb);
     }
     return cudaErrorInvalidValue;
 }

@@ -30,6 +30,8 @@ namespace qmoe {
 namespace {
 
 constexpr int QG_CW = 16;                     // consumer warps
+constexpr int QG_GW = 4;                      // warps per consumer group (one tile at a time)
+constexpr int QG_GROUPS = QG_CW / QG_GW;
 constexpr int QG_CT = QG_CW * 32;             // consumer threads
 constexpr int QG_THREADS = QG_CT + 32;        // + one producer warp
 constexpr int QG_MAX_STAGES = 8;
@@ -72,15 +74,6 @@ __host__ __device__ inline QgLayout qg_layout(int K, int bits, int ncol, int NS,
     return L;
 }
 
-// scale and folded-bias factor of one parameter word of the bf16 formats:
-// ZP4 w = s(q - z) -> (s, -s z); SYM8 w = s(q' - 128) with q' = q + 128 -> (s, -128 s)
-template <int FMT>
-__device__ __forceinline__ void fmt_scale_bias(uint32_t p, float &s, float &b)
-{
-    s = __uint_as_float(p << 16);
-    b = FMT == QG_ZP4 ? -s * (float)((p >> 16) & 0xFFu) : -128.f * s;
-}
-
 template <int BITS, bool SWZ, int FMT, bool ROT>
 __global__ void __launch_bounds__(QG_THREADS, 1)
     qgemv_kernel(QgemvArgs a, int NS, const __grid_constant__ CUtensorMap codes_map)
@@ -102,7 +95,7 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], QG_CW);
+            mbar_init(&empty[s], QG_GW);   // the warps of the group that reads it
         }
         mbar_init_fence();
     }
@@ -173,15 +166,21 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                       ctid, QG_CT);
     named_bar_sync(1, QG_CT);
 
-    // this warp's groups: a contiguous block, so that with G % 64 == 0 the
-    // scales and biases of a row come as one 8-byte load per 4 groups
-    const int gpw = (L.G + QG_CW - 1) / QG_CW;
-    const int g0 = min(L.G, warp * gpw), g1 = min(L.G, g0 + gpw);
+    // Tiles go to groups of QG_GW warps in turn (tile k of this CTA to group
+    // k % QG_GROUPS), so a slow warp holds up its own group only; the warps of
+    // a group split the tile's 64-input groups into contiguous blocks, so
+    // that with G % 64 == 0 a row's scales and biases come as one 8-byte load
+    // per 4 groups.
+    const int grp = warp / QG_GW, wg = warp % QG_GW;
+    const int gpw = (L.G + QG_GW - 1) / QG_GW;
+    const int g0 = min(L.G, wg * gpw), g1 = min(L.G, g0 + gpw);
     const bool vec_sb = (L.G & 63) == 0;
     const int gid = lane >> 2, tig = lane & 3;
     bool failed = false;
     int k = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
+        if (k % QG_GROUPS != grp)
+            continue;   // another group's tile
         const int st = k % NS, use = k / NS;
         if (!failed && !mbar_wait(&full[st], use & 1, a.status))
             failed = true;
@@ -320,12 +319,16 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&empty[st]);
-        red[((k & 1) * QG_CW + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        named_bar_sync(1, QG_CT);
-        if (warp == k % QG_CW) {
+        // partials of the group's warps; two buffers alternate between the
+        // group's tiles, so a warp that runs ahead cannot overwrite the ones
+        // the first warp is still adding
+        const int par = (k / QG_GROUPS) & 1;
+        red[(par * QG_CW + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        named_bar_sync(2 + grp, QG_GW * 32);
+        if (wg == 0) {
             float v[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int w = 0; w < QG_CW; ++w) {
-                const float4 p = red[((k & 1) * QG_CW + w) * 32 + lane];
+            for (int w = 0; w < QG_GW; ++w) {
+                const float4 p = red[(par * QG_CW + grp * QG_GW + w) * 32 + lane];
                 v[0] += p.x;
                 v[1] += p.y;
                 v[2] += p.z;
@@ -445,6 +448,22 @@ bool encode_u16_map_2d(CUtensorMap *m, const void *base, long rows, int cols, in
     const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_u32_map_2d(CUtensorMap *m, const void *base, long rows, int cols, int box_cols,
+                       int box_rows)
+{
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn || (reinterpret_cast<uintptr_t>(base) & 15u) || (cols * 4) % 16 || (box_cols * 4) % 16 ||
+        box_cols < 1 || box_cols > 256 || box_cols > cols || box_rows < 1 || box_rows > 256)
+        return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+    const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -57,6 +57,8 @@ def lib():
             "moe_expert_qmlp_ep": [p, p, p, p, i32, i32, i32, p, p, sz, p, p],
             "qmoe_f32_to_f16": [p, p, ctypes.c_int64, p],
             "qgemv_fmt": [p, p, i32, p, p, p],
+            "qgemv_fmt_workspace_bytes": [i32, i32, i32, i32, i32],
+            "qgemv_fmt_ws": [p, p, i32, p, p, sz, p, p],
             "moe_router_topk": [p, p, i32, i32, p, p, p, p, p],
             "moe_expert_workspace_bytes": [p, i32],
             "moe_expert_qmlp": [p, p, p, p, i32, p, p, sz, p, p],
@@ -74,6 +76,8 @@ def lib():
             "qmoe_check_status": [p, p, p],
             "qmoe_status_string": [ctypes.c_int],
             "qmoe_set_dependent_launch": [i32],
+            "qmoe_set_prefill_tensor_min": [i32],
+            "qmoe_set_decode_wait_limit_ns": [ctypes.c_uint64],
             "qmoe_version": [],
             "qmoe_lfu_create": [i32, p],
             "qmoe_lfu_destroy": [p],
@@ -90,12 +94,15 @@ def lib():
             fn.restype = ctypes.c_int
         L.moe_expert_workspace_bytes.restype = sz
         L.qgemv_affine_workspace_bytes.restype = sz
+        L.qgemv_fmt_workspace_bytes.restype = sz
         L.moe_prefill_workspace_bytes.restype = sz
         L.moe_decode_workspace_bytes.restype = sz
         L.moe_decode_pack_bytes.restype = sz
         L.qmoe_status_string.restype = ctypes.c_char_p
         L.qmoe_version.restype = i32
         L.qmoe_set_dependent_launch.restype = i32
+        L.qmoe_set_prefill_tensor_min.restype = i32
+        L.qmoe_set_decode_wait_limit_ns.restype = ctypes.c_uint64
         L.qmoe_lfu_destroy.restype = None
         L.qmoe_cache_destroy.restype = None
         L.qmoe_lfu_plan.restype = i32
@@ -430,16 +437,31 @@ def qgemv_affine(W, x, y=None, status=None, one_pass=True, workspace=None):
     return y
 
 
-def qgemv_fmt(W, x, y=None, status=None):
+def qgemv_fmt(W, x, y=None, status=None, one_pass=True, workspace=None):
     """y[b] = W (R x[b]) (R the rotation when W has signs) for x [B][K]
-    float16 (B <= 32), W a QMatrixFmt.  Returns y [B][N] float16."""
+    float16 (B <= 32), W a QMatrixFmt.  Returns y [B][N] float16.  A batch
+    of 9..32 runs in one pass over the weights (qgemv_fmt_ws) where the shape
+    allows it (workspace as qgemv_affine); one_pass=False runs one launch per
+    8 rows."""
     x = _need(x, torch.float16, "x")
     x2 = x.reshape(-1, W.cols)
+    B = x2.shape[0]
     if y is None:
-        y = torch.empty(x2.shape[0], W.rows, dtype=torch.float16, device=x.device)
-    _need(y, torch.float16, "y", (x2.shape[0], W.rows))
-    _check(lib().qgemv_fmt(ctypes.byref(W.c), _ptr(x2), x2.shape[0], _ptr(y), _ptr(status),
-                           _stream()), "qgemv_fmt")
+        y = torch.empty(B, W.rows, dtype=torch.float16, device=x.device)
+    _need(y, torch.float16, "y", (B, W.rows))
+    rotated = 1 if W.c.rht_signs else 0
+    need = (lib().qgemv_fmt_workspace_bytes(W.rows, W.cols, W.c.format, rotated, B)
+            if one_pass and B > 8 else 0)
+    if one_pass and B > 8:
+        ws = None
+        if need:
+            ws = workspace if workspace is not None else _shared_workspace(need, x.device)
+        _check(lib().qgemv_fmt_ws(ctypes.byref(W.c), _ptr(x2), B, _ptr(y), _ptr(ws),
+                                  0 if ws is None else ws.numel() * ws.element_size(),
+                                  _ptr(status), _stream()), "qgemv_fmt_ws")
+    else:
+        _check(lib().qgemv_fmt(ctypes.byref(W.c), _ptr(x2), B, _ptr(y), _ptr(status), _stream()),
+               "qgemv_fmt")
     return y
 
 
@@ -620,6 +642,22 @@ def qmoe_check_status(status=None):
 
 def qmoe_set_dependent_launch(enable):
     return bool(lib().qmoe_set_dependent_launch(1 if enable else 0))
+
+
+def qmoe_set_decode_wait_limit_ns(ns):
+    """Limit of every wait inside the fused decode (0: the default 2 s).
+    Returns the previous setting."""
+    return int(lib().qmoe_set_decode_wait_limit_ns(int(ns)))
+
+
+# the library's threshold when the tensor-core prefill path is on
+TENSOR_MIN_DEFAULT = 16
+
+
+def qmoe_set_prefill_tensor_min(min_tokens):
+    """Experts of a prefill chunk with at least min_tokens tokens run on the
+    tensor-core kernels (0: none).  Returns the previous setting."""
+    return int(lib().qmoe_set_prefill_tensor_min(int(min_tokens)))
 
 
 def qmoe_version():

@@ -49,3 +49,18 @@ def assert_close_rows(y, ref, tol=REL_TOL, what=""):
     for i in range(y.shape[0]):
         assert_close(y[i], ref[i], tol, "%s, row %d" % (what, i))
 
+
+
+def assert_close_f16(y16, ref64, ref16, tol=REL_TOL, what=""):
+    """An fp16 output against the oracle where some outputs exceed the fp16
+    range: +-inf exactly where the oracle's own fp16 rounding (ref16, bit
+    patterns) gives +-inf, the finite outputs within the tolerance on the
+    scale of the finite reference values."""
+    y = np.asarray(y16, dtype=np.float16).astype(np.float64)
+    want = np.asarray(ref16, dtype=np.uint16).view(np.float16).astype(np.float64)
+    inf = np.isinf(want)
+    assert np.array_equal(np.isinf(y), inf), "%s: infinities differ from the oracle's" % what
+    assert np.array_equal(np.sign(y[inf]), np.sign(want[inf])), "%s: signs of inf" % what
+    fin = ~inf
+    if fin.any():
+        assert_close(y[fin], np.asarray(ref64)[fin], tol, what)

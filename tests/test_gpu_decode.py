@@ -7,7 +7,7 @@ import torch
 
 import oracle
 from moe_expert_gemv_b200 import qmoe, synth
-from tests._util import REL_TOL, assert_close, f16_bits
+from tests._util import REL_TOL, assert_close, assert_close_f16, f16_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -27,9 +27,11 @@ def check_layers(ms, E, H, I, k, x16, y, idx, wt, lg, layers=None):
         assert np.array_equal(idx[l], sidx[0]), "layer %d: selection on device logits" % l
         assert_close(wt[l], swt[0], what="layer %d weights" % l)
         assert np.array_equal(idx[l], oidx[0]), "layer %d: indices differ from the fp64 oracle" % l
-        y64, _ = oracle.Layer(m, E, H, I).moe(x16[l:l + 1], idx[l:l + 1],
-                                              wt[l:l + 1].astype(np.float64))
-        assert_close(y[l].view(np.float16), y64[0], what="layer %d output" % l)
+        y64, y16o = oracle.Layer(m, E, H, I).moe(x16[l:l + 1], idx[l:l + 1],
+                                                 wt[l:l + 1].astype(np.float64))
+        # (a layer whose outputs leave the fp16 range must give +-inf exactly
+        # where the oracle's fp16 rounding does)
+        assert_close_f16(y[l].view(np.float16), y64[0], y16o[0], what="layer %d output" % l)
 
 
 def run(stack, x16, E, k):
@@ -59,11 +61,14 @@ def test_moe_e128_three_layers_and_repeat(cuda_dev):
     x16 = np.concatenate([synth.activations(3, 1, H, layer=l) for l in range(3)])
     y, idx, wt, lg = run(stack, x16, E, k)
     check_layers(ms, E, H, I, k, x16, y, idx, wt, lg)
-    # the workspace is back to zero and a second call reproduces every bit
-    assert torch.count_nonzero(stack.workspace[:16]) == 0
+    # the workspace is back to zero; a second call reproduces the routing bit
+    # for bit and the outputs within the tolerance (the cross-cluster fp32
+    # sums of a layer output are atomic, so their order may change the last
+    # bits)
+    assert torch.count_nonzero(stack.workspace) == 0
     y2, idx2, wt2, lg2 = run(stack, x16, E, k)
-    assert np.array_equal(y, y2) and np.array_equal(idx, idx2)
-    assert np.array_equal(wt, wt2) and np.array_equal(lg, lg2)
+    assert np.array_equal(idx, idx2) and np.array_equal(wt, wt2) and np.array_equal(lg, lg2)
+    check_layers(ms, E, H, I, k, x16, y2, idx2, wt2, lg2)
 
 
 def test_matches_unfused_path(cuda_dev):
@@ -84,40 +89,55 @@ def test_matches_unfused_path(cuda_dev):
 
 
 @pytest.mark.slow
-def test_moe_e128_thirty_layers_sampled(cuda_dev):
-    """The full decode step: 30 layers, 12.96 GB of weights; every layer's
-    routing is checked, outputs of a sample of layers against the oracle."""
+def test_moe_e128_thirty_layers_all(cuda_dev):
+    """The full decode step: 30 layers, 12.96 GB of weights, one launch.
+    Every layer's routing and output is checked against the oracle; the host
+    keeps only the routers while the stack is on the device and regenerates
+    each layer from its seed for the oracle afterwards."""
     E, H, I, k, n = synth.MOE_E, synth.MOE_H, synth.MOE_I, synth.MOE_TOPK, synth.MOE_LAYERS
-    layers, ms = [], []
+    layers, routers = [], []
     for l in range(n):
         m = synth.moe_layer(0, l)
         layers.append(qmoe.MoELayer.from_numpy(m, E, H, I))
-        ms.append({"router": m["router"]} if l not in (0, 13, 29) else m)
+        routers.append({"router": m["router"]})
+        del m
     stack = qmoe.DecodeStack(layers, k)
     x16 = np.concatenate([synth.activations(0, 1, H, layer=l) for l in range(n)])
     y, idx, wt, lg = run(stack, x16, E, k)
+    del stack, layers
     for l in range(n):
-        l64, oidx, _ = oracle.router(*ms[l]["router"], E, H, 8, x16[l:l + 1], k)
-        assert np.array_equal(idx[l], oidx[0])
-    check_layers(ms, E, H, I, k, x16, y, idx, wt, lg, layers=(0, 13, 29))
+        m = synth.moe_layer(0, l)
+        ms = [None] * n
+        ms[l] = m
+        check_layers(ms, E, H, I, k, x16, y, idx, wt, lg, layers=(l,))
 
 
 def expected_pack(m, E, H, I):
     """The packed streaming layout, rebuilt with numpy from the row-major
-    arrays (bytes)."""
-    GH, GI = H // 64, I // 64
+    arrays (bytes): 8 router blocks of E/8 rows, then per expert (the shared
+    expert last), per group g of 64 intermediate indices and per cluster rank
+    r: gate rows 64g+8r..+7, the same up rows, and down rows H/8*r..+H/8-1
+    restricted to inputs 64g..64g+63; codes of 16-byte chunk c of row i of a
+    gate/up/router block at chunk (c & ~7) | ((c ^ i) & 7)."""
+    GH, GI, Rr, Hc = H // 64, I // 64, E // 8, H // 8
     out = []
+    sb = lambda S, B: np.stack([S, B], axis=-1).astype(np.uint16).view(np.uint8).reshape(-1)
+
+    def swizzled(codes):
+        rows, nb = codes.shape
+        ch = codes.reshape(rows, nb // 16, 16)
+        res = np.empty_like(ch)
+        for i in range(rows):
+            for c in range(nb // 16):
+                res[i, (c & ~7) | ((c ^ i) & 7)] = ch[i, c]
+        return res.reshape(-1)
+
     rP = m["router"][0].view(np.uint8).reshape(E, H)
     rS, rB = m["router"][1].reshape(E, GH), m["router"][2].reshape(E, GH)
-    sb = lambda S, B: np.stack([S, B], axis=-1).astype(np.uint16).view(np.uint8).reshape(-1)
-    for rb in range(E // 8):
-        for kh in range(2):
-            codes = rP[rb * 8:rb * 8 + 8, kh * H // 2:(kh + 1) * H // 2].reshape(8, H // 32, 16)
-            perm = np.array([[c ^ (4 * (r & 1)) for c in range(H // 32)] for r in range(8)])
-            codes = np.stack([codes[r][perm[r]] for r in range(8)])
-            rows = slice(rb * 8, rb * 8 + 8)
-            half = slice(kh * GH // 2, (kh + 1) * GH // 2)
-            out += [codes.reshape(-1), sb(rS[rows, half], rB[rows, half])]
+    for r in range(8):
+        rows = slice(Rr * r, Rr * r + Rr)
+        out += [swizzled(rP[rows]), sb(rS[rows], rB[rows])]
+
     def mat(name, e, rows_n, cols):
         P, S, B = m[name]
         P = P.reshape(-1, rows_n, cols // 8)[e if P.ndim == 3 else 0]
@@ -125,19 +145,17 @@ def expected_pack(m, E, H, I):
         Bb = B.reshape(-1, rows_n, cols // 64)[e if B.ndim == 3 else 0]
         return P.view(np.uint8).reshape(rows_n, cols // 2), S, Bb
     for e in range(E + 1):
-        g, u, d = ("gate", "up", "down") if e < E else ("sh_gate", "sh_up", "sh_down")
-        gP, gS, gB = mat(g, e, I, H)
-        uP, uS, uB = mat(u, e, I, H)
-        dP, dS, dB = mat(d, e, H, I)
-        for o in range(I // 4):
-            r = slice(4 * o, 4 * o + 4)
-            codes = np.concatenate([gP[r], uP[r]]).reshape(8, H // 32, 16)
-            perm = np.array([[c ^ (2 * (rr & 3)) for c in range(H // 32)] for rr in range(8)])
-            codes = np.stack([codes[rr][perm[rr]] for rr in range(8)])
-            out += [codes.reshape(-1), sb(np.concatenate([gS[r], uS[r]]), np.concatenate([gB[r], uB[r]]))]
-        for t in range(H // 32):
-            r = slice(32 * t, 32 * t + 32)
-            out += [dP[r].reshape(-1), sb(dS[r], dB[r])]
+        g_, u_, d_ = ("gate", "up", "down") if e < E else ("sh_gate", "sh_up", "sh_down")
+        gP, gS, gB = mat(g_, e, I, H)
+        uP, uS, uB = mat(u_, e, I, H)
+        dP, dS, dB = mat(d_, e, H, I)
+        for g in range(GI):
+            for r in range(8):
+                rows = slice(64 * g + 8 * r, 64 * g + 8 * r + 8)
+                out += [swizzled(gP[rows]), sb(gS[rows], gB[rows])]
+                out += [swizzled(uP[rows]), sb(uS[rows], uB[rows])]
+                dr = slice(Hc * r, Hc * r + Hc)
+                out += [dP[dr, 32 * g:32 * g + 32].reshape(-1), sb(dS[dr, g], dB[dr, g])]
     return np.concatenate(out)
 
 

@@ -68,28 +68,33 @@ def chunk128():
 
 
 @pytest.mark.slow
-def test_chunk128_chunk_sampled_tokens(cuda_dev, chunk128):
-    """The 128-token chunk with Zipf(1.1) routing; every output of a sample of
-    32 tokens (spread over the chunk) against the oracle."""
+def test_chunk128_every_token(cuda_dev, chunk128):
+    """The 128-token chunk with Zipf(1.1) routing: every output of every token
+    against the oracle, each token on its own scale (and the chunk as a
+    whole)."""
     m, G, idx, wt, x16 = chunk128
     E, H, I = synth.MOE_E, synth.MOE_H, synth.MOE_I
     y, flags = run_prefill(G, x16, idx, wt)
     assert flags == 0
-    rows = np.unique(np.concatenate([np.arange(0, 128, 5), [127]]))[:32]
-    y64, _ = oracle.Layer(m, E, H, I).moe(x16[rows], idx[rows], wt[rows].astype(np.float64))
-    assert_close(y.view(np.float16)[rows], y64, what="128-token chunk sampled tokens")
+    y64, _ = oracle.Layer(m, E, H, I).moe(x16, idx, wt.astype(np.float64))
+    yv = y.view(np.float16)
+    assert_close(yv, y64, what="128-token chunk")
+    for t in range(synth.PREFILL_T):
+        assert_close(yv[t], y64[t], what="128-token chunk, token %d" % t)
 
 
-def test_chunk128_rows_equal_decode_layer(cuda_dev, chunk128):
-    """Row t of the chunk = the decode layer on token t with the same routing
-    (two independent device paths)."""
+def test_decode_layer_on_chunk_tokens_matches_oracle(cuda_dev, chunk128):
+    """The per-token decode layer (moe_expert_qmlp) on tokens of the chunk,
+    with the chunk's routing, against the oracle."""
     m, G, idx, wt, x16 = chunk128
-    y, _ = run_prefill(G, x16, idx, wt)
+    E, H, I = synth.MOE_E, synth.MOE_H, synth.MOE_I
+    L = oracle.Layer(m, E, H, I)
     for t in (0, 63, 127):
         yd = qmoe.moe_expert_qmlp(G, dev(x16[t].view(np.float16), np.float16), dev(idx[t], np.int32),
                                   dev(wt[t], np.float32))
-        assert_close(y.view(np.float16)[t], f16_bits(yd).view(np.float16).astype(np.float64),
-                     what="row %d vs decode" % t)
+        assert qmoe.qmoe_check_status() == 0
+        y64, _ = L.moe(x16[t:t + 1], idx[t:t + 1], wt[t:t + 1].astype(np.float64))
+        assert_close(f16_bits(yd).view(np.float16), y64[0], what="decode layer, token %d" % t)
 
 
 def test_bad_expert_ids_flagged(cuda_dev):

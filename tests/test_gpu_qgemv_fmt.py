@@ -88,3 +88,29 @@ def test_bad_format_and_alignment_rejected(cuda_dev):
     x = buf[1:].view(1, K)   # 2-byte aligned only: the rotation needs 16-byte aligned x
     with pytest.raises(qmoe.QmoeError):
         qmoe.qgemv_fmt(W, x)
+
+
+@pytest.mark.parametrize("fmt", [qmoe.FMT_ZP4_BF16, qmoe.FMT_SYM8_BF16])
+@pytest.mark.parametrize("rotate", [False, True])
+@pytest.mark.parametrize("N,K,Bt", [(256, 4096, 9), (200, 2048, 16), (1000, 4096, 29),
+                                    (512, 8192, 32)])
+def test_small_m_one_pass(cuda_dev, fmt, rotate, N, K, Bt):
+    """Batch 9..32 of the format variants in one pass over the weights
+    (qgemv_fmt_ws; K split into slices whose x, or rotated x hi/lo pair,
+    fits on chip): every row against the oracle, and the 8-row-slice path
+    on the same inputs agrees within the tolerance."""
+    P, params, signs = synth.qmatrix_fmt(synth.rng(N, K, fmt, Bt, 31), N, K, fmt)
+    x16 = synth.activations(N + Bt + 7 * fmt, Bt, K)
+    W = qmoe.QMatrixFmt.from_numpy(P, params, signs, N, K, fmt, rotate=rotate)
+    xd = torch.from_numpy(x16.view(np.float16).copy()).cuda()
+    need = qmoe.lib().qgemv_fmt_workspace_bytes(N, K, fmt, int(rotate), Bt)
+    ws = torch.zeros(max(need, 16), dtype=torch.uint8, device="cuda")
+    y1 = qmoe.qgemv_fmt(W, xd, workspace=ws)
+    assert qmoe.qmoe_check_status() == 0
+    y0 = qmoe.qgemv_fmt(W, xd, one_pass=False)
+    y64, _ = oracle.qgemv_fmt(P, params, N, K, fmt, x16, signs, rotate)
+    what = "one-pass fmt %d rot %d N=%d K=%d B=%d" % (fmt, rotate, N, K, Bt)
+    assert_close_rows(y1.cpu().numpy(), y64, what=what)
+    assert_close_rows(y1.cpu().numpy(), y0.cpu().numpy().astype(np.float64), what=what + " vs slices")
+    if need:   # the workspace's counters are back at zero
+        assert torch.count_nonzero(ws[:65536]) == 0
