@@ -343,15 +343,14 @@ def run_decode(args, dist):
             g_unfused.replay()
         unfused_ms = timed_replays(g_unfused.replay, reps) / reps
 
-        # end to end through host buffers: H2D of every layer's input token,
-        # the step, D2H of every layer's output, each step
+        # end to end through host buffers with the C call that takes them
+        # (moe_decode_layers_host): H2D of every layer's input token, the
+        # step, D2H of every layer's output, each step
         x_host = x.cpu().pin_memory()
         y_host = torch.empty_like(y, device="cpu").pin_memory()
 
         def e2e_step():
-            x.copy_(x_host, non_blocking=True)
-            fused_step()
-            y_host.copy_(y, non_blocking=True)
+            qmoe.moe_decode_layers_host(stack, x_host, y_host, x, y)
 
         for _ in range(3):
             e2e_step()

@@ -355,6 +355,19 @@ qmoe_status moe_decode_layers(const void *const *packed_layers, int32_t n_layers
                               float *weights, float *logits, void *workspace,
                               size_t workspace_bytes, int32_t *status_dev, void *stream);
 
+/* moe_decode_layers from HOST buffers: x_host -> x_dev (cudaMemcpyAsync), the
+ * fused decode, y_dev -> y_host, all enqueued on `stream` in that order (the
+ * call returns at once; synchronise the stream before reading y_host).
+ * x_host, y_host: fp16 [n_layers][hidden] in host memory (pinned memory lets
+ * the copies run asynchronously); x_dev (16-byte aligned), y_dev: device
+ * staging buffers of the same size owned by the caller -- the library still
+ * allocates nothing.  Checks as moe_decode_layers, made before any copy. */
+qmoe_status moe_decode_layers_host(const void *const *packed_layers, int32_t n_layers,
+                                   int32_t num_experts, int32_t hidden, int32_t inter,
+                                   const uint16_t *x_host, uint16_t *y_host, int32_t top_k,
+                                   uint16_t *x_dev, uint16_t *y_dev, void *workspace,
+                                   size_t workspace_bytes, int32_t *status_dev, void *stream);
+
 /* ---------------------------------------------------------------------------
  * Host-memory expert streaming through a per-layer LFU cache (TurboFieldfare
  * article, "내부 구조" section: the CPU takes the router's top-8 ids, plans

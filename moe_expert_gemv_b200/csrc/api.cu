@@ -573,11 +573,13 @@ size_t moe_decode_workspace_bytes(int32_t num_experts, int32_t hidden, int32_t i
     return decode_workspace_layout(num_experts, hidden, inter, top_k, nullptr, nullptr);
 }
 
-qmoe_status moe_decode_layers(const void *const *packed_layers, int32_t n_layers,
-                              int32_t num_experts, int32_t hidden, int32_t inter,
-                              const uint16_t *x, int32_t top_k, uint16_t *y, int32_t *idx,
-                              float *weights, float *logits, void *workspace,
-                              size_t workspace_bytes, int32_t *status_dev, void *stream)
+// every check of moe_decode_layers, before anything is enqueued
+static qmoe_status decode_validate(const void *const *packed_layers, int32_t n_layers,
+                                   int32_t num_experts, int32_t hidden, int32_t inter,
+                                   const uint16_t *x, int32_t top_k, const uint16_t *y,
+                                   const int32_t *idx, const float *weights, const float *logits,
+                                   const void *workspace, size_t workspace_bytes,
+                                   const int32_t *status_dev)
 {
     if (!packed_layers || !x || !y || n_layers < 1)
         return QMOE_ERR_INVALID_ARG;
@@ -605,7 +607,21 @@ qmoe_status moe_decode_layers(const void *const *packed_layers, int32_t n_layers
     if (workspace_bytes < moe_decode_workspace_bytes(num_experts, hidden, inter, top_k))
         return QMOE_ERR_WORKSPACE;
     DevState *d;
-    qmoe_status s;
+    return device_state(&d);
+}
+
+qmoe_status moe_decode_layers(const void *const *packed_layers, int32_t n_layers,
+                              int32_t num_experts, int32_t hidden, int32_t inter,
+                              const uint16_t *x, int32_t top_k, uint16_t *y, int32_t *idx,
+                              float *weights, float *logits, void *workspace,
+                              size_t workspace_bytes, int32_t *status_dev, void *stream)
+{
+    qmoe_status s = decode_validate(packed_layers, n_layers, num_experts, hidden, inter, x, top_k,
+                                    y, idx, weights, logits, workspace, workspace_bytes,
+                                    status_dev);
+    if (s != QMOE_OK)
+        return s;
+    DevState *d;
     if ((s = device_state(&d)) != QMOE_OK)
         return s;
     const LaunchCfg c = launch_cfg(d, stream);
@@ -631,6 +647,33 @@ qmoe_status moe_decode_layers(const void *const *packed_layers, int32_t n_layers
         if ((s = cuda_status(launch_decode(a, c))) != QMOE_OK)
             return s;
     }
+    return QMOE_OK;
+}
+
+qmoe_status moe_decode_layers_host(const void *const *packed_layers, int32_t n_layers,
+                                   int32_t num_experts, int32_t hidden, int32_t inter,
+                                   const uint16_t *x_host, uint16_t *y_host, int32_t top_k,
+                                   uint16_t *x_dev, uint16_t *y_dev, void *workspace,
+                                   size_t workspace_bytes, int32_t *status_dev, void *stream)
+{
+    if (!x_host || !y_host)
+        return QMOE_ERR_INVALID_ARG;
+    // every check of the decode first: a rejected call copies nothing
+    qmoe_status s = decode_validate(packed_layers, n_layers, num_experts, hidden, inter, x_dev,
+                                    top_k, y_dev, nullptr, nullptr, nullptr, workspace,
+                                    workspace_bytes, status_dev);
+    if (s != QMOE_OK)
+        return s;
+    const size_t bytes = (size_t)n_layers * hidden * 2;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return QMOE_ERR_CUDA;
+    if ((s = moe_decode_layers(packed_layers, n_layers, num_experts, hidden, inter, x_dev, top_k,
+                               y_dev, nullptr, nullptr, nullptr, workspace, workspace_bytes,
+                               status_dev, stream)) != QMOE_OK)
+        return s;
+    if (cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return QMOE_ERR_CUDA;
     return QMOE_OK;
 }
 

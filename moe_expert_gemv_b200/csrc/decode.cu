@@ -569,8 +569,9 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
         int gu_buf = 0;
         auto do_gu = [&](int seq0, int slot, int l) {
             const int sa = seq0 % NS, sb = (seq0 + 1) % NS;
-            bool good = ok && wait_bar(a, &full[sa], (seq0 / NS) & 1) &&
-                        wait_bar(a, &full[sb], ((seq0 + 1) / NS) & 1);
+            // the lanes of a warp decide together: the mma below is warp-collective
+            const bool good = __all_sync(0xffffffffu, ok && wait_bar(a, &full[sa], (seq0 / NS) & 1) &&
+                                                          wait_bar(a, &full[sb], ((seq0 + 1) / NS) & 1));
             float ag = 0.f, au = 0.f, bg = 0.f, bu = 0.f;
             if (good) {
                 const unsigned char *A = ring + (size_t)sa * P.st_bytes;
@@ -664,11 +665,12 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
         // ---------------------------------------- one down work item
         auto do_dn = [&](int seq, int slot, int j, int l) {
             const int st = seq % NS;
-            bool good = ok && wait_bar(a, &full[st], (seq / NS) & 1) &&
-                        wait_bar_cluster(a, &hbar[slot], l & 1);
+            // the lanes of a warp decide together: the mma below is warp-collective
+            bool good = __all_sync(0xffffffffu, ok && wait_bar(a, &full[st], (seq / NS) & 1) &&
+                                                    wait_bar_cluster(a, &hbar[slot], l & 1));
             float w = 1.f;
             if (good && j < K) {
-                good = wait_bar(a, topk_bar, l & 1);
+                good = __all_sync(0xffffffffu, wait_bar(a, topk_bar, l & 1));
                 w = s_wt[j];
             }
             if (good) {
@@ -730,7 +732,7 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
             }
             // ---- router: this CTA's Rr rows, K split over the 16 warps
             {
-                const bool good = ok && wait_bar(a, rfull, l & 1);
+                const bool good = __all_sync(0xffffffffu, ok && wait_bar(a, rfull, l & 1));
                 float acc_lo = 0.f, acc_hi = 0.f, b_lo = 0.f, b_hi = 0.f;
                 if (good) {
                     const int ra = gid % Rr, rb = (gid + 8) % Rr;

@@ -222,6 +222,8 @@ __global__ void __launch_bounds__(GU_THREADS, 1) expert_gateup_kernel(ExpertArgs
         const int st = k % GU_STAGES, use = k / GU_STAGES;
         if (!failed && !mbar_wait(&full[st], use & 1, a.status))
             failed = true;
+        // the lanes of a warp decide together: the mma below is warp-collective
+        failed = __any_sync(0xffffffffu, failed);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         if (!failed) {
             const unsigned char *stage = smem + L.stage_off + (size_t)st * L.stage_bytes;
@@ -402,6 +404,8 @@ __global__ void __launch_bounds__(DN_THREADS, 1) expert_down_kernel(ExpertArgs a
         const int st = k % NS, use = k / NS;
         if (!failed && !mbar_wait(&full[st], use & 1, a.status))
             failed = true;
+        // the lanes of a warp decide together: the mma below is warp-collective
+        failed = __any_sync(0xffffffffu, failed);
         const int so = item / tiles, tile = item % tiles;
         const int slot = so == 0 ? a.top_k : so - 1;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};

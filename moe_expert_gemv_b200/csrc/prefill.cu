@@ -507,7 +507,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     int k = 0;
     for (int q = 0;; ++q) {
         const int b = q & 1;
-        if (!pf_wait(&afull[b], (q >> 1) & 1, a.status, abort_word))
+        // every decision below is taken by whole warps (the mma is warp-collective)
+        if (!__all_sync(0xffffffffu, pf_wait(&afull[b], (q >> 1) & 1, a.status, abort_word)))
             break;
         const int u = s_unit[b];
         if (u < 0)
@@ -520,8 +521,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         const float *xsm = reinterpret_cast<const float *>(act + (size_t)TILE_T * d.xg_stride * 16);
         if (warp < nsub) {
             const int kk = k + warp, slot = kk % NS;
-            if (pf_wait_seq(s_unit + 4 + slot, kk, a.status, abort_word) &&
-                pf_wait(&full[slot], (kk / NS) & 1, a.status, abort_word)) {
+            if (__all_sync(0xffffffffu, pf_wait_seq(s_unit + 4 + slot, kk, a.status, abort_word) &&
+                                            pf_wait(&full[slot], (kk / NS) & 1, a.status, abort_word))) {
                 const unsigned char *stage = smem + L.stage_off + (size_t)slot * st.bytes;
                 const unsigned char *gt = stage, *utl = stage + st.codes;
                 const __half *gs = reinterpret_cast<const __half *>(stage + 2 * st.codes);
@@ -707,7 +708,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     int k = 0;
     for (int q = 0;; ++q) {
         const int b = q & 1;
-        if (!pf_wait(&afull[b], (q >> 1) & 1, a.status, abort_word))
+        // every decision below is taken by whole warps (the mma is warp-collective)
+        if (!__all_sync(0xffffffffu, pf_wait(&afull[b], (q >> 1) & 1, a.status, abort_word)))
             break;
         const int u = s_unit[b];
         if (u < 0)
@@ -720,8 +722,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         const float *hsm = reinterpret_cast<const float *>(act + (size_t)TILE_T * d.hf_stride * 16);
         if (warp < nsub) {
             const int kk = k + warp, slot = kk % NS;
-            if (pf_wait_seq(s_unit + 4 + slot, kk, a.status, abort_word) &&
-                pf_wait(&full[slot], (kk / NS) & 1, a.status, abort_word)) {
+            if (__all_sync(0xffffffffu, pf_wait_seq(s_unit + 4 + slot, kk, a.status, abort_word) &&
+                                            pf_wait(&full[slot], (kk / NS) & 1, a.status, abort_word))) {
                 const unsigned char *wt = smem + L.stage_off + (size_t)slot * st.bytes;
                 const __half *sc = reinterpret_cast<const __half *>(wt + st.codes);
                 const __half *bi = sc + DN_ROWS * d.GI;

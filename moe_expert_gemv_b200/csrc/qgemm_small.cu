@@ -262,6 +262,8 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
         const int st = k % NS, use = k / NS;
         if (!failed && !mbar_wait(&full[st], use & 1, a.status))
             failed = true;
+        // the lanes of a warp decide together: the mma below is warp-collective
+        failed = __any_sync(0xffffffffu, failed);
         // code products and folded biases in one accumulator; the power-of-two
         // code scale rides on the group scale (exact)
         float acc[NT][4];

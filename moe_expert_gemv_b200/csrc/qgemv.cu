@@ -27,6 +27,31 @@
 #include "kernels.h"
 
 namespace qmoe {
+
+// ---------------------------------------------------- host: tensor map --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            (void)cudaGetLastError();
+    }
+    return fn;
+}
+
 namespace {
 
 constexpr int QG_CW = 16;                     // consumer warps
@@ -76,7 +101,9 @@ __host__ __device__ inline QgLayout qg_layout(int K, int bits, int ncol, int NS,
 
 template <int BITS, bool SWZ, int FMT, bool ROT>
 __global__ void __launch_bounds__(QG_THREADS, 1)
-    qgemv_kernel(QgemvArgs a, int NS, const __grid_constant__ CUtensorMap codes_map)
+    qgemv_kernel(QgemvArgs a, int NS, const __grid_constant__ CUtensorMap codes_map,
+                 const __grid_constant__ CUtensorMap sb0_map,
+                 const __grid_constant__ CUtensorMap sb1_map, int sbT)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -119,7 +146,8 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                 const int r0 = item * 16;
                 const int rows = min(16, a.N - r0);
                 const uint32_t row_bytes = (uint32_t)Kw * 4;
-                const uint32_t sb = (uint32_t)(rows * L.G * 2);
+                // (a transposed tensor copy delivers all 16 rows, past N zero-filled)
+                const uint32_t sb = (uint32_t)(((SWZ && sbT) ? 16 : rows) * L.G * 2);
                 unsigned char *stage = smem + L.stage_off + (size_t)st * L.stage_bytes;
                 if (SWZ) {
                     // the tensor copy always delivers the whole 16-row box
@@ -132,7 +160,14 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                         bulk_g2s(stage + (size_t)r * L.S * 4, a.packed + (size_t)(r0 + r) * Kw,
                                  row_bytes, &full[st], pol);
                 }
-                if (FMT == QG_AFFINE) {
+                if (SWZ && sbT) {
+                    // transposed: [G / 8][16 rows][8 halves] (or [G / 4][16][4
+                    // words]), so the 8 rows of a fragment read 16 bytes apart
+                    tma_load_3d(stage + L.codes_bytes, &sb0_map, 0, r0, 0, &full[st], pol);
+                    if (FMT == QG_AFFINE)
+                        tma_load_3d(stage + L.codes_bytes + L.sb_bytes, &sb1_map, 0, r0, 0,
+                                    &full[st], pol);
+                } else if (FMT == QG_AFFINE) {
                     bulk_g2s(stage + L.codes_bytes, a.scales + (size_t)r0 * L.G, sb, &full[st], pol);
                     bulk_g2s(stage + L.codes_bytes + L.sb_bytes, a.biases + (size_t)r0 * L.G, sb,
                              &full[st], pol);
@@ -184,6 +219,8 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
         const int st = k % NS, use = k / NS;
         if (!failed && !mbar_wait(&full[st], use & 1, a.status))
             failed = true;
+        // the lanes of a warp decide together: the mma below is warp-collective
+        failed = __any_sync(0xffffffffu, failed);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         if (!failed) {
             const unsigned char *stage = smem + L.stage_off + (size_t)st * L.stage_bytes;
@@ -267,10 +304,14 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                     const unsigned char *base =
                         stage + (SWZ ? (gb / GPC) * 2048 : gb * (BITS == 4 ? 32 : 64));
                     if (FMT == QG_AFFINE) {
-                        const uint2 slo = *reinterpret_cast<const uint2 *>(sc + gid * L.G + gb);
-                        const uint2 shi = *reinterpret_cast<const uint2 *>(sc + (gid + 8) * L.G + gb);
-                        const uint2 blo = *reinterpret_cast<const uint2 *>(bi + gid * L.G + gb);
-                        const uint2 bhi = *reinterpret_cast<const uint2 *>(bi + (gid + 8) * L.G + gb);
+                        // row r, groups gb..gb+3: row-major [16][G], or
+                        // transposed [G/8][16][8]
+                        const int olo = sbT ? ((gb >> 3) * 16 + gid) * 8 + (gb & 7) : gid * L.G + gb;
+                        const int ohi = sbT ? olo + 8 * 8 : (gid + 8) * L.G + gb;
+                        const uint2 slo = *reinterpret_cast<const uint2 *>(sc + olo);
+                        const uint2 shi = *reinterpret_cast<const uint2 *>(sc + ohi);
+                        const uint2 blo = *reinterpret_cast<const uint2 *>(bi + olo);
+                        const uint2 bhi = *reinterpret_cast<const uint2 *>(bi + ohi);
                         const uint32_t sl[2] = {slo.x, slo.y}, sh[2] = {shi.x, shi.y};
                         const uint32_t bl[2] = {blo.x, blo.y}, bh[2] = {bhi.x, bhi.y};
 #pragma unroll
@@ -285,8 +326,11 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                         }
                     } else {
                         const uint32_t *prm = reinterpret_cast<const uint32_t *>(sc);
-                        const uint4 plo = *reinterpret_cast<const uint4 *>(prm + gid * L.G + gb);
-                        const uint4 phi = *reinterpret_cast<const uint4 *>(prm + (gid + 8) * L.G + gb);
+                        // row-major [16][G] words, or transposed [G/4][16][4]
+                        const int olo = sbT ? ((gb >> 2) * 16 + gid) * 4 : gid * L.G + gb;
+                        const int ohi = sbT ? olo + 8 * 4 : (gid + 8) * L.G + gb;
+                        const uint4 plo = *reinterpret_cast<const uint4 *>(prm + olo);
+                        const uint4 phi = *reinterpret_cast<const uint4 *>(prm + ohi);
                         const uint32_t pl[4] = {plo.x, plo.y, plo.z, plo.w};
                         const uint32_t ph[4] = {phi.x, phi.y, phi.z, phi.w};
 #pragma unroll
@@ -352,6 +396,26 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
     }
 }
 
+// 3-D map of a per-group parameter array [rows][G] of elem-byte entries seen
+// as [G / n16][rows][n16] (n16 entries = 16 bytes): one copy delivers a
+// 16-row tile transposed, [G / n16][16][n16]
+bool encode_param_map_t(CUtensorMap *m, const void *base, long rows, int G, int elem)
+{
+    EncodeTiledFn fn = encode_tiled_fn();
+    const int n16 = 16 / elem;
+    if (!fn || (reinterpret_cast<uintptr_t>(base) & 15u) || G % n16 || G / n16 > 256 ||
+        ((size_t)G * elem) % 16)
+        return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)n16, (cuuint64_t)rows, (cuuint64_t)(G / n16)};
+    const cuuint64_t strides[2] = {(cuuint64_t)G * elem, 16};
+    const cuuint32_t box[3] = {(cuuint32_t)n16, 16, (cuuint32_t)(G / n16)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32, 3,
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BITS, bool SWZ, int FMT, bool ROT>
 cudaError_t launch_qgemv_t(const QgemvArgs &a, const LaunchCfg &c, const CUtensorMap &m)
 {
@@ -369,8 +433,22 @@ cudaError_t launch_qgemv_t(const QgemvArgs &a, const LaunchCfg &c, const CUtenso
     cudaError_t e;
     if ((e = set_smem(qgemv_kernel<BITS, SWZ, FMT, ROT>, L.total)) != cudaSuccess)
         return e;
+    // scales and biases (or the parameter words) transposed by tensor copies
+    // where the rows take the swizzled tile path and G % 64 == 0
+    const int G = a.K / kGroup;
+    CUtensorMap m0, m1;
+    memset(&m0, 0, sizeof(m0));
+    memset(&m1, 0, sizeof(m1));
+    int sbT = 0;
+    if (SWZ && G % 64 == 0) {
+        if (FMT == QG_AFFINE)
+            sbT = encode_param_map_t(&m0, a.scales, a.N, G, 2) &&
+                  encode_param_map_t(&m1, a.biases, a.N, G, 2);
+        else
+            sbT = encode_param_map_t(&m0, a.params, a.N, G, 4);
+    }
     return launch_ex(qgemv_kernel<BITS, SWZ, FMT, ROT>, dim3(grid), dim3(QG_THREADS), L.total, c, 1,
-                     a, NS, m);
+                     a, NS, m, m0, m1, sbT);
 }
 
 template <bool SWZ>
@@ -392,30 +470,6 @@ cudaError_t launch_qgemv_fmt(const QgemvArgs &a, const LaunchCfg &c, const CUten
 }
 
 }  // namespace
-
-// ---------------------------------------------------- host: tensor map --
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_tiled_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-        else
-            (void)cudaGetLastError();
-    }
-    return fn;
-}
 
 bool encode_codes_map(CUtensorMap *m, const uint32_t *packed, long rows, int Kw, int box_rows,
                       int box_chunks)

@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(RT_THREADS, 1) router_kernel(RouterArgs a, int
         named_bar_sync(1, RT_CW * 32);
         const int gid = lane >> 2, tig = lane & 3;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (rows > 0 && mbar_wait(full, 0, a.status)) {
+        // the lanes of a warp decide together: the mma below is warp-collective
+        if (__all_sync(0xffffffffu, rows > 0 && mbar_wait(full, 0, a.status))) {
             const uint32_t *tile = reinterpret_cast<const uint32_t *>(tile_base);
             const __half *sc = reinterpret_cast<const __half *>(tile_base + L.codes_bytes);
             const __half *bi = reinterpret_cast<const __half *>(tile_base + L.codes_bytes + L.sb_bytes);

@@ -69,6 +69,7 @@ def lib():
             "moe_decode_pack_layer": [p, p, p, sz, p],
             "moe_decode_workspace_bytes": [i32, i32, i32, i32],
             "moe_decode_layers": [p, i32, i32, i32, i32, p, i32, p, p, p, p, p, sz, p, p],
+            "moe_decode_layers_host": [p, i32, i32, i32, i32, p, p, i32, p, p, p, sz, p, p],
             "moe_prefill_workspace_bytes": [p, i32, i32],
             "moe_prefill_qgemm": [p, p, i32, p, p, i32, p, p, sz, p, p],
             "qmoe_pack_codes": [p, i32, i32, i32, p, p],
@@ -574,6 +575,28 @@ def moe_decode_layers(stack, x, y=None, idx=None, weights=None, logits=None, sta
                                    _ptr(stack.workspace), stack.workspace.numel(), _ptr(status),
                                    _stream()), "moe_decode_layers")
     return y
+
+
+def moe_decode_layers_host(stack, x_host, y_host, x_dev, y_dev, status=None):
+    """The decode step from host buffers through the C call that copies them:
+    x_host -> x_dev, the fused decode, y_dev -> y_host, enqueued on the
+    current stream (synchronise before reading y_host).  x_host / y_host:
+    float16 [n_layers][hidden] CPU tensors (pinned for asynchronous copies);
+    x_dev / y_dev: device staging tensors of the same shape."""
+    n = len(stack.packed)
+    for t, name in ((x_host, "x_host"), (y_host, "y_host")):
+        if t.device.type != "cpu" or t.dtype != torch.float16 or tuple(t.shape) != (n, stack.H) \
+                or not t.is_contiguous():
+            raise ValueError("%s: expected a contiguous CPU float16 [%d, %d] tensor" % (name, n, stack.H))
+    _need(x_dev, torch.float16, "x_dev", (n, stack.H))
+    _need(y_dev, torch.float16, "y_dev", (n, stack.H))
+    _check(lib().moe_decode_layers_host(stack.c_packed, n, stack.E, stack.H, stack.I,
+                                        ctypes.c_void_p(x_host.data_ptr()),
+                                        ctypes.c_void_p(y_host.data_ptr()), stack.top_k,
+                                        _ptr(x_dev), _ptr(y_dev), _ptr(stack.workspace),
+                                        stack.workspace.numel(), _ptr(status), _stream()),
+           "moe_decode_layers_host")
+    return y_host
 
 
 def moe_group_tokens(idx, num_experts, status=None):

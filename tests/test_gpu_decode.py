@@ -71,6 +71,28 @@ def test_moe_e128_three_layers_and_repeat(cuda_dev):
     check_layers(ms, E, H, I, k, x16, y2, idx2, wt2, lg2)
 
 
+def test_host_buffer_entry_point(cuda_dev):
+    """moe_decode_layers_host: x from a pinned host buffer, y back into one,
+    through the C call that enqueues both copies and the decode; outputs match
+    the oracle like the device-buffer call."""
+    E, H, I, k, n = 32, 512, 128, 8, 3
+    ms, stack = make_stack(81, n, E, H, I, k)
+    x16 = np.concatenate([synth.activations(81 + l, 1, H, layer=l) for l in range(n)])
+    x_host = torch.from_numpy(x16.view(np.float16).copy()).pin_memory()
+    y_host = torch.empty(n, H, dtype=torch.float16).pin_memory()
+    x_dev = torch.empty(n, H, dtype=torch.float16, device="cuda")
+    y_dev = torch.empty(n, H, dtype=torch.float16, device="cuda")
+    qmoe.moe_decode_layers_host(stack, x_host, y_host, x_dev, y_dev)
+    assert qmoe.qmoe_check_status() == 0   # synchronises the stream
+    y, idx, wt, lg = run(stack, x16, E, k)
+    assert_close(y_host.numpy(), y.view(np.float16).astype(np.float64), what="host entry vs device")
+    for l in range(n):
+        _, oidx, owt = oracle.router(*ms[l]["router"], E, H, 8, x16[l:l + 1], k)
+        y64, _ = oracle.Layer(ms[l], E, H, I).moe(x16[l:l + 1], idx[l:l + 1],
+                                                  wt[l:l + 1].astype(np.float64))
+        assert_close(y_host.numpy()[l], y64[0], what="host entry layer %d vs oracle" % l)
+
+
 def test_matches_unfused_path(cuda_dev):
     """Same bits as moe_router_topk + moe_expert_qmlp would give within the
     tolerance, and identical routing."""
