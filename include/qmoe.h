@@ -111,11 +111,13 @@ typedef struct qmoe_moe_layer {
  * batch 1..32: up to 8 rows of x per kernel launch (tensor-core N = 8); a
  * larger batch (e.g. the 16-32 draft tokens a speculative-decoding step
  * verifies) runs one launch per 8 rows, the later ones reading a matrix
- * that fits L2 from L2.
+ * that fits L2 from L2.  Where 8 rows of x beside one 16-row weight tile
+ * overflow shared memory (long 8-bit rows, e.g. cols 8192), each launch
+ * takes as many rows as fit.
  * Errors: INVALID_ARG (NULL, batch outside 1..32, shape), ALIGNMENT,
- * UNSUPPORTED (group != 64, cols % 64, rows % 8, or x of up to 8 rows plus
- * one 16-row tile over shared memory: e.g. 8-bit cols 8192 at batch 8;
- * qgemv_affine_ws takes such rows from batch 9 on), CUDA.
+ * UNSUPPORTED (group != 64, cols % 64, rows % 8, or rows too long for one
+ * row of x plus one 16-row tile in shared memory: cols above 18624 at 4 bits,
+ * 11008 at 8 bits; qgemv_affine_ws takes such rows from batch 9 on), CUDA.
  * ------------------------------------------------------------------------- */
 qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch,
                          uint16_t *y, int32_t *status_dev, void *stream);
@@ -169,7 +171,8 @@ qmoe_status qgemv_affine_ws(const qmoe_qmatrix *W, const uint16_t *x, int32_t ba
  *           as an fp16 (hi, lo) pair (about 22 significant bits).
  * batch 1..32 (as qgemv_affine); cols a multiple of 64, rows of 8;
  * y fp16 [batch][rows].  Errors as qgemv_affine (INVALID_ARG also for an
- * unknown format).
+ * unknown format; with rht_signs the x pair halves the room, and rows of
+ * more than 15872 cols at 4 bits or 9984 at 8 bits are UNSUPPORTED).
  * ------------------------------------------------------------------------- */
 #define QMOE_FMT_ZP4_BF16 1
 #define QMOE_FMT_SYM8_BF16 2

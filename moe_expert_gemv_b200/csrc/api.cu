@@ -292,7 +292,7 @@ qmoe_status qgemv_affine_ws(const qmoe_qmatrix *W, const uint16_t *x, int32_t ba
     a.y = reinterpret_cast<__half *>(y);
     a.status = status_dev ? status_dev : d->status;
     if (batch <= 8)
-        return cuda_status(launch_qgemv(a, launch_cfg(d, stream)));
+        return cuda_status(launch_qgemv_batched(a, launch_cfg(d, stream)));
     bool used = false;
     return cuda_status(launch_qgemm_small(a, workspace, workspace_bytes, launch_cfg(d, stream), &used));
 }

@@ -55,8 +55,6 @@ static EncodeTiledFn encode_tiled_fn()
 namespace {
 
 constexpr int QG_CW = 16;                     // consumer warps
-constexpr int QG_GW = 4;                      // warps per consumer group (one tile at a time)
-constexpr int QG_GROUPS = QG_CW / QG_GW;
 constexpr int QG_CT = QG_CW * 32;             // consumer threads
 constexpr int QG_THREADS = QG_CT + 32;        // + one producer warp
 constexpr int QG_MAX_STAGES = 8;
@@ -122,7 +120,7 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], QG_GW);   // the warps of the group that reads it
+            mbar_init(&empty[s], QG_CW);
         }
         mbar_init_fence();
     }
@@ -201,21 +199,15 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                       ctid, QG_CT);
     named_bar_sync(1, QG_CT);
 
-    // Tiles go to groups of QG_GW warps in turn (tile k of this CTA to group
-    // k % QG_GROUPS), so a slow warp holds up its own group only; the warps of
-    // a group split the tile's 64-input groups into contiguous blocks, so
-    // that with G % 64 == 0 a row's scales and biases come as one 8-byte load
-    // per 4 groups.
-    const int grp = warp / QG_GW, wg = warp % QG_GW;
-    const int gpw = (L.G + QG_GW - 1) / QG_GW;
-    const int g0 = min(L.G, wg * gpw), g1 = min(L.G, g0 + gpw);
+    // this warp's groups: a contiguous block, so that with G % 64 == 0 the
+    // scales and biases of a row come as one 8-byte load per 4 groups
+    const int gpw = (L.G + QG_CW - 1) / QG_CW;
+    const int g0 = min(L.G, warp * gpw), g1 = min(L.G, g0 + gpw);
     const bool vec_sb = (L.G & 63) == 0;
     const int gid = lane >> 2, tig = lane & 3;
     bool failed = false;
     int k = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
-        if (k % QG_GROUPS != grp)
-            continue;   // another group's tile
         const int st = k % NS, use = k / NS;
         if (!failed && !mbar_wait(&full[st], use & 1, a.status))
             failed = true;
@@ -363,16 +355,12 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&empty[st]);
-        // partials of the group's warps; two buffers alternate between the
-        // group's tiles, so a warp that runs ahead cannot overwrite the ones
-        // the first warp is still adding
-        const int par = (k / QG_GROUPS) & 1;
-        red[(par * QG_CW + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        named_bar_sync(2 + grp, QG_GW * 32);
-        if (wg == 0) {
+        red[((k & 1) * QG_CW + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        named_bar_sync(1, QG_CT);
+        if (warp == k % QG_CW) {
             float v[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int w = 0; w < QG_GW; ++w) {
-                const float4 p = red[(par * QG_CW + grp * QG_GW + w) * 32 + lane];
+            for (int w = 0; w < QG_CW; ++w) {
+                const float4 p = red[((k & 1) * QG_CW + w) * 32 + lane];
                 v[0] += p.x;
                 v[1] += p.y;
                 v[2] += p.z;
@@ -532,13 +520,28 @@ cudaError_t launch_qgemv(const QgemvArgs &a, const LaunchCfg &c)
     return swz ? launch_qgemv_fmt<true>(a, c, m) : launch_qgemv_fmt<false>(a, c, m);
 }
 
+// does a slice of b rows of x fit on chip beside one stage of 16 weight rows
+// (either tile layout launch_qgemv may pick)?
+static bool slice_fits(const QgemvArgs &a, int b)
+{
+    const bool rot = a.signs != nullptr;
+    const size_t budget = 227 * 1024;
+    const bool swz_ok = (a.K * a.bits / 32) % 32 == 0 &&
+                        qg_layout(a.K, a.bits, b, 1, true, rot).total <= budget;
+    return swz_ok || qg_layout(a.K, a.bits, b, 1, false, rot).total <= budget;
+}
+
 cudaError_t launch_qgemv_batched(const QgemvArgs &a, const LaunchCfg &c)
 {
-    for (int b0 = 0; b0 < a.B; b0 += 8) {
+    // rows of x per launch: 8, fewer where long 8-bit rows leave no room
+    int step = a.B < 8 ? a.B : 8;
+    while (step > 1 && !slice_fits(a, step))
+        --step;
+    for (int b0 = 0; b0 < a.B; b0 += step) {
         QgemvArgs s = a;
         s.x = a.x + (size_t)b0 * a.K;
         s.y = a.y + (size_t)b0 * a.N;
-        s.B = a.B - b0 < 8 ? a.B - b0 : 8;
+        s.B = a.B - b0 < step ? a.B - b0 : step;
         const cudaError_t e = launch_qgemv(s, c);
         if (e != cudaSuccess)
             return e;

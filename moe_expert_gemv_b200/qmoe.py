@@ -18,6 +18,13 @@ from . import build as _build
 _lib = None
 
 OK = 0
+ERR_INVALID_ARG = -1
+ERR_ALIGNMENT = -2
+ERR_UNSUPPORTED = -3
+ERR_CUDA = -4
+ERR_DEVICE_STATUS = -5
+ERR_TIMEOUT = -6
+ERR_WORKSPACE = -7
 DEV_BAD_EXPERT = 0x1
 DEV_TIMEOUT = 0x2
 

@@ -36,6 +36,16 @@ def test_status_strings_without_gpu():
         assert lib.qmoe_status_string(code).startswith(b"QMOE_")
 
 
+def test_binding_status_codes_match_the_header():
+    """The binding's ERR_* constants carry the values of the header's enum."""
+    from moe_expert_gemv_b200 import qmoe
+    src = open(os.path.join(ROOT, "include", "qmoe.h")).read()
+    codes = dict(re.findall(r"QMOE_(ERR_[A-Z_]+)\s*=\s*(-?\d+)", src))
+    assert len(codes) == 7
+    for name, value in codes.items():
+        assert getattr(qmoe, name) == int(value), name
+
+
 def test_one_pass_workspace_sizes_without_gpu():
     """qgemv_affine_workspace_bytes is host arithmetic: the one-pass plan for
     batch 9..32 (K slices whose x fits 64 KB of shared memory, ~32 KB weight

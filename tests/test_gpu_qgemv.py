@@ -223,3 +223,30 @@ def test_repeat_calls_bitwise_identical(cuda_dev):
     a = qmoe.qgemv_affine(W, x).clone()
     for _ in range(3):
         assert torch.equal(qmoe.qgemv_affine(W, x), a)
+
+
+@pytest.mark.parametrize("Bt", [6, 8])
+def test_long_8bit_rows_take_fewer_rows_per_launch(cuda_dev, Bt):
+    """8-bit rows of 8192 columns: 8 rows of x beside a 16-row tile overflow
+    shared memory, so each launch takes 4 rows; every output against the
+    oracle."""
+    N, K = 136, 8192
+    P, S, B = synth.qmatrix(synth.rng(N, K, 8, 41), N, K, 8)
+    x16 = synth.activations(K + Bt, Bt, K)
+    y = run_qgemv(P, S, B, N, K, 8, x16)
+    y64, _ = oracle.qgemv(P, S, B, N, K, 8, x16)
+    assert_close_rows(y.view(np.float16), y64, what="8-bit K=8192 B=%d" % Bt)
+
+
+def test_rows_too_long_for_one_tile_unsupported(cuda_dev):
+    """A 16-row tile of 8-bit rows of 11072 columns plus one row of x does
+    not fit in shared memory (11008 is the longest that does): UNSUPPORTED,
+    and nothing is launched."""
+    N, K = 16, 11072
+    P, S, B = synth.qmatrix(synth.rng(N, K, 8, 42), N, K, 8)
+    W = qmoe.QMatrix.from_numpy(P, S, B, N, K, 8)
+    x = to_dev_f16(synth.activations(43, 1, K))
+    with pytest.raises(qmoe.QmoeError) as e:
+        qmoe.qgemv_affine(W, x)
+    assert e.value.code == qmoe.ERR_UNSUPPORTED
+    assert qmoe.qmoe_check_status() == 0
