@@ -205,6 +205,20 @@ __device__ __forceinline__ void dequant4_word(uint32_t w, uint32_t *p)
     p[3] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(ws, 0x00F000F0u, magic)), k1_16, km64));
 }
 
+// The same pairs centred, q - 8 (exact: 1024 + q - 1032, (1024 + 16q)/16 - 72).
+__device__ __forceinline__ void dequant4c_word(uint32_t w, uint32_t *p)
+{
+    const uint32_t magic = 0x64006400u;
+    const __half2 k1032 = __floats2half2_rn(1032.f, 1032.f);
+    const __half2 k1_16 = __floats2half2_rn(0.0625f, 0.0625f);
+    const __half2 km72 = __floats2half2_rn(-72.f, -72.f);
+    const uint32_t ws = w >> 8;
+    p[0] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, magic)), k1032));
+    p[1] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(w, 0x00F000F0u, magic)), k1_16, km72));
+    p[2] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(ws, 0x000F000Fu, magic)), k1032));
+    p[3] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(ws, 0x00F000F0u, magic)), k1_16, km72));
+}
+
 // 8-bit: one word holds codes c0..c3 (byte i = code i).
 //   p[0] = (c0, c2)  p[1] = (c1, c3)
 __device__ __forceinline__ void dequant8_word(uint32_t w, uint32_t *p)
@@ -216,30 +230,31 @@ __device__ __forceinline__ void dequant8_word(uint32_t w, uint32_t *p)
 }
 
 // Cheaper dequantisation for the streaming kernels: the code itself becomes
-// the fp16 bit pattern (no exponent bits), i.e. the subnormal q * 2^-24, or
-// 16q * 2^-24 for a nibble in bits 4..7.  fp16 subnormals enter the tensor
-// core without being flushed (measured: group partials within ~2e-6 relative
-// of exact), so a whole word costs one shift and four ANDs.  Pairs:
-//   p[0] = (c0, c4) * 2^-24     p[1] = (c1, c5) * 2^-20
-//   p[2] = (c2, c6) * 2^-24     p[3] = (c3, c7) * 2^-20
-// The 2^-24 and 2^-20 classes go to separate mma accumulators c (class 0)
-// and d (class 1) and are recombined as 2^20 * (16 c + d).
+// the fp16 bit pattern (no exponent bits), i.e. an fp16 subnormal.  Every
+// code is placed in the top mantissa bits (a nibble in bits 6..9: 64q *
+// 2^-24 = q * 2^-18; a byte in bits 2..9: b * 2^-22).  Measured on B200
+// (mma.sync m16n8k16, f16 x f16 -> f32): with the codes in the top mantissa
+// bits the products are as accurate as with the codes as normal fp16
+// integers (~1e-7 of sum |a b|); a nibble left in bits 0..3 (q * 2^-24)
+// loses up to 2e-5 of sum |a b|.  A word costs four shifts and four ANDs.
+// Pairs (both halves of a register):
+//   p[0] = (c0, c4)   p[1] = (c1, c5)   p[2] = (c2, c6)   p[3] = (c3, c7)
+// all in units of 2^-18; callers scale results by kCode4 = 2^18.
 __device__ __forceinline__ void dequant4s_word(uint32_t w, uint32_t *p)
 {
-    const uint32_t ws = w >> 8;
-    p[0] = w & 0x000F000Fu;
-    p[1] = w & 0x00F000F0u;
-    p[2] = ws & 0x000F000Fu;
-    p[3] = ws & 0x00F000F0u;
+    p[0] = (w << 6) & 0x03C003C0u;
+    p[1] = (w << 2) & 0x03C003C0u;
+    p[2] = (w >> 2) & 0x03C003C0u;
+    p[3] = (w >> 6) & 0x03C003C0u;
 }
-// 8-bit: bytes as subnormals q * 2^-24: p[0] = (c0, c2), p[1] = (c1, c3).
+// 8-bit: bytes as subnormals b * 2^-22: p[0] = (c0, c2), p[1] = (c1, c3).
 __device__ __forceinline__ void dequant8s_word(uint32_t w, uint32_t *p)
 {
-    p[0] = w & 0x00FF00FFu;
-    p[1] = (w >> 8) & 0x00FF00FFu;
+    p[0] = (w << 2) & 0x03FC03FCu;
+    p[1] = (w >> 6) & 0x03FC03FCu;
 }
-constexpr float kSub24 = 16777216.f;   // 2^24
-constexpr float kSub20 = 1048576.f;    // 2^20
+constexpr float kCode4 = 262144.f;    // 2^18: undoes dequant4s_word
+constexpr float kCode8 = 4194304.f;   // 2^22: undoes dequant8s_word
 
 // x order matching dequant4s_word, k-blocks (c0,c4)(c2,c6) | (c8,c12)(c10,c14)
 // | (c1,c5)(c3,c7) | (c9,c13)(c11,c15): class-0 codes in the first 8 slots.
@@ -363,9 +378,8 @@ __device__ __forceinline__ const void *swz128_frag(const unsigned char *tile, in
 
 // Subnormal-code group product of a 16-row tile (rows gid, gid+8 from wa, wb;
 // x fragments in the order of xperm(kPermS4, .) for 4-bit, xperm(8, .) for
-// 8-bit): returns sum_k q x per C element, scaled by 2^-20 (4-bit) or 2^-24
-// (8-bit).  4-bit: class-0 k-blocks accumulate in c, class-1 in d, combined
-// as 16c + d.
+// 8-bit): returns sum_k q x per C element, scaled by 2^-18 (4-bit) or 2^-22
+// (8-bit).  Two accumulators (c, d) per call keep two mma chains in flight.
 __device__ __forceinline__ void mma_group_s4(float (&r)[4], uint2 wa, uint2 wb, uint4 x0, uint4 x1)
 {
     uint32_t pa[8], pb[8];
@@ -380,7 +394,7 @@ __device__ __forceinline__ void mma_group_s4(float (&r)[4], uint2 wa, uint2 wb, 
     mma_16816(d, pa[5], pb[5], pa[7], pb[7], x1.z, x1.w);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        r[i] = fmaf(16.f, c[i], d[i]);
+        r[i] = c[i] + d[i];
 }
 __device__ __forceinline__ void mma_group_s8(float (&r)[4], uint4 wa, uint4 wb, uint4 x0, uint4 x1)
 {
@@ -404,8 +418,11 @@ __device__ __forceinline__ void mma_group_s8(float (&r)[4], uint4 wa, uint4 wb, 
 }
 
 // The same products with an activation held as an fp16 (hi, lo) pair: the
-// codes are dequantised once and both parts accumulate, i.e. the result is
-// that of mma_group_s4 / mma_group_s8 applied to hi + lo.
+// codes are dequantised once and the result is that of mma_group_s4 /
+// mma_group_s8 applied to hi + lo.  The lo products (about 2^-11 of the hi
+// ones) accumulate in their own registers and meet the hi sums only in an
+// fp32 add: chained into the hi accumulator, part of their bits were lost
+// inside the tensor-core addition.
 __device__ __forceinline__ void mma_group_s4_hilo(float (&r)[4], uint2 wa, uint2 wb, uint4 h0,
                                                   uint4 h1, uint4 l0, uint4 l1)
 {
@@ -415,17 +432,18 @@ __device__ __forceinline__ void mma_group_s4_hilo(float (&r)[4], uint2 wa, uint2
     dequant4s_word(wb.x, pb);
     dequant4s_word(wb.y, pb + 4);
     float c[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
+    float cl[4] = {0.f, 0.f, 0.f, 0.f}, el[4] = {0.f, 0.f, 0.f, 0.f};
     mma_16816(c, pa[0], pb[0], pa[2], pb[2], h0.x, h0.y);
     mma_16816(e, pa[1], pb[1], pa[3], pb[3], h1.x, h1.y);
     mma_16816(c, pa[4], pb[4], pa[6], pb[6], h0.z, h0.w);
     mma_16816(e, pa[5], pb[5], pa[7], pb[7], h1.z, h1.w);
-    mma_16816(c, pa[0], pb[0], pa[2], pb[2], l0.x, l0.y);
-    mma_16816(e, pa[1], pb[1], pa[3], pb[3], l1.x, l1.y);
-    mma_16816(c, pa[4], pb[4], pa[6], pb[6], l0.z, l0.w);
-    mma_16816(e, pa[5], pb[5], pa[7], pb[7], l1.z, l1.w);
+    mma_16816(cl, pa[0], pb[0], pa[2], pb[2], l0.x, l0.y);
+    mma_16816(el, pa[1], pb[1], pa[3], pb[3], l1.x, l1.y);
+    mma_16816(cl, pa[4], pb[4], pa[6], pb[6], l0.z, l0.w);
+    mma_16816(el, pa[5], pb[5], pa[7], pb[7], l1.z, l1.w);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        r[i] = fmaf(16.f, c[i], e[i]);
+        r[i] = (c[i] + e[i]) + (cl[i] + el[i]);
 }
 __device__ __forceinline__ void mma_group_s8_hilo(float (&r)[4], uint4 wa, uint4 wb, uint4 h0,
                                                   uint4 h1, uint4 l0, uint4 l1)
@@ -440,17 +458,18 @@ __device__ __forceinline__ void mma_group_s8_hilo(float (&r)[4], uint4 wa, uint4
     dequant8s_word(wa.w, pa + 6);
     dequant8s_word(wb.w, pb + 6);
     float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
+    float cl[4] = {0.f, 0.f, 0.f, 0.f}, dl[4] = {0.f, 0.f, 0.f, 0.f};
     mma_16816(c, pa[0], pb[0], pa[1], pb[1], h0.x, h0.y);
     mma_16816(d, pa[2], pb[2], pa[3], pb[3], h0.z, h0.w);
     mma_16816(c, pa[4], pb[4], pa[5], pb[5], h1.x, h1.y);
     mma_16816(d, pa[6], pb[6], pa[7], pb[7], h1.z, h1.w);
-    mma_16816(c, pa[0], pb[0], pa[1], pb[1], l0.x, l0.y);
-    mma_16816(d, pa[2], pb[2], pa[3], pb[3], l0.z, l0.w);
-    mma_16816(c, pa[4], pb[4], pa[5], pb[5], l1.x, l1.y);
-    mma_16816(d, pa[6], pb[6], pa[7], pb[7], l1.z, l1.w);
+    mma_16816(cl, pa[0], pb[0], pa[1], pb[1], l0.x, l0.y);
+    mma_16816(dl, pa[2], pb[2], pa[3], pb[3], l0.z, l0.w);
+    mma_16816(cl, pa[4], pb[4], pa[5], pb[5], l1.x, l1.y);
+    mma_16816(dl, pa[6], pb[6], pa[7], pb[7], l1.z, l1.w);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        r[i] = c[i] + d[i];
+        r[i] = (c[i] + d[i]) + (cl[i] + dl[i]);
 }
 
 // Smem row stride (in 32-bit words) for a tile of `cols` inputs so that the

@@ -612,8 +612,8 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
             gu_buf ^= 1;
             float *gr = gub + (size_t)warp * 16;
             if (tig == 0) {
-                gr[gid] = ag * kSub20 + bg;       // gate row gid
-                gr[8 + gid] = au * kSub20 + bu;   // up row gid
+                gr[gid] = ag * kCode4 + bg;       // gate row gid
+                gr[8 + gid] = au * kCode4 + bu;   // up row gid
             }
             named_bar_sync(BAR_GROUP0 + q, DC_GW * 32);
             if (wq == 0) {
@@ -696,8 +696,8 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                     if (tig == 0) {
                         const float2 pa = sb_word(S + P.st_codes + 4 * (size_t)r0);
                         const float2 pb = sb_word(S + P.st_codes + 4 * (size_t)(r0 + 8));
-                        const float va = fmaf(pa.x * kSub20, r[0] + r[1], pa.y * X);
-                        const float vb = fmaf(pb.x * kSub20, r[2] + r[3], pb.y * X);
+                        const float va = fmaf(pa.x * kCode4, r[0] + r[1], pa.y * X);
+                        const float vb = fmaf(pb.x * kCode4, r[2] + r[3], pb.y * X);
                         my_ypart[r0] = fmaf(w, va, my_ypart[r0]);
                         my_ypart[r0 + 8] = fmaf(w, vb, my_ypart[r0 + 8]);
                     }
@@ -766,8 +766,8 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                 if (!good)
                     ok = false;
                 if (tig == 0) {
-                    red[warp * 16 + gid] = acc_lo * kSub24 + b_lo;
-                    red[warp * 16 + 8 + gid] = acc_hi * kSub24 + b_hi;
+                    red[warp * 16 + gid] = acc_lo * kCode8 + b_lo;
+                    red[warp * 16 + 8 + gid] = acc_hi * kCode8 + b_hi;
                 }
                 named_bar_sync(BAR_ALL, DC_CT);
                 if (ctid == 0)

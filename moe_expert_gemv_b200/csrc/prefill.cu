@@ -547,7 +547,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         off[j] = gid * st.S * 4 + j * 32 + tig * 8;
                 }
                 // code products and folded biases accumulate apart; the
-                // subnormal factor 2^20 is applied once at the end
+                // subnormal factor 2^18 is applied once at the end
                 float aq[4] = {0.f, 0.f, 0.f, 0.f}, ab[4] = {0.f, 0.f, 0.f, 0.f};
                 const int nch = d.GH / 4;
                 for (int q4 = 0; q4 < nch; ++q4) {
@@ -592,7 +592,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 float acc[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
-                    acc[i] = fmaf(aq[i], kSub20, ab[i]);
+                    acc[i] = fmaf(aq[i], kCode4, ab[i]);
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&empty[slot]);
@@ -779,7 +779,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 float acc[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    acc[i] = fmaf(aq[i], kSub20, ab[i]);
+                    acc[i] = fmaf(aq[i], kCode4, ab[i]);
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&empty[slot]);

@@ -13,15 +13,23 @@
 // W[rows, K] X[N tokens, K]^T, the weights as the M operand and the slot's
 // tokens (N <= 128, padded to a multiple of 16) as N.  Per 64-input group:
 //   * a TMA copy brings the group's 4-bit codes of the 128 rows (4 KB);
-//   * 8 dequantisation warps turn them into w' = s*q as an EXACT pair of
-//     fp16 values: hi = fp16(s*q) (one HMUL2) and lo = s*q - hi (one HFMA2,
-//     exact because s*q has at most 15 significant bits), written in the
-//     128-byte-swizzled K-major layout the tensor core reads;
-//   * one thread issues tcgen05.mma kind::f16 for hi and lo into the same
-//     fp32 accumulator in tensor memory.
-// The bias is one more K-block: A = b[row][group] (fp16, exact), B = the
-// group sums of the activations as an fp16 (hi, lo) pair, so that
-//   D = sum_g s_g sum_k q x + sum_g b_g X_g   (= the affine product)
+//   * 8 dequantisation warps turn them into w' = s*(q - 8) as an EXACT pair
+//     of fp16 values: hi = fp16(w') (one HMUL2) and lo = w' - hi (one HFMA2,
+//     exact because w' has at most 15 significant bits), written in the
+//     128-byte-swizzled K-major layout the tensor core reads.  The centred
+//     codes keep the running sums small: the tensor core's additions lose
+//     bits in proportion to the accumulator's magnitude, and 0..15 codes
+//     would add a 7.5 s sum(x) drift to every partial sum;
+//   * one thread issues tcgen05.mma kind::f16: the hi x hi products into
+//     one fp32 accumulator in tensor memory, the small cross products
+//     (about 2^-11 of the others) into a second one; the epilogue adds the
+//     two in fp32.  Chained into the same accumulator, part of the cross
+//     products' bits were lost inside the tensor-core additions.
+// The bias is one more K-block: A = b' = b + 8 s per (row, group) as an fp16
+// (hi, lo) pair, B = the group sums of the activations as an fp16 (hi, lo)
+// pair, so that
+//   D = sum_g s_g sum_k (q - 8) x + sum_g (b_g + 8 s_g) X_g
+//     = sum_g s_g sum_k q x + sum_g b_g X_g   (= the affine product)
 // to fp32 accumulation.  A single fp16 or bf16 dequantised tile (s*q + b
 // rounded once) would cost up to 2e-2 of relative error on these
 // cancellation-heavy outputs; the exact pair keeps the products exact.
@@ -60,7 +68,8 @@ constexpr int TC_NA = 3;                               // A stages: hi + lo tile
 constexpr int TC_NB = 2;                               // B stages: two tiles
 constexpr int TC_TILE = 16384;                         // one 128 x 64 fp16 tile
 constexpr int TC_CODES = TC_M * 32;                    // codes of one group, 128 rows
-constexpr uint32_t TC_TMEM_COLS = 256;
+constexpr uint32_t TC_TMEM_COLS = 512;                 // all of an SM's tensor memory
+constexpr uint32_t TC_LO_COL = 256;                    // first column of the cross products
 constexpr int TC_BAR_EPI = 1;                          // named barrier of the epilogue warps
 constexpr int TC_SC_STRIDE = 66;                       // scale row stride in halves (33 words: odd)
 
@@ -402,19 +411,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         tc_fence_after();
                         const uint32_t ahi = smem_u32(a_ring + (size_t)sa * 2 * TC_TILE);
                         const uint32_t alo = ahi + TC_TILE;
+                        // hi x hi products in d; the small cross products
+                        // (lo x hi, hi x lo) in their own accumulator dl
                         const uint32_t d = tmem + (uint32_t)(m * 128);
+                        const uint32_t dl = d + TC_LO_COL;
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks) {
                             const uint32_t ko = 32u * ks;
                             const uint32_t acc0 = (kb > 0 || ks > 0) ? 1u : 0u;
                             if (bias) {
                                 tc_mma(d, tc_desc(ahi + ko), tc_desc(b0 + ko), idesc, 1u);
-                                tc_mma(d, tc_desc(ahi + ko), tc_desc(b1 + ko), idesc, 1u);
+                                tc_mma(dl, tc_desc(alo + ko), tc_desc(b0 + ko), idesc, 1u);
+                                tc_mma(dl, tc_desc(ahi + ko), tc_desc(b1 + ko), idesc, 1u);
                             } else {
                                 tc_mma(d, tc_desc(ahi + ko), tc_desc(b0 + ko), idesc, acc0);
-                                tc_mma(d, tc_desc(alo + ko), tc_desc(b0 + ko), idesc, 1u);
+                                tc_mma(dl, tc_desc(alo + ko), tc_desc(b0 + ko), idesc, acc0);
                                 if (DOWN)
-                                    tc_mma(d, tc_desc(ahi + ko), tc_desc(b1 + ko), idesc, 1u);
+                                    tc_mma(dl, tc_desc(ahi + ko), tc_desc(b1 + ko), idesc, 1u);
                             }
                         }
                         issued = true;
@@ -495,7 +508,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                         for (int w = 0; w < 4; ++w) {
                             uint32_t qv[4], hi[4], lo[4];
-                            dequant4_word(words[w], qv);   // (c0,c4)(c1,c5)(c2,c6)(c3,c7) exact
+                            dequant4c_word(words[w], qv);   // q - 8: (c0,c4)(c1,c5)(c2,c6)(c3,c7)
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
                                 const __half2 h = __hmul2(s2, u32_as_h2(qv[i]));
@@ -508,23 +521,36 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                             *reinterpret_cast<uint4 *>(rowlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                         }
                     } else {
-                        // bias block: A = b[row][group] for the K / 64 groups, zeros after
+                        // bias block: A = b' = b + 8 s per (row, group) for the K / 64
+                        // groups (zeros after) as an fp16 (hi, lo) pair -- the 8 s
+                        // the centred codes q - 8 left out
                         const QMat &W = DOWN ? (sh ? a.sh_down : a.down)
                                              : (m == 0 ? (sh ? a.sh_gate : a.gate) : (sh ? a.sh_up : a.up));
+                        const __half *srow = sc + ((size_t)m * TC_M + r) * TC_SC_STRIDE;
 #pragma unroll
                         for (int c4 = 0; c4 < 4; ++c4) {
                             const int chunk = hw * 4 + c4;
-                            uint32_t v[4];
+                            uint32_t vh[4], vl[4];
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
                                 // memory order of the chunk: groups 8c + (0,4,1,5,2,6,3,7)
                                 const int g0 = chunk * 8 + i, g1 = chunk * 8 + i + 4;
-                                const __half b0 = (rvalid && g0 < GK) ? W.biases[grow * GK + g0] : __float2half(0.f);
-                                const __half b1 = (rvalid && g1 < GK) ? W.biases[grow * GK + g1] : __float2half(0.f);
-                                v[i] = h2_as_u32(__halves2half2(b0, b1));
+                                const float f0 = (rvalid && g0 < GK)
+                                                     ? __half2float(W.biases[grow * GK + g0]) +
+                                                           8.f * __half2float(srow[g0])
+                                                     : 0.f;
+                                const float f1 = (rvalid && g1 < GK)
+                                                     ? __half2float(W.biases[grow * GK + g1]) +
+                                                           8.f * __half2float(srow[g1])
+                                                     : 0.f;
+                                const __half h0 = __float2half_rn(f0), h1 = __float2half_rn(f1);
+                                vh[i] = h2_as_u32(__halves2half2(h0, h1));
+                                vl[i] = h2_as_u32(__halves2half2(__float2half_rn(f0 - __half2float(h0)),
+                                                                 __float2half_rn(f1 - __half2float(h1))));
                             }
                             const int off = ((chunk ^ (r & 7)) << 4);
-                            *reinterpret_cast<uint4 *>(rowhi + off) = make_uint4(v[0], v[1], v[2], v[3]);
+                            *reinterpret_cast<uint4 *>(rowhi + off) = make_uint4(vh[0], vh[1], vh[2], vh[3]);
+                            *reinterpret_cast<uint4 *>(rowlo + off) = make_uint4(vl[0], vl[1], vl[2], vl[3]);
                         }
                     }
                     // generic-proxy writes -> visible to the tensor core
@@ -546,9 +572,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int c0 = 16 * chalf; c0 < t.npad; c0 += 32) {
                     float dv[16], uv[16];
                     const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0;
+                    float lv[16];
                     tc_ld16(ta, dv);
-                    if (!DOWN)
+                    tc_ld16(ta + TC_LO_COL, lv);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        dv[i] += lv[i];
+                    if (!DOWN) {
                         tc_ld16(ta + 128, uv);
+                        tc_ld16(ta + 128 + TC_LO_COL, lv);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            uv[i] += lv[i];
+                    }
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int n = c0 + i;

@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
     pdl_trigger();
     const int ctid = threadIdx.x;
     constexpr int KIND = BITS == 4 ? kPermS4 : 8;
-    constexpr float kCodeScale = BITS == 4 ? kSub20 : kSub24;
+    constexpr float kCodeScale = BITS == 4 ? kCode4 : kCode8;
     // this slice of x: columns 0..B-1 staged, sums of columns B..31 zero
     if (ROT)
         stage_x_groups<KIND, true>(xs, xsum, L.GS, a.B, a.x + (size_t)q * a.KS, a.K, ctid, SM_CT, 32,
@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
                     float r[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        r[i] = BITS == 4 ? fmaf(16.f, c[nt][i], d[nt][i]) : c[nt][i] + d[nt][i];
+                        r[i] = c[nt][i] + d[nt][i];
                     const float2 X = *reinterpret_cast<const float2 *>(xsum + g * 32 + nt * 8 + 2 * tig);
                     acc[nt][0] = fmaf(b_lo, X.x, fmaf(s_lo, r[0], acc[nt][0]));
                     acc[nt][1] = fmaf(b_lo, X.y, fmaf(s_lo, r[1], acc[nt][1]));

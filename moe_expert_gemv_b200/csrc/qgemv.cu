@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
     pdl_trigger();
     const int ctid = threadIdx.x;
     constexpr int KIND = BITS == 4 ? kPermS4 : 8;
-    constexpr float kCodeScale = BITS == 4 ? kSub20 : kSub24;   // undoes the subnormal codes
+    constexpr float kCodeScale = BITS == 4 ? kCode4 : kCode8;   // undoes the subnormal codes
     if (ROT)
         stage_x_groups<KIND, true>(xs, xsum, L.G, a.B, a.x, a.K, ctid, QG_CT, 8, a.signs, xs_lo);
     else if ((reinterpret_cast<uintptr_t>(a.x) & 15u) == 0)
