@@ -26,10 +26,13 @@
 //     projection by the unit's 64 h values.  The gate/up -> down dependency
 //     never leaves the cluster.
 //   * Each CTA adds its weighted down rows of all its units in shared memory
-//     and then into an fp32 layer accumulator with one vector atomic per four
-//     rows; one grid-wide arrival counter per layer then says the layer's
-//     output is complete, and the next layer starts (its input would be this
-//     layer's output in a real model).
+//     and then into an fp32 layer accumulator with one vector reduction per
+//     four rows; the thread that issued it then increments a grid-wide
+//     arrival counter with release semantics, so no CTA-wide barrier or fence
+//     sits between the last work item and the arrival.  When the counter
+//     shows every reduction of the layer, the layer's output is complete and
+//     the next layer starts (its input would be this layer's output in a
+//     real model).
 //   * One producer thread streams the CTA's weights as ~12.7 KB bulk copies
 //     (every copy is one contiguous block of the packed layer) through a
 //     shared-memory ring, in the order the consumers use them: the shared
@@ -38,7 +41,13 @@
 //     warp itself computes the top-k, since it is the one waiting for it.
 //   * 16 consumer warps in 4 groups; work item k of a layer goes to group
 //     k % 4 (gate/up items: the 4 warps split K; down items: the 4 warps
-//     split the rows).
+//     split the rows).  Consumers hand partial sums over through shared
+//     memory and an mbarrier and move on: an exchange warp adds the router
+//     partials and sends the CTA's logits to the cluster, and adds each
+//     unit's gate/up partials, applies SwiGLU and sends the h values (four
+//     8-byte stores and one 4-byte store per destination CTA).  Remote
+//     stores wait on their acknowledgement; kept on one warp, that latency
+//     never holds a consumer group.
 //
 // The fp32 atomics make the last bits of a layer output depend on the order
 // in which clusters finish; routing, h and every per-CTA sum do not.
@@ -57,11 +66,13 @@ constexpr int DC_GROUPS = 4;                  // consumer groups
 constexpr int DC_GW = 4;                      // warps per group
 constexpr int DC_CW = DC_GROUPS * DC_GW;      // consumer warps
 constexpr int DC_CT = DC_CW * 32;             // consumer threads
-constexpr int DC_THREADS = DC_CT + 32;        // + the producer warp
+constexpr int DC_PW = DC_CW;                  // producer warp
+constexpr int DC_XW = DC_CW + 1;              // first exchange warp
+constexpr int DC_XN = 4;                      // exchange warps
+constexpr int DC_THREADS = DC_CT + 32 * (1 + DC_XN);   // + producer and exchange warps
 constexpr int DC_MAX_UNITS = 16;              // units per cluster and layer
 constexpr int DC_MAX_STAGES = 16;
 constexpr int BAR_ALL = 1;                    // named barrier of all consumer threads
-constexpr int BAR_GROUP0 = 2;                 // 2..5: one per consumer group
 
 // control words of the workspace
 enum { C_ARRIVE = 0, C_ABORT, C_EXIT, C_WORDS };
@@ -149,8 +160,20 @@ __device__ __forceinline__ void unit_of(int s, const Units &u, int c, int NC, in
 
 // ------------------------------------------------------- shared memory --
 struct DcLayout {
-    size_t router_off, xraw_off, xs4_off, xs8_off, xsum_off, logit_off, topk_off, hfrag_off,
-        hsum_off, ypart_off, red_off, gured_off, bar_off, ring_off, total;
+    size_t router_off, xs4_off, xs8_off, xsum_off, logit_off, topk_off, unit_off, hfrag_off,
+        hsum_off, ypart_off, red_off, gupart_off, bar_off, ring_off, total;
+};
+
+// barriers (indices into the barrier array after the ring's full/empty pairs)
+enum {
+    DB_RFULL = 0,        // router rows of the layer landed
+    DB_REMPTY,           // router rows consumed
+    DB_TOPK,             // top-k of the layer in s_idx / s_wt
+    DB_LOGIT,            // the cluster's logits (one arrival per CTA)
+    DB_RED,              // router partials of every consumer warp
+    DB_H,                // + unit: the unit's h from every CTA of the cluster
+    DB_GU = DB_H + DC_MAX_UNITS,   // + unit: gate/up partials of the unit's warps
+    DB_COUNT = DB_GU + DC_MAX_UNITS
 };
 
 __host__ __device__ inline size_t dc_take(size_t *off, size_t n, size_t align)
@@ -166,18 +189,19 @@ __host__ __device__ inline DcLayout dc_layout(const PackDims &p, int NS)
     DcLayout L;
     size_t off = 0;
     L.router_off = dc_take(&off, p.rb_bytes, 128);
-    L.xraw_off = dc_take(&off, (size_t)p.H * 2, 16);
     L.xs4_off = dc_take(&off, (size_t)p.GH * 2 * 4 * 16, 16);
     L.xs8_off = dc_take(&off, (size_t)p.GH * 2 * 4 * 16, 16);
     L.xsum_off = dc_take(&off, (size_t)p.GH * 8 * 4, 16);
     L.logit_off = dc_take(&off, (size_t)p.E * 4, 16);
     L.topk_off = dc_take(&off, 32 * 4 * 2, 16);
+    L.unit_off = dc_take(&off, (size_t)2 * DC_MAX_UNITS * 4, 16);   // (slot j, group g) per unit
     L.hfrag_off = dc_take(&off, (size_t)DC_MAX_UNITS * 256, 16);
     L.hsum_off = dc_take(&off, (size_t)DC_MAX_UNITS * DC_CLUSTER * 4, 16);
     L.ypart_off = dc_take(&off, (size_t)DC_GROUPS * p.Hc * 4, 16);
-    L.red_off = dc_take(&off, (size_t)DC_CW * 16 * 4, 16);        // router partials
-    L.gured_off = dc_take(&off, (size_t)2 * DC_CW * 16 * 4, 16);  // gate/up partials, 2 buffers
-    L.bar_off = dc_take(&off, (size_t)(2 * DC_MAX_STAGES + 4 + DC_MAX_UNITS) * 8, 8);
+    L.red_off = dc_take(&off, (size_t)DC_CW * 16 * 4, 16);   // router partials
+    // gate/up partials [unit][warp of the group][gate 8 | up 8]
+    L.gupart_off = dc_take(&off, (size_t)DC_MAX_UNITS * DC_GW * 16 * 4, 16);
+    L.bar_off = dc_take(&off, (size_t)(2 * DC_MAX_STAGES + DB_COUNT) * 8, 8);
     L.ring_off = dc_take(&off, (size_t)NS * p.st_bytes, 128);
     L.total = off;
     return L;
@@ -219,9 +243,29 @@ __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v)
 {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
-__device__ __forceinline__ void st_cluster_u16(uint32_t addr, unsigned short v)
+__device__ __forceinline__ void st_cluster_v4f32(uint32_t addr, float4 v)
 {
-    asm volatile("st.shared::cluster.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x),
+                 "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ void st_cluster_v2u32(uint32_t addr, uint32_t a, uint32_t b)
+{
+    asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b)
+                 : "memory");
+}
+// fire-and-forget vector add (no value returned, so the thread does not wait)
+__device__ __forceinline__ void red_add_v4(float4 *p, float4 v)
+{
+    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x),
+                 "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+// increment with release semantics at GPU scope: this thread's earlier
+// writes (and reductions) are visible to whoever acquires the new value
+__device__ __forceinline__ void red_release_add(unsigned *p, unsigned v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 // arrive on an mbarrier of a CTA of the cluster; orders this thread's
 // earlier shared::cluster stores before the arrival
@@ -328,16 +372,10 @@ __device__ __forceinline__ float2 sb_word(const unsigned char *p)
     return __half22float2(*reinterpret_cast<const __half2 *>(p));   // (scale, bias)
 }
 
-// position (in halves) of intermediate index k (0..63) of a unit, column col
-// (0: hi, 1: lo) in the down projection's B fragments [hh][col][tig][8], in
-// the x order of mma_group_s4
-__device__ __forceinline__ int hfrag_pos(int k, int col)
-{
-    const int tig = k >> 4, p = k & 15;
-    const int i = xperm_s4_inv(p);
-    const int hh = i >> 3, e = i & 7;
-    return (((hh * 2 + col) * 4 + tig) * 8) + e;
-}
+// The h of a unit (64 intermediate indices k, fp16 hi and lo columns) sits in
+// hfrag[unit] as the down projection's B fragments [hh][col][tig][8], in the x
+// order of mma_group_s4: index k = 16 tig + xperm_s4(8 hh + e) at slot
+// ((hh * 2 + col) * 4 + tig) * 8 + e.
 
 // ------------------------------------------------------------------ kernel --
 __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS, 1)
@@ -347,22 +385,25 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
     const PackDims P = pack_dims(a.E, a.H, a.I);
     const DcLayout L = dc_layout(P, a.NS);
     unsigned char *rbuf = smem + L.router_off;
-    uint4 *xraw = reinterpret_cast<uint4 *>(smem + L.xraw_off);
     uint4 *xs4 = reinterpret_cast<uint4 *>(smem + L.xs4_off);
     uint4 *xs8 = reinterpret_cast<uint4 *>(smem + L.xs8_off);
     float *xsum = reinterpret_cast<float *>(smem + L.xsum_off);
     float *s_logit = reinterpret_cast<float *>(smem + L.logit_off);
     int *s_idx = reinterpret_cast<int *>(smem + L.topk_off);
     float *s_wt = reinterpret_cast<float *>(smem + L.topk_off + 32 * 4);
+    int *s_uj = reinterpret_cast<int *>(smem + L.unit_off);   // unit -> expert slot j (K: shared)
+    int *s_ug = s_uj + DC_MAX_UNITS;                          // unit -> group of 64 indices
     __half *hfrag = reinterpret_cast<__half *>(smem + L.hfrag_off);   // [unit][128]
     float *hsum = reinterpret_cast<float *>(smem + L.hsum_off);       // [unit][8]
     float *ypart = reinterpret_cast<float *>(smem + L.ypart_off);     // [group][Hc]
-    float *red = reinterpret_cast<float *>(smem + L.red_off);
-    float *gured = reinterpret_cast<float *>(smem + L.gured_off);
+    float *red = reinterpret_cast<float *>(smem + L.red_off);         // [warp][16]
+    float *gupart = reinterpret_cast<float *>(smem + L.gupart_off);   // [unit][wq][16]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
     uint64_t *full = bars, *empty = bars + DC_MAX_STAGES;
-    uint64_t *rfull = bars + 2 * DC_MAX_STAGES, *rempty = rfull + 1, *topk_bar = rfull + 2,
-             *logit_bar = rfull + 3, *hbar = rfull + 4;
+    uint64_t *db = bars + 2 * DC_MAX_STAGES;
+    uint64_t *rfull = db + DB_RFULL, *rempty = db + DB_REMPTY, *topk_bar = db + DB_TOPK,
+             *logit_bar = db + DB_LOGIT, *red_bar = db + DB_RED, *hbar = db + DB_H,
+             *gubar = db + DB_GU;
     unsigned char *ring = smem + L.ring_off;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -382,9 +423,22 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
         mbar_init(rempty, 1);
         mbar_init(topk_bar, 1);
         mbar_init(logit_bar, DC_CLUSTER);
-        for (int s = 0; s < DC_MAX_UNITS; ++s)
+        mbar_init(red_bar, DC_CW);
+        for (int s = 0; s < DC_MAX_UNITS; ++s) {
             mbar_init(&hbar[s], DC_CLUSTER);
+            mbar_init(&gubar[s], DC_GW);
+        }
         mbar_init_fence();
+    }
+    // columns 1..7 of the x group sums stay zero (one input column)
+    for (int t = threadIdx.x; t < P.GH * 8; t += blockDim.x)
+        xsum[t] = 0.f;
+    // the cluster's units are the same in every layer
+    if (threadIdx.x < U.nu) {
+        int j, g;
+        unit_of(threadIdx.x, U, cl, NC, K, P.GI, &j, &g);
+        s_uj[threadIdx.x] = j;
+        s_ug[threadIdx.x] = g;
     }
     // every CTA of the cluster has initialised its barriers before anyone
     // signals one remotely
@@ -392,7 +446,7 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
     // the workspace may still be in use by the previous launch on the stream
     pdl_wait();
 
-    if (warp == DC_CW) {
+    if (warp == DC_PW) {
         // ====================================================== producer
         const uint64_t pol = l2_evict_first_policy();
         bool ok = true;
@@ -416,16 +470,12 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
         for (int l = 0; l < a.L; ++l) {
             const unsigned char *lp = static_cast<const unsigned char *>(a.layer[l]);
             if (lane == 0 && ok) {
-                int j, g;
                 for (int s = 0; s < U.ns; ++s) {   // shared gate/up
-                    unit_of(s, U, cl, NC, K, P.GI, &j, &g);
-                    issue(lp + pack_copy_off(P, a.E, g, rank, 0));
-                    issue(lp + pack_copy_off(P, a.E, g, rank, 1));
+                    issue(lp + pack_copy_off(P, a.E, s_ug[s], rank, 0));
+                    issue(lp + pack_copy_off(P, a.E, s_ug[s], rank, 1));
                 }
-                for (int s = 0; s < U.ns; ++s) {   // shared down
-                    unit_of(s, U, cl, NC, K, P.GI, &j, &g);
-                    issue(lp + pack_copy_off(P, a.E, g, rank, 2));
-                }
+                for (int s = 0; s < U.ns; ++s)     // shared down
+                    issue(lp + pack_copy_off(P, a.E, s_ug[s], rank, 2));
                 // the next layer's input into L2 (where a real model's previous
                 // layer output would be), and its router rows once this
                 // layer's are consumed
@@ -465,30 +515,63 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                     for (int qq = 0; qq < 4; ++qq)
                         if (!taken[qq])
                             a.logits[(size_t)l * a.E + lane + 32 * qq] = v[qq];
+                // each lane sorts its 4 candidates (key descending, lower
+                // index first on equal keys); the warp then pops the largest
+                // head K times
+                unsigned hk[4];
+                int hi[4];
+                float hv[4];
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    hk[qq] = taken[qq] ? 0u : key[qq];
+                    hi[qq] = taken[qq] ? 0x7fffffff : lane + 32 * qq;
+                    hv[qq] = v[qq];
+                }
+                auto cx = [&](int x, int y) {   // order (x, y)
+                    const bool sw = hk[y] > hk[x] || (hk[y] == hk[x] && hi[y] < hi[x]);
+                    if (sw) {
+                        const unsigned tk = hk[x];
+                        const int ti = hi[x];
+                        const float tv = hv[x];
+                        hk[x] = hk[y], hi[x] = hi[y], hv[x] = hv[y];
+                        hk[y] = tk, hi[y] = ti, hv[y] = tv;
+                    }
+                };
+                cx(0, 1), cx(2, 3), cx(0, 2), cx(1, 3), cx(1, 2);
                 float my_v = 0.f;
                 int my_i = 0;
+                int nxt = U.ns;   // next routed unit whose gate/up copies are due
                 for (int jj = 0; jj < K; ++jj) {
-                    unsigned bk = 0u;
-                    int be = 0x7fffffff;
-                    float bv = 0.f;
-#pragma unroll
-                    for (int qq = 0; qq < 4; ++qq)
-                        if (!taken[qq] && key[qq] > bk) {   // strict: the lower index wins ties
-                            bk = key[qq];
-                            be = lane + 32 * qq;
-                            bv = v[qq];
-                        }
-                    const unsigned mk = __reduce_max_sync(0xffffffffu, bk);
-                    const int win = (int)__reduce_min_sync(0xffffffffu,
-                                                           (unsigned)(bk == mk ? be : 0x7fffffff));
-                    const float wv = __shfl_sync(0xffffffffu, bv, win & 31);
-#pragma unroll
-                    for (int qq = 0; qq < 4; ++qq)
-                        if (win == lane + 32 * qq)
-                            taken[qq] = true;
+                    const unsigned mk = __reduce_max_sync(0xffffffffu, hk[0]);
+                    // one lane holds the maximum unless keys tie: then the
+                    // lowest index among the tied heads wins
+                    const unsigned tied = __ballot_sync(0xffffffffu, hk[0] == mk);
+                    const int wl = __popc(tied) == 1
+                                       ? __ffs(tied) - 1
+                                       : (int)(__reduce_min_sync(0xffffffffu,
+                                                                 (unsigned)(hk[0] == mk ? hi[0] : 0x7fffffff)) &
+                                               31u);
+                    const int win = __shfl_sync(0xffffffffu, hi[0], wl);
+                    const float wv = __shfl_sync(0xffffffffu, hv[0], wl);
+                    if (lane == wl) {   // pop the head
+                        hk[0] = hk[1], hi[0] = hi[1], hv[0] = hv[1];
+                        hk[1] = hk[2], hi[1] = hi[2], hv[1] = hv[2];
+                        hk[2] = hk[3], hi[2] = hi[3], hv[2] = hv[3];
+                        hk[3] = 0u, hi[3] = 0x7fffffff, hv[3] = 0.f;
+                    }
                     if (lane == jj) {
                         my_v = wv;
                         my_i = win;
+                    }
+                    // the jj-th expert is final: its units' gate/up copies go
+                    // out now, while the rest of the top-k is still being found
+                    // (units come in slot order)
+                    if (lane == 0 && ok) {
+                        const int e = (win >= 0 && win < a.E) ? win : 0;
+                        for (; nxt < U.nu && s_uj[nxt] == jj; ++nxt) {
+                            issue(lp + pack_copy_off(P, e, s_ug[nxt], rank, 0));
+                            issue(lp + pack_copy_off(P, e, s_ug[nxt], rank, 1));
+                        }
                     }
                 }
                 const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
@@ -512,19 +595,9 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                 if (lane == 0)
                     mbar_arrive(topk_bar);   // the routed down items may read s_wt
             }
-            if (lane == 0 && ok) {
-                int j, g;
-                for (int s = U.ns; s < U.nu; ++s) {   // routed gate/up
-                    unit_of(s, U, cl, NC, K, P.GI, &j, &g);
-                    const int e = s_idx[j];
-                    issue(lp + pack_copy_off(P, e, g, rank, 0));
-                    issue(lp + pack_copy_off(P, e, g, rank, 1));
-                }
-                for (int s = U.ns; s < U.nu; ++s) {   // routed down
-                    unit_of(s, U, cl, NC, K, P.GI, &j, &g);
-                    issue(lp + pack_copy_off(P, s_idx[j], g, rank, 2));
-                }
-            }
+            if (lane == 0 && ok)   // the routed down copies
+                for (int s = U.ns; s < U.nu; ++s)
+                    issue(lp + pack_copy_off(P, s_idx[s_uj[s]], s_ug[s], rank, 2));
             ok = __shfl_sync(0xffffffffu, ok, 0);
             __syncwarp();
         }
@@ -536,6 +609,93 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
             }
         }
         __syncwarp();
+    } else if (warp >= DC_XW) {
+        // ====================================================== exchange
+        // Finishes what the consumer warps hand over, so that they never wait
+        // on distributed-shared-memory traffic: the CTA's logits (first
+        // exchange warp) and, unit by unit, SwiGLU and the unit's h, sent to
+        // every CTA of the cluster (unit s by exchange warp s % DC_XN: a
+        // send takes about a microsecond, so several run at once).
+        const int xw = warp - DC_XW;
+        const int Rr = P.Rr;
+        bool ok = true;
+        for (int l = 0; l < a.L && ok; ++l) {
+            if (xw == 0) {
+                ok = __all_sync(0xffffffffu, wait_bar(a, red_bar, l & 1));
+                if (!ok)
+                    break;
+                if (lane == 0)
+                    mbar_arrive(rempty);   // the router rows are consumed
+                {
+                    // row lane & 15, half of the consumer warps each
+                    const int row = lane & 15, w0 = (lane >> 4) * (DC_CW / 2);
+                    float v = 0.f;
+#pragma unroll
+                    for (int w = 0; w < DC_CW / 2; ++w)
+                        v += red[(w0 + w) * 16 + row];
+                    v += __shfl_xor_sync(0xffffffffu, v, 16);
+                    if (lane < Rr)
+                        s_logit[Rr * rank + lane] = v;
+                }
+                __syncwarp();
+                if (lane < DC_CLUSTER) {
+                    const float *mine = s_logit + Rr * rank;
+                    const uint32_t tb = mapa_rank(smem_u32(mine), lane);
+                    if ((Rr & 3) == 0) {
+                        for (int i = 0; i < Rr; i += 4)
+                            st_cluster_v4f32(tb + 4 * i, *reinterpret_cast<const float4 *>(mine + i));
+                    } else {
+                        for (int i = 0; i < Rr; ++i)
+                            st_cluster_f32(tb + 4 * i, mine[i]);
+                    }
+                    mbar_arrive_remote(mapa_rank(smem_u32(logit_bar), lane));
+                }
+            }
+            for (int s = xw; s < U.nu; s += DC_XN) {
+                ok = __all_sync(0xffffffffu, wait_bar(a, &gubar[s], l & 1));
+                if (!ok)
+                    break;
+                float h = 0.f;
+                if (lane < 8) {
+                    float gs = 0.f, us = 0.f;
+#pragma unroll
+                    for (int w = 0; w < DC_GW; ++w) {
+                        gs += gupart[((size_t)s * DC_GW + w) * 16 + lane];
+                        us += gupart[((size_t)s * DC_GW + w) * 16 + 8 + lane];
+                    }
+                    h = gs / (1.f + expf(-gs)) * us;
+                }
+                const __half hh = __float2half_rn(h);
+                const __half hl = __float2half_rn(h - __half2float(hh));
+                float part = __half2float(hh) + __half2float(hl);
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                part += __shfl_xor_sync(0xffffffffu, part, 2);
+                part += __shfl_xor_sync(0xffffffffu, part, 4);
+                const unsigned bh = __half_as_ushort(hh), bl = __half_as_ushort(hl);
+                unsigned vh[8], vl[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    vh[i] = __shfl_sync(0xffffffffu, bh, i);
+                    vl[i] = __shfl_sync(0xffffffffu, bl, i);
+                }
+                if (lane < DC_CLUSTER) {
+                    // the CTA's 8 indices k = 8 rank + j sit, per (hh, column),
+                    // in 4 consecutive fragment slots: j = hh + (0, 4, 2, 6)
+                    const uint32_t tb = mapa_rank(smem_u32(hfrag + (size_t)s * 128), lane);
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const int pos_hi = ((hf * 2 + 0) * 4 + (rank >> 1)) * 8 + 4 * (rank & 1);
+                        const int pos_lo = ((hf * 2 + 1) * 4 + (rank >> 1)) * 8 + 4 * (rank & 1);
+                        st_cluster_v2u32(tb + 2 * pos_hi, vh[hf] | (vh[hf + 4] << 16),
+                                         vh[hf + 2] | (vh[hf + 6] << 16));
+                        st_cluster_v2u32(tb + 2 * pos_lo, vl[hf] | (vl[hf + 4] << 16),
+                                         vl[hf + 2] | (vl[hf + 6] << 16));
+                    }
+                    st_cluster_f32(mapa_rank(smem_u32(hsum + s * DC_CLUSTER + rank), lane), part);
+                    mbar_arrive_remote(mapa_rank(smem_u32(&hbar[s]), lane));
+                }
+            }
+        }
     } else {
         // ====================================================== consumers
         const int ctid = threadIdx.x;
@@ -563,11 +723,11 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
         };
 
         // ---------------------------------------- one gate/up work item
-        // gate/up partials alternate between two buffers from item to item of a
-        // group, so a warp that runs ahead into the next item cannot overwrite
-        // what the group's first warp is still reading
-        int gu_buf = 0;
-        auto do_gu = [&](int seq0, int slot, int l) {
+        // Each warp of the group takes a quarter of K; its partial sums of the
+        // unit's 8 gate and 8 up rows go to gupart[slot] and the exchange warp
+        // finishes the unit (SwiGLU, h to the cluster), so the group moves on
+        // at once.
+        auto do_gu = [&](int seq0, int slot) {
             const int sa = seq0 % NS, sb = (seq0 + 1) % NS;
             // the lanes of a warp decide together: the mma below is warp-collective
             const bool good = __all_sync(0xffffffffu, ok && wait_bar(a, &full[sa], (seq0 / NS) & 1) &&
@@ -608,56 +768,14 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                 mbar_arrive(&empty[sa]);
                 mbar_arrive(&empty[sb]);
             }
-            float *gub = gured + (size_t)gu_buf * DC_CW * 16;
-            gu_buf ^= 1;
-            float *gr = gub + (size_t)warp * 16;
+            float *gr = gupart + ((size_t)slot * DC_GW + wq) * 16;
             if (tig == 0) {
                 gr[gid] = ag * kCode4 + bg;       // gate row gid
                 gr[8 + gid] = au * kCode4 + bu;   // up row gid
             }
-            named_bar_sync(BAR_GROUP0 + q, DC_GW * 32);
-            if (wq == 0) {
-                // SwiGLU of the CTA's 8 intermediate indices, then to every CTA
-                // of the cluster as fp16 (hi, lo) fragments + their sum
-                const float *g0r = gub + (size_t)(q * DC_GW) * 16;
-                float h = 0.f;
-                if (lane < 8) {
-                    float gs = 0.f, us = 0.f;
-#pragma unroll
-                    for (int w = 0; w < DC_GW; ++w) {
-                        gs += g0r[w * 16 + lane];
-                        us += g0r[w * 16 + 8 + lane];
-                    }
-                    h = gs / (1.f + expf(-gs)) * us;
-                }
-                const __half hh = __float2half_rn(h);
-                const __half hl = __float2half_rn(h - __half2float(hh));
-                float part = __half2float(hh) + __half2float(hl);
-                part += __shfl_xor_sync(0xffffffffu, part, 1);
-                part += __shfl_xor_sync(0xffffffffu, part, 2);
-                part += __shfl_xor_sync(0xffffffffu, part, 4);
-                const unsigned short bh = __half_as_ushort(hh), bl = __half_as_ushort(hl);
-                unsigned short vh[8], vl[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    vh[i] = (unsigned short)__shfl_sync(0xffffffffu, (unsigned)bh, i);
-                    vl[i] = (unsigned short)__shfl_sync(0xffffffffu, (unsigned)bl, i);
-                }
-                part = __shfl_sync(0xffffffffu, part, 0);
-                if (lane < DC_CLUSTER) {
-                    const uint32_t base = smem_u32(hfrag + (size_t)slot * 128);
-                    const uint32_t tbase = mapa_rank(base, lane);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int k = 8 * rank + i;
-                        st_cluster_u16(tbase + 2 * hfrag_pos(k, 0), vh[i]);
-                        st_cluster_u16(tbase + 2 * hfrag_pos(k, 1), vl[i]);
-                    }
-                    st_cluster_f32(mapa_rank(smem_u32(hsum + slot * DC_CLUSTER + rank), lane), part);
-                    mbar_arrive_remote(mapa_rank(smem_u32(&hbar[slot]), lane));
-                }
-                (void)l;
-            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&gubar[slot]);   // release: the partials above
             if (!good)
                 ok = false;
         };
@@ -669,7 +787,7 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
             bool good = __all_sync(0xffffffffu, ok && wait_bar(a, &full[st], (seq / NS) & 1) &&
                                                     wait_bar_cluster(a, &hbar[slot], l & 1));
             float w = 1.f;
-            if (good && j < K) {
+            if (good && j < K) {   // a routed unit: its router weight
                 good = __all_sync(0xffffffffu, wait_bar(a, topk_bar, l & 1));
                 w = s_wt[j];
             }
@@ -710,24 +828,56 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                 ok = false;
         };
 
+        // every consumer thread with t < Hc / 4 adds one float4 of the CTA's
+        // output rows per layer and then one release increment of the
+        // arrival counter: the layer is complete once the counter reaches
+        // G * Hc / 4 per layer
+        const unsigned nred = (unsigned)(Hc / 4);
+
         for (int l = 0; l < a.L; ++l) {
             // ---- the previous layer's output is complete in every CTA
             if (l > 0) {
-                if (ctid == 0 && !spin_until(a, ctl + C_ARRIVE, (unsigned)(l * G)))
+                if (ctid == 0 && !spin_until(a, ctl + C_ARRIVE, (unsigned)l * G * nred))
                     ok = false;
                 named_bar_sync(BAR_ALL, DC_CT);
             }
-            // ---- x of this layer: 16-byte loads, then both fragment orders
+            // ---- x of this layer straight from memory into both fragment
+            // orders: thread (g, half, tig) loads x[64 g + 16 tig .. + 15]
             {
                 const uint4 *xg = reinterpret_cast<const uint4 *>(a.x + (size_t)l * H);
-                for (int t = ctid; t < H / 8; t += DC_CT)
-                    xraw[t] = __ldcg(xg + t);
-                named_bar_sync(BAR_ALL, DC_CT);
-                const __half *xh = reinterpret_cast<const __half *>(xraw);
-                stage_x<kPermS4>(xs4, xsum, GH, 1, 1,
-                                 [&](int, int, int k) { return __half2float(xh[k]); }, ctid, DC_CT);
-                stage_x<8>(xs8, nullptr, GH, 1, 1,
-                           [&](int, int, int k) { return __half2float(xh[k]); }, ctid, DC_CT);
+                for (int t0 = 0; t0 < GH * 8; t0 += DC_CT) {
+                    const int t = t0 + ctid;
+                    const bool act = t < GH * 8;
+                    const int g = t >> 3, hs = (t >> 2) & 1, tg = t & 3;
+                    uint4 raw[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+                    if (act) {
+                        raw[0] = __ldcg(xg + g * 8 + tg * 2);
+                        raw[1] = __ldcg(xg + g * 8 + tg * 2 + 1);
+                    }
+                    const __half *xv = reinterpret_cast<const __half *>(raw);
+                    uint32_t w4[4], w8[4];
+                    float sum = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const __half a0 = hs ? xv[xperm(kPermS4, 8 + 2 * i)] : xv[xperm(kPermS4, 2 * i)];
+                        const __half a1 =
+                            hs ? xv[xperm(kPermS4, 9 + 2 * i)] : xv[xperm(kPermS4, 2 * i + 1)];
+                        const __half b0 = hs ? xv[xperm(8, 8 + 2 * i)] : xv[xperm(8, 2 * i)];
+                        const __half b1 = hs ? xv[xperm(8, 9 + 2 * i)] : xv[xperm(8, 2 * i + 1)];
+                        w4[i] = h2_as_u32(__halves2half2(a0, a1));
+                        w8[i] = h2_as_u32(__halves2half2(b0, b1));
+                        sum += __half2float(a0) + __half2float(a1);
+                    }
+                    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+                    sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+                    if (act) {
+                        xs4[(g * 2 + hs) * 4 + tg] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        xs8[(g * 2 + hs) * 4 + tg] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+                        if ((t & 7) == 0)
+                            xsum[g * 8] = sum;
+                    }
+                }
                 named_bar_sync(BAR_ALL, DC_CT);
             }
             // ---- router: this CTA's Rr rows, K split over the 16 warps
@@ -765,30 +915,15 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                 }
                 if (!good)
                     ok = false;
+                // the warp's partials to the exchange warp (which also frees
+                // the router rows for the next layer)
                 if (tig == 0) {
                     red[warp * 16 + gid] = acc_lo * kCode8 + b_lo;
                     red[warp * 16 + 8 + gid] = acc_hi * kCode8 + b_hi;
                 }
-                named_bar_sync(BAR_ALL, DC_CT);
-                if (ctid == 0)
-                    mbar_arrive(rempty);   // the producer may load the next layer's rows
-                if (warp == 0) {
-                    if (lane < 16) {
-                        float v = 0.f;
-                        for (int w = 0; w < DC_CW; ++w)
-                            v += red[w * 16 + lane];
-                        if (lane < Rr)
-                            s_logit[Rr * rank + lane] = v;
-                    }
-                    __syncwarp();
-                    if (lane < DC_CLUSTER) {   // this CTA's logits to every CTA of the cluster
-                        for (int i = 0; i < Rr; ++i) {
-                            const uint32_t adr = smem_u32(s_logit + Rr * rank + i);
-                            st_cluster_f32(mapa_rank(adr, lane), s_logit[Rr * rank + i]);
-                        }
-                        mbar_arrive_remote(mapa_rank(smem_u32(logit_bar), lane));
-                    }
-                }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(red_bar);
             }
             // ---- the previous layer's output to fp16 (off the critical path)
             if (l > 0)
@@ -812,13 +947,10 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                         slot = U.ns + m;
                         seq = base + 3 * U.ns + 2 * U.nr + m;
                     }
-                    if (gu) {
-                        do_gu(seq, slot, l);
-                    } else {
-                        int j, g;
-                        unit_of(slot, U, cl, NC, K, P.GI, &j, &g);
-                        do_dn(seq, slot, j, l);
-                    }
+                    if (gu)
+                        do_gu(seq, slot);
+                    else
+                        do_dn(seq, slot, s_uj[slot], l);
                 }
             }
             // ---- this CTA's rows of the layer output into the accumulator
@@ -837,17 +969,13 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                         reinterpret_cast<float4 *>(ypart + (size_t)g * Hc)[t] =
                             make_float4(0.f, 0.f, 0.f, 0.f);
                     }
-                    atomicAdd(reinterpret_cast<float4 *>(acc) + t, v);
+                    red_add_v4(reinterpret_cast<float4 *>(acc) + t, v);
+                    red_release_add(ctl + C_ARRIVE, 1u);   // ordered after the add above
                 }
-            }
-            named_bar_sync(BAR_ALL, DC_CT);
-            if (ctid == 0) {
-                __threadfence();
-                atomicAdd(ctl + C_ARRIVE, 1u);
             }
         }
         // ---- the last layer's output
-        if (ctid == 0 && !spin_until(a, ctl + C_ARRIVE, (unsigned)(a.L * G)))
+        if (ctid == 0 && !spin_until(a, ctl + C_ARRIVE, (unsigned)a.L * G * nred))
             ok = false;
         named_bar_sync(BAR_ALL, DC_CT);
         convert_slice(a.L - 1);

@@ -2,10 +2,10 @@
 instead of hanging, and the context stays usable.
 
 The fused decode's layer barrier waits until an arrival counter in its
-workspace reaches (layers done) x (CTAs).  The test presets that counter to
-2^32 - 1: after the first layer's arrivals it has wrapped to just below the
-target of the second layer, so that wait can never complete (a flag nothing
-sets).  With the wait limit lowered to 1 ms the launch must return, report
+workspace reaches (layers done) x (arrivals per layer).  The test presets that
+counter to 2^32 - 1: after the first layer's arrivals it has wrapped to just
+below the target of the second layer, so that wait can never complete (a
+flag nothing sets).  With the wait limit lowered to 1 ms the launch must return, report
 QMOE_DEV_TIMEOUT, and leave its control words at zero; after the workspace is
 zeroed again, the same call gives the oracle's results."""
 import numpy as np
