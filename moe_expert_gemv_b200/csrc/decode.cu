@@ -68,7 +68,7 @@ constexpr int DC_CW = DC_GROUPS * DC_GW;      // consumer warps
 constexpr int DC_CT = DC_CW * 32;             // consumer threads
 constexpr int DC_PW = DC_CW;                  // producer warp
 constexpr int DC_XW = DC_CW + 1;              // first exchange warp
-constexpr int DC_XN = 4;                      // exchange warps
+constexpr int DC_XN = 3;                      // exchange warps (20 warps in all: 96 registers)
 constexpr int DC_THREADS = DC_CT + 32 * (1 + DC_XN);   // + producer and exchange warps
 constexpr int DC_MAX_UNITS = 16;              // units per cluster and layer
 constexpr int DC_MAX_STAGES = 16;
@@ -161,7 +161,7 @@ __device__ __forceinline__ void unit_of(int s, const Units &u, int c, int NC, in
 // ------------------------------------------------------- shared memory --
 struct DcLayout {
     size_t router_off, xs4_off, xs8_off, xsum_off, logit_off, topk_off, unit_off, hfrag_off,
-        hsum_off, ypart_off, red_off, gupart_off, bar_off, ring_off, total;
+        hsum_off, ypart_off, red_off, gupart_off, bar_off, arm_off, ring_off, total;
 };
 
 // barriers (indices into the barrier array after the ring's full/empty pairs)
@@ -173,7 +173,8 @@ enum {
     DB_RED,              // router partials of every consumer warp
     DB_H,                // + unit: the unit's h from every CTA of the cluster
     DB_GU = DB_H + DC_MAX_UNITS,   // + unit: gate/up partials of the unit's warps
-    DB_COUNT = DB_GU + DC_MAX_UNITS
+    DB_ROUND = DB_GU + DC_MAX_UNITS,   // + j: the j-th expert of the top-k is known
+    DB_COUNT = DB_ROUND + 16
 };
 
 __host__ __device__ inline size_t dc_take(size_t *off, size_t n, size_t align)
@@ -202,6 +203,7 @@ __host__ __device__ inline DcLayout dc_layout(const PackDims &p, int NS)
     // gate/up partials [unit][warp of the group][gate 8 | up 8]
     L.gupart_off = dc_take(&off, (size_t)DC_MAX_UNITS * DC_GW * 16 * 4, 16);
     L.bar_off = dc_take(&off, (size_t)(2 * DC_MAX_STAGES + DB_COUNT) * 8, 8);
+    L.arm_off = dc_take(&off, (size_t)DC_MAX_STAGES * 4, 16);   // sequence each slot holds
     L.ring_off = dc_take(&off, (size_t)NS * p.st_bytes, 128);
     L.total = off;
     return L;
@@ -366,6 +368,31 @@ __device__ __noinline__ bool spin_until(const DecodeArgs &a, const unsigned *p, 
     return true;
 }
 
+// Bounded wait until a ring slot has been armed for sequence `sq`.
+__device__ __noinline__ bool wait_arm_slow(const DecodeArgs &a, const volatile int *arm, int sq)
+{
+    unsigned *abort = a.ws.ctl + C_ABORT;
+    const unsigned long long t0 = global_timer_ns();
+    for (unsigned n = 1;; ++n) {
+        if (*arm == sq)
+            return true;
+        __nanosleep(20);
+        if ((n & 63u) == 0u) {
+            if (ld_acquire_u32(abort) != 0u)
+                return false;
+            if (global_timer_ns() - t0 > a.wait_ns) {
+                atomicExch(abort, 1u);
+                flag_status(a.status, QMOE_DEV_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ bool wait_arm(const DecodeArgs &a, const volatile int *arm, int sq)
+{
+    return *arm == sq || wait_arm_slow(a, arm, sq);
+}
+
 // ------------------------------------------------------------ helpers --
 __device__ __forceinline__ float2 sb_word(const unsigned char *p)
 {
@@ -388,6 +415,9 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
     uint4 *xs4 = reinterpret_cast<uint4 *>(smem + L.xs4_off);
     uint4 *xs8 = reinterpret_cast<uint4 *>(smem + L.xs8_off);
     float *xsum = reinterpret_cast<float *>(smem + L.xsum_off);
+    // 16 zero bytes (group 0's unused sum columns 4..7), read by lanes whose
+    // B fragment column is not x
+    const uint4 *xzero = reinterpret_cast<const uint4 *>(xsum + 4);
     float *s_logit = reinterpret_cast<float *>(smem + L.logit_off);
     int *s_idx = reinterpret_cast<int *>(smem + L.topk_off);
     float *s_wt = reinterpret_cast<float *>(smem + L.topk_off + 32 * 4);
@@ -400,10 +430,15 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
     float *gupart = reinterpret_cast<float *>(smem + L.gupart_off);   // [unit][wq][16]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
     uint64_t *full = bars, *empty = bars + DC_MAX_STAGES;
+    // ring sequence number each slot has been armed for (written by the
+    // producer before the copy): a consumer first sees its own sequence
+    // there, so it never takes an older phase of the slot's full barrier for
+    // its own when it runs more than one use of the slot ahead
+    volatile int *s_arm = reinterpret_cast<volatile int *>(smem + L.arm_off);
     uint64_t *db = bars + 2 * DC_MAX_STAGES;
     uint64_t *rfull = db + DB_RFULL, *rempty = db + DB_REMPTY, *topk_bar = db + DB_TOPK,
              *logit_bar = db + DB_LOGIT, *red_bar = db + DB_RED, *hbar = db + DB_H,
-             *gubar = db + DB_GU;
+             *gubar = db + DB_GU, *round_bar = db + DB_ROUND;
     unsigned char *ring = smem + L.ring_off;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -418,6 +453,7 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], DC_GW);   // one arrival per warp of the consuming group
+            s_arm[s] = -1;
         }
         mbar_init(rfull, 1);
         mbar_init(rempty, 1);
@@ -428,6 +464,8 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
             mbar_init(&hbar[s], DC_CLUSTER);
             mbar_init(&gubar[s], DC_GW);
         }
+        for (int j = 0; j < 16; ++j)
+            mbar_init(&round_bar[j], 1);
         mbar_init_fence();
     }
     // columns 1..7 of the x group sums stay zero (one input column)
@@ -451,17 +489,46 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
         const uint64_t pol = l2_evict_first_policy();
         bool ok = true;
         int seq = 0;
-        auto issue = [&](const unsigned char *src) {
-            const int st = seq % NS, use = seq / NS;
+        auto issue_to = [&](const unsigned char *src, int st, int use, int sq) {
             if (use > 0 && ok && !wait_bar(a, &empty[st], (use - 1) & 1))
                 ok = false;
             if (ok) {
+                s_arm[st] = sq;
                 mbar_arrive_expect_tx(&full[st], (uint32_t)P.st_bytes);
                 bulk_g2s(ring + (size_t)st * P.st_bytes, src, (uint32_t)P.st_bytes, &full[st], pol);
             }
+        };
+        auto issue = [&](const unsigned char *src) {   // the next copy of the ring
+            issue_to(src, seq % NS, seq / NS, seq);
             ++seq;
         };
-        if (lane == 0) {
+        // A unit's gate and up halves are adjacent in the packed layer: one
+        // copy fills both of their (adjacent) ring slots unless the pair
+        // wraps around the ring.  Fewer, larger copies keep more bytes in
+        // flight per copy the SM's bulk-copy engine holds at once.  The
+        // second slot's full barrier is completed by a plain arrival (its
+        // data is counted on the first).
+        auto issue_pair = [&](const unsigned char *src) {
+            const int st = seq % NS;
+            if (st + 1 == NS) {
+                issue(src);
+                issue(src + P.st_bytes);
+                return;
+            }
+            const int use = seq / NS;
+            if (use > 0 && ok &&
+                !(wait_bar(a, &empty[st], (use - 1) & 1) && wait_bar(a, &empty[st + 1], (use - 1) & 1)))
+                ok = false;
+            if (ok) {
+                s_arm[st] = seq;
+                s_arm[st + 1] = seq + 1;
+                mbar_arrive_expect_tx(&full[st], (uint32_t)(2 * P.st_bytes));
+                bulk_g2s(ring + (size_t)st * P.st_bytes, src, (uint32_t)(2 * P.st_bytes), &full[st], pol);
+                mbar_arrive(&full[st + 1]);
+            }
+            seq += 2;
+        };
+        if (lane == 0) {   // the first layer's router rows
             mbar_arrive_expect_tx(rfull, (uint32_t)P.rb_bytes);
             bulk_g2s_plain(rbuf, static_cast<const unsigned char *>(a.layer[0]) +
                                      pack_router_off(P, rank),
@@ -470,10 +537,8 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
         for (int l = 0; l < a.L; ++l) {
             const unsigned char *lp = static_cast<const unsigned char *>(a.layer[l]);
             if (lane == 0 && ok) {
-                for (int s = 0; s < U.ns; ++s) {   // shared gate/up
-                    issue(lp + pack_copy_off(P, a.E, s_ug[s], rank, 0));
-                    issue(lp + pack_copy_off(P, a.E, s_ug[s], rank, 1));
-                }
+                for (int s = 0; s < U.ns; ++s)     // shared gate/up
+                    issue_pair(lp + pack_copy_off(P, a.E, s_ug[s], rank, 0));
                 for (int s = 0; s < U.ns; ++s)     // shared down
                     issue(lp + pack_copy_off(P, a.E, s_ug[s], rank, 2));
                 // the next layer's input into L2 (where a real model's previous
@@ -493,107 +558,24 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
-            // ---- top-k of this layer (the whole producer warp)
-            if (ok && !wait_bar_cluster(a, logit_bar, l & 1))
-                ok = false;
-            ok = __all_sync(0xffffffffu, ok);
-            {
-                float v[4];
-                unsigned key[4];
-                bool taken[4];
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const int e = lane + 32 * qq;
-                    taken[qq] = e >= a.E;
-                    v[qq] = taken[qq] ? 0.f : s_logit[e];
-                    const unsigned u = __float_as_uint(v[qq]);   // order-preserving key
-                    key[qq] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+            // ---- routed gate/up copies, expert by expert as the exchange
+            // warp's top-k rounds finish (units come in slot order), then the
+            // routed down copies once the whole top-k is known
+            if (lane == 0 && ok) {
+                int nxt = U.ns;
+                for (int jj = 0; jj < K && nxt < U.nu && ok; ++jj) {
+                    if (s_uj[nxt] != jj)
+                        continue;   // no unit of this cluster belongs to the jj-th expert
+                    if (!wait_bar(a, &round_bar[jj], l & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    const int e = s_idx[jj];
+                    for (; nxt < U.nu && s_uj[nxt] == jj; ++nxt)
+                        issue_pair(lp + pack_copy_off(P, e, s_ug[nxt], rank, 0));
                 }
-                const bool out0 = blockIdx.x == 0;
-                if (a.logits && out0)
-#pragma unroll
-                    for (int qq = 0; qq < 4; ++qq)
-                        if (!taken[qq])
-                            a.logits[(size_t)l * a.E + lane + 32 * qq] = v[qq];
-                // each lane sorts its 4 candidates (key descending, lower
-                // index first on equal keys); the warp then pops the largest
-                // head K times
-                unsigned hk[4];
-                int hi[4];
-                float hv[4];
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    hk[qq] = taken[qq] ? 0u : key[qq];
-                    hi[qq] = taken[qq] ? 0x7fffffff : lane + 32 * qq;
-                    hv[qq] = v[qq];
-                }
-                auto cx = [&](int x, int y) {   // order (x, y)
-                    const bool sw = hk[y] > hk[x] || (hk[y] == hk[x] && hi[y] < hi[x]);
-                    if (sw) {
-                        const unsigned tk = hk[x];
-                        const int ti = hi[x];
-                        const float tv = hv[x];
-                        hk[x] = hk[y], hi[x] = hi[y], hv[x] = hv[y];
-                        hk[y] = tk, hi[y] = ti, hv[y] = tv;
-                    }
-                };
-                cx(0, 1), cx(2, 3), cx(0, 2), cx(1, 3), cx(1, 2);
-                float my_v = 0.f;
-                int my_i = 0;
-                int nxt = U.ns;   // next routed unit whose gate/up copies are due
-                for (int jj = 0; jj < K; ++jj) {
-                    const unsigned mk = __reduce_max_sync(0xffffffffu, hk[0]);
-                    // one lane holds the maximum unless keys tie: then the
-                    // lowest index among the tied heads wins
-                    const unsigned tied = __ballot_sync(0xffffffffu, hk[0] == mk);
-                    const int wl = __popc(tied) == 1
-                                       ? __ffs(tied) - 1
-                                       : (int)(__reduce_min_sync(0xffffffffu,
-                                                                 (unsigned)(hk[0] == mk ? hi[0] : 0x7fffffff)) &
-                                               31u);
-                    const int win = __shfl_sync(0xffffffffu, hi[0], wl);
-                    const float wv = __shfl_sync(0xffffffffu, hv[0], wl);
-                    if (lane == wl) {   // pop the head
-                        hk[0] = hk[1], hi[0] = hi[1], hv[0] = hv[1];
-                        hk[1] = hk[2], hi[1] = hi[2], hv[1] = hv[2];
-                        hk[2] = hk[3], hi[2] = hi[3], hv[2] = hv[3];
-                        hk[3] = 0u, hi[3] = 0x7fffffff, hv[3] = 0.f;
-                    }
-                    if (lane == jj) {
-                        my_v = wv;
-                        my_i = win;
-                    }
-                    // the jj-th expert is final: its units' gate/up copies go
-                    // out now, while the rest of the top-k is still being found
-                    // (units come in slot order)
-                    if (lane == 0 && ok) {
-                        const int e = (win >= 0 && win < a.E) ? win : 0;
-                        for (; nxt < U.nu && s_uj[nxt] == jj; ++nxt) {
-                            issue(lp + pack_copy_off(P, e, s_ug[nxt], rank, 0));
-                            issue(lp + pack_copy_off(P, e, s_ug[nxt], rank, 1));
-                        }
-                    }
-                }
-                const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
-                const float ex = lane < K ? expf(my_v - vmax) : 0.f;
-                float sum = ex;
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1)
-                    sum += __shfl_xor_sync(0xffffffffu, sum, off);
-                if (lane < K) {
-                    const int ei = (my_i >= 0 && my_i < a.E) ? my_i : 0;
-                    s_idx[lane] = ei;
-                    s_wt[lane] = ex / sum;
-                    if (out0) {
-                        if (a.idx)
-                            a.idx[(size_t)l * K + lane] = ei;
-                        if (a.weights)
-                            a.weights[(size_t)l * K + lane] = ex / sum;
-                    }
-                }
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(topk_bar);   // the routed down items may read s_wt
+                if (ok && !wait_bar(a, topk_bar, l & 1))
+                    ok = false;
             }
             if (lane == 0 && ok)   // the routed down copies
                 for (int s = U.ns; s < U.nu; ++s)
@@ -604,7 +586,7 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
         // drain: every copy issued has landed before the CTA may exit
         if (lane == 0) {
             for (int st = 0; st < NS && st < seq; ++st) {
-                const int last = seq - 1 - ((seq - 1 - st) % NS);   // last seq that used stage st
+                const int last = seq - 1 - ((seq - 1 - st) % NS);   // last seq that used slot st
                 wait_bar(a, &full[st], (last / NS) & 1);
             }
         }
@@ -650,6 +632,102 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                     }
                     mbar_arrive_remote(mapa_rank(smem_u32(logit_bar), lane));
                 }
+            }
+            // ---- top-k of this layer (exchange warp 0): each round's
+            // winner is published at once (round_bar) so that the producer
+            // streams its units while the later rounds run
+            if (xw == 0) {
+                ok = __all_sync(0xffffffffu, ok && wait_bar_cluster(a, logit_bar, l & 1));
+                if (!ok)
+                    break;
+                float v[4];
+                unsigned key[4];
+                bool taken[4];
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const int e = lane + 32 * qq;
+                    taken[qq] = e >= a.E;
+                    v[qq] = taken[qq] ? 0.f : s_logit[e];
+                    const unsigned u = __float_as_uint(v[qq]);   // order-preserving key
+                    key[qq] = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+                }
+                const bool out0 = blockIdx.x == 0;
+                if (a.logits && out0)
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq)
+                        if (!taken[qq])
+                            a.logits[(size_t)l * a.E + lane + 32 * qq] = v[qq];
+                // each lane sorts its 4 candidates (key descending, lower
+                // index first on equal keys); the warp then pops the largest
+                // head K times
+                unsigned hk[4];
+                int hi[4];
+                float hv[4];
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    hk[qq] = taken[qq] ? 0u : key[qq];
+                    hi[qq] = taken[qq] ? 0x7fffffff : lane + 32 * qq;
+                    hv[qq] = v[qq];
+                }
+                auto cx = [&](int x, int y) {   // order (x, y)
+                    const bool sw = hk[y] > hk[x] || (hk[y] == hk[x] && hi[y] < hi[x]);
+                    if (sw) {
+                        const unsigned tk = hk[x];
+                        const int ti = hi[x];
+                        const float tv = hv[x];
+                        hk[x] = hk[y], hi[x] = hi[y], hv[x] = hv[y];
+                        hk[y] = tk, hi[y] = ti, hv[y] = tv;
+                    }
+                };
+                cx(0, 1), cx(2, 3), cx(0, 2), cx(1, 3), cx(1, 2);
+                float my_v = 0.f;
+                int my_i = 0;
+                for (int jj = 0; jj < K; ++jj) {
+                    const unsigned mk = __reduce_max_sync(0xffffffffu, hk[0]);
+                    // one lane holds the maximum unless keys tie: then the
+                    // lowest index among the tied heads wins
+                    const unsigned tied = __ballot_sync(0xffffffffu, hk[0] == mk);
+                    const int wl = __popc(tied) == 1
+                                       ? __ffs(tied) - 1
+                                       : (int)(__reduce_min_sync(0xffffffffu,
+                                                                 (unsigned)(hk[0] == mk ? hi[0] : 0x7fffffff)) &
+                                               31u);
+                    const int win = __shfl_sync(0xffffffffu, hi[0], wl);
+                    const float wv = __shfl_sync(0xffffffffu, hv[0], wl);
+                    if (lane == wl) {   // pop the head
+                        hk[0] = hk[1], hi[0] = hi[1], hv[0] = hv[1];
+                        hk[1] = hk[2], hi[1] = hi[2], hv[1] = hv[2];
+                        hk[2] = hk[3], hi[2] = hi[3], hv[2] = hv[3];
+                        hk[3] = 0u, hi[3] = 0x7fffffff, hv[3] = 0.f;
+                    }
+                    if (lane == jj) {
+                        my_v = wv;
+                        my_i = win;
+                    }
+                    if (lane == 0) {
+                        s_idx[jj] = (win >= 0 && win < a.E) ? win : 0;
+                        mbar_arrive(&round_bar[jj]);   // release: s_idx[jj]
+                    }
+                }
+                const float vmax = __shfl_sync(0xffffffffu, my_v, 0);
+                const float ex = lane < K ? expf(my_v - vmax) : 0.f;
+                float sum = ex;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+                    sum += __shfl_xor_sync(0xffffffffu, sum, off);
+                if (lane < K) {
+                    const int ei = (my_i >= 0 && my_i < a.E) ? my_i : 0;
+                    s_wt[lane] = ex / sum;
+                    if (out0) {
+                        if (a.idx)
+                            a.idx[(size_t)l * K + lane] = ei;
+                        if (a.weights)
+                            a.weights[(size_t)l * K + lane] = ex / sum;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(topk_bar);   // the down copies and items may read s_wt
             }
             for (int s = xw; s < U.nu; s += DC_XN) {
                 ok = __all_sync(0xffffffffu, wait_bar(a, &gubar[s], l & 1));
@@ -727,10 +805,12 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
         // unit's 8 gate and 8 up rows go to gupart[slot] and the exchange warp
         // finishes the unit (SwiGLU, h to the cluster), so the group moves on
         // at once.
-        auto do_gu = [&](int seq0, int slot) {
+        auto do_gu = [&](int seq0, int slot) {   // seq0, seq0 + 1: the ring sequences
             const int sa = seq0 % NS, sb = (seq0 + 1) % NS;
             // the lanes of a warp decide together: the mma below is warp-collective
-            const bool good = __all_sync(0xffffffffu, ok && wait_bar(a, &full[sa], (seq0 / NS) & 1) &&
+            const bool good = __all_sync(0xffffffffu, ok && wait_arm(a, s_arm + sa, seq0) &&
+                                                          wait_bar(a, &full[sa], (seq0 / NS) & 1) &&
+                                                          wait_arm(a, s_arm + sb, seq0 + 1) &&
                                                           wait_bar(a, &full[sb], ((seq0 + 1) / NS) & 1));
             float ag = 0.f, au = 0.f, bg = 0.f, bu = 0.f;
             if (good) {
@@ -741,26 +821,26 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                 const unsigned char *sbA = A + P.st_codes + (size_t)gid * GH * 4;
                 const unsigned char *sbB = B + P.st_codes + (size_t)gid * GH * 4;
                 const int g0 = wq * GH / DC_GW, g1 = (wq + 1) * GH / DC_GW;
+                // branch-free: column 0 of B is x (lanes gid == 0; the other
+                // lanes read a zero block), and every lane does the per-group
+                // scale and bias steps (only column 0, lanes tig == 0, counts)
+                const int th = tig >> 1;
+                const uint4 *xq = gid == 0 ? xs4 + tig : xzero;
+                const int xst = gid == 0 ? 8 : 0, x1o = gid == 0 ? 4 : 0;
 #pragma unroll 2
                 for (int g = g0; g < g1; ++g) {
-                    const int ch = swz_chunk(2 * g + (tig >> 1), gid);
+                    const int ch = ((2 * g) | th) ^ gid;   // 16-byte chunk, swizzled by row
                     const uint2 wa = *reinterpret_cast<const uint2 *>(rowA + 16 * ch);
                     const uint2 wb = *reinterpret_cast<const uint2 *>(rowB + 16 * ch);
-                    uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
-                    if (gid == 0) {
-                        x0 = xs4[(g * 2 + 0) * 4 + tig];
-                        x1 = xs4[(g * 2 + 1) * 4 + tig];
-                    }
+                    const uint4 x0 = xq[g * xst], x1 = xq[g * xst + x1o];
                     float r[4];
                     mma_group_s4(r, wa, wb, x0, x1);
-                    if (tig == 0) {
-                        const float X = xsum[g * 8];
-                        const float2 pa = sb_word(sbA + 4 * g), pb = sb_word(sbB + 4 * g);
-                        ag = fmaf(pa.x, r[0], ag);
-                        au = fmaf(pb.x, r[2], au);
-                        bg = fmaf(pa.y, X, bg);
-                        bu = fmaf(pb.y, X, bu);
-                    }
+                    const float X = xsum[g * 8];
+                    const float2 pa = sb_word(sbA + 4 * g), pb = sb_word(sbB + 4 * g);
+                    ag = fmaf(pa.x, r[0], ag);
+                    au = fmaf(pb.x, r[2], au);
+                    bg = fmaf(pa.y, X, bg);
+                    bu = fmaf(pb.y, X, bu);
                 }
             }
             __syncwarp();
@@ -781,10 +861,11 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
         };
 
         // ---------------------------------------- one down work item
-        auto do_dn = [&](int seq, int slot, int j, int l) {
+        auto do_dn = [&](int seq, int slot, int j, int l) {   // seq: the ring sequence
             const int st = seq % NS;
             // the lanes of a warp decide together: the mma below is warp-collective
-            bool good = __all_sync(0xffffffffu, ok && wait_bar(a, &full[st], (seq / NS) & 1) &&
+            bool good = __all_sync(0xffffffffu, ok && wait_arm(a, s_arm + st, seq) &&
+                                                    wait_bar(a, &full[st], (seq / NS) & 1) &&
                                                     wait_bar_cluster(a, &hbar[slot], l & 1));
             float w = 1.f;
             if (good && j < K) {   // a routed unit: its router weight
@@ -811,11 +892,11 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                         *reinterpret_cast<const uint2 *>(S + (size_t)(r0 + 8) * 32 + 8 * tig);
                     float r[4];
                     mma_group_s4(r, wa, wb, x0, x1);
-                    if (tig == 0) {
-                        const float2 pa = sb_word(S + P.st_codes + 4 * (size_t)r0);
-                        const float2 pb = sb_word(S + P.st_codes + 4 * (size_t)(r0 + 8));
-                        const float va = fmaf(pa.x * kCode4, r[0] + r[1], pa.y * X);
-                        const float vb = fmaf(pb.x * kCode4, r[2] + r[3], pb.y * X);
+                    const float2 pa = sb_word(S + P.st_codes + 4 * (size_t)r0);
+                    const float2 pb = sb_word(S + P.st_codes + 4 * (size_t)(r0 + 8));
+                    const float va = fmaf(pa.x * kCode4, r[0] + r[1], pa.y * X);
+                    const float vb = fmaf(pb.x * kCode4, r[2] + r[3], pb.y * X);
+                    if (tig == 0) {   // columns 0 and 1 (h hi, lo) of rows r0, r0 + 8
                         my_ypart[r0] = fmaf(w, va, my_ypart[r0]);
                         my_ypart[r0 + 8] = fmaf(w, vb, my_ypart[r0 + 8]);
                     }
@@ -891,26 +972,24 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                     const unsigned char *sba = rbuf + P.rb_codes + (size_t)ra * GH * 4;
                     const unsigned char *sbb = rbuf + P.rb_codes + (size_t)rb * GH * 4;
                     const int g0 = warp * GH / DC_CW, g1 = (warp + 1) * GH / DC_CW;
+                    // branch-free, as in the gate/up items
+                    const uint4 *xq = gid == 0 ? xs8 + tig : xzero;
+                    const int xst = gid == 0 ? 8 : 0, x1o = gid == 0 ? 4 : 0;
+#pragma unroll 2
                     for (int g = g0; g < g1; ++g) {
                         const uint4 wa = *reinterpret_cast<const uint4 *>(
                             rowa + 16 * swz_chunk(4 * g + tig, ra & 7));
                         const uint4 wb = *reinterpret_cast<const uint4 *>(
                             rowb + 16 * swz_chunk(4 * g + tig, rb & 7));
-                        uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
-                        if (gid == 0) {
-                            x0 = xs8[(g * 2 + 0) * 4 + tig];
-                            x1 = xs8[(g * 2 + 1) * 4 + tig];
-                        }
+                        const uint4 x0 = xq[g * xst], x1 = xq[g * xst + x1o];
                         float r[4];
                         mma_group_s8(r, wa, wb, x0, x1);
-                        if (tig == 0) {
-                            const float X = xsum[g * 8];
-                            const float2 pa = sb_word(sba + 4 * g), pb = sb_word(sbb + 4 * g);
-                            acc_lo = fmaf(pa.x, r[0], acc_lo);
-                            acc_hi = fmaf(pb.x, r[2], acc_hi);
-                            b_lo = fmaf(pa.y, X, b_lo);
-                            b_hi = fmaf(pb.y, X, b_hi);
-                        }
+                        const float X = xsum[g * 8];
+                        const float2 pa = sb_word(sba + 4 * g), pb = sb_word(sbb + 4 * g);
+                        acc_lo = fmaf(pa.x, r[0], acc_lo);
+                        acc_hi = fmaf(pb.x, r[2], acc_hi);
+                        b_lo = fmaf(pa.y, X, b_lo);
+                        b_hi = fmaf(pb.y, X, b_hi);
                     }
                 }
                 if (!good)
@@ -930,27 +1009,22 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                 convert_slice(l - 1);
             // ---- the layer's work items, dealt to the groups
             {
+                // ring order of a layer: shared gate/up, shared down, routed
+                // gate/up, routed down; the items follow it
                 const int base = l * 3 * U.nu;
                 for (int k = q; k < nitems; k += DC_GROUPS) {
-                    int seq, slot;
-                    bool gu;
                     if (k < U.ns) {
-                        gu = true, slot = k, seq = base + 2 * k;
+                        do_gu(base + 2 * k, k);
                     } else if (k < 2 * U.ns) {
-                        gu = false, slot = k - U.ns, seq = base + 2 * U.ns + slot;
+                        const int s = k - U.ns;
+                        do_dn(base + 2 * U.ns + s, s, s_uj[s], l);
                     } else if (k < 2 * U.ns + U.nr) {
-                        gu = true, slot = U.ns + (k - 2 * U.ns);
-                        seq = base + 3 * U.ns + 2 * (k - 2 * U.ns);
+                        const int m = k - 2 * U.ns;
+                        do_gu(base + 3 * U.ns + 2 * m, U.ns + m);
                     } else {
-                        gu = false;
                         const int m = k - 2 * U.ns - U.nr;
-                        slot = U.ns + m;
-                        seq = base + 3 * U.ns + 2 * U.nr + m;
+                        do_dn(base + 3 * U.ns + 2 * U.nr + m, U.ns + m, s_uj[U.ns + m], l);
                     }
-                    if (gu)
-                        do_gu(seq, slot);
-                    else
-                        do_dn(seq, slot, s_uj[slot], l);
                 }
             }
             // ---- this CTA's rows of the layer output into the accumulator

@@ -203,20 +203,6 @@ __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, int32_t 
     return false;
 }
 
-// named barrier of n threads that also ORs a predicate over them: every
-// participant gets the same answer (used to leave loops together)
-__device__ __forceinline__ bool bar_any(int id, int n, bool v)
-{
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)v), "r"(id), "r"(n)
-        : "memory");
-    return r != 0;
-}
-
 // -------------------------------------------------------------- schedule --
 // unit u = (heavy slot list entry u / RB, row block u % RB); slots sorted by
 // decreasing token count, so the largest units are spread first
