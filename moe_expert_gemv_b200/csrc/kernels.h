@@ -194,9 +194,13 @@ struct PrefillWorkspace {
     __half *hb_lo;
     __half *hs_hi;      // [npos][64] group sums of h (hi + lo), as a pair, zero-padded
     __half *hs_lo;
+    float *tcpart;      // [kTcMaxCtas][128 rows][128 positions][gate, up] partial sums of
+                        // the first half of K (each tensor-core CTA its own block)
 };
 size_t prefill_workspace_layout(int E, int hidden, int inter, int T, int top_k, void *base,
                                 PrefillWorkspace *ws);
+constexpr int kTcMaxCtas = 160;                         // tensor-core prefill CTAs at most
+constexpr size_t kTcPartBytes = (size_t)128 * 128 * 2 * 4;   // one CTA's partial-sum block
 
 struct GroupArgs {
     const int32_t *idx;

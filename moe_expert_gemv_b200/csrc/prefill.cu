@@ -885,6 +885,7 @@ size_t prefill_workspace_layout(int E, int H, int I, int T, int top_k, void *bas
     const size_t xb_off = take((size_t)d.npos * 64 * 2 * 2);
     const size_t hb_off = take((size_t)d.npos * I * 2 * 2);
     const size_t hs_off = take((size_t)d.npos * 64 * 2 * 2);
+    const size_t tcpart_off = take((size_t)kTcMaxCtas * kTcPartBytes);
     if (base && ws) {
         unsigned char *b = static_cast<unsigned char *>(base);
         ws->counts = reinterpret_cast<int32_t *>(b + counts_off);
@@ -906,6 +907,7 @@ size_t prefill_workspace_layout(int E, int H, int I, int T, int top_k, void *bas
         ws->hb_lo = ws->hb_hi + (size_t)d.npos * I;
         ws->hs_hi = reinterpret_cast<__half *>(b + hs_off);
         ws->hs_lo = ws->hs_hi + (size_t)d.npos * 64;
+        ws->tcpart = reinterpret_cast<float *>(b + tcpart_off);
     }
     return off;
 }

@@ -255,9 +255,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     volatile int *abort_word = reinterpret_cast<volatile int *>(smem + L.misc_off + 4);
 
     constexpr int NM = DOWN ? 1 : 2;                 // matrices per unit
+    // gate/up units run their K in NKH halves with fresh accumulators; the
+    // epilogue adds the halves in fp32 (partial sums through tcpart), so no
+    // tensor-memory accumulator chains more than half the k-blocks
+    constexpr int NKH = DOWN ? 1 : 2;
     const int rows = DOWN ? a.H : a.I;               // rows of one expert's matrix
     const int K = DOWN ? a.I : a.H;
     const int GK = K / kGroup;                       // main k-blocks
+    // end of K part kh's k-blocks; the last part also takes the bias block (kb == GK)
+    auto kb_end = [&](int kh) { return kh + 1 == NKH ? GK + 1 : (kh + 1) * GK / NKH; };
     const int RB = (rows + TC_M - 1) / TC_M;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -317,7 +323,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 const bool sh = t.slot == a.E;
                 const int row0 = (sh ? 0 : t.slot * rows) + t.rb * TC_M;
                 const uint32_t btile = (uint32_t)t.npad * 128;
-                for (int kb = 0; kb <= GK && ok; ++kb) {
+                for (int kh = 0; kh < NKH && ok; ++kh)
+                for (int kb = kh * GK / NKH; kb < kb_end(kh) && ok; ++kb) {
                     if (kb < GK) {
                         for (int m = 0; m < NM && ok; ++m) {
                             const int s = cs % TC_NC;
@@ -370,16 +377,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (lane == 0 && nunits > 0) {
             int as = 0, bs = 0, nu = 0;
             bool ok = true, issued = false;
-            for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++nu) {
+            for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x)
+            for (int kh = 0; kh < NKH && ok; ++kh, ++nu) {
                 const TcUnit t = tc_unit(a, RB, u);
                 const uint32_t idesc = tc_idesc(t.npad);
-                // the epilogue has read the previous unit's accumulators
+                const int kb0 = kh * GK / NKH;
+                // the epilogue has read the previous accumulators
                 if (nu > 0 && !tc_wait(&bar[B_ACC_EMPTY], (nu - 1) & 1, a.status, abort_word)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                for (int kb = 0; kb <= GK && ok; ++kb) {
+                for (int kb = kb0; kb < kb_end(kh) && ok; ++kb) {
                     const bool bias = kb == GK;
                     const int sb = bs % TC_NB;
                     if (!tc_wait(&bar[B_FULL_B + sb], (bs / TC_NB) & 1, a.status, abort_word)) {
@@ -404,7 +413,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks) {
                             const uint32_t ko = 32u * ks;
-                            const uint32_t acc0 = (kb > 0 || ks > 0) ? 1u : 0u;
+                            const uint32_t acc0 = (kb > kb0 || ks > 0) ? 1u : 0u;
                             if (bias) {
                                 tc_mma(d, tc_desc(ahi + ko), tc_desc(b0 + ko), idesc, 1u);
                                 tc_mma(dl, tc_desc(alo + ko), tc_desc(b0 + ko), idesc, 1u);
@@ -426,7 +435,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     ++bs;
                 }
                 if (ok)
-                    tc_commit(&bar[B_ACC_FULL]);   // the unit's accumulators are complete
+                    tc_commit(&bar[B_ACC_FULL]);   // the accumulators of this K part are complete
             }
             // every MMA issued has finished before the tensor memory is freed
             if (issued) {
@@ -444,7 +453,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int chalf = dw >> 2;                // column half of the epilogue
         int cs = 0, as = 0, nu = 0;
         bool dead = false;   // this warp saw a failed wait (uniform within the warp)
-        for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++nu) {
+        for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
             // the 8 warps leave together once any of them failed, and only
             // then may this unit's scales overwrite the previous unit's
             if (bar_any(TC_BAR_EPI + 1, TC_DQ * 32, dead || *abort_word != 0))
@@ -464,7 +473,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 }
             }
             named_bar_sync(TC_BAR_EPI + 1, TC_DQ * 32);
-            for (int kb = 0; kb <= GK && !dead; ++kb) {
+            for (int kh = 0; kh < NKH; ++kh, ++nu) {
+            for (int kb = kh * GK / NKH; kb < kb_end(kh) && !dead; ++kb) {
                 for (int m = 0; m < NM && !dead; ++m) {
                     const int sa = as % TC_NA;
                     if (as >= TC_NA &&
@@ -554,6 +564,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 dead = true;
             tc_fence_after();
             const int myrow = t.rb * TC_M + 32 * q + lane;
+            // this thread's (gate, up) partial sums of the earlier K parts:
+            // row 32 q + lane, the thread's own columns, written and read
+            // back by the same thread
+            float2 *part = reinterpret_cast<float2 *>(a.ws.tcpart) +
+                           (size_t)blockIdx.x * (kTcPartBytes / 8) + (size_t)(32 * q + lane) * 128;
             if (acc_ok) {
                 for (int c0 = 16 * chalf; c0 < t.npad; c0 += 32) {
                     float dv[16], uv[16];
@@ -570,6 +585,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
                             uv[i] += lv[i];
+                        if (kh > 0) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const float2 pv = part[c0 + i];
+                                dv[i] += pv.x;
+                                uv[i] += pv.y;
+                            }
+                        }
+                        if (kh + 1 < NKH) {   // not the last K part: keep the sums
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                part[c0 + i] = make_float2(dv[i], uv[i]);
+                            continue;
+                        }
                     }
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
@@ -606,7 +635,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&bar[B_ACC_EMPTY]);
-            if (!DOWN) {
+            if (!DOWN && kh + 1 == NKH) {
                 // group sums of h: rows 0..63 of the unit are group 2 rb, 64..127
                 // group 2 rb + 1; every warp's partials are in before they are read
                 const bool all_ok = !bar_any(TC_BAR_EPI, TC_DQ * 32, !acc_ok);
@@ -624,6 +653,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     }
                 named_bar_sync(TC_BAR_EPI, TC_DQ * 32);   // hsp is free for the next unit
             }
+            }   // K parts
         }
     }
 
@@ -730,15 +760,16 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, const LaunchCfg &c, bool dow
     if (!ok)
         return cudaErrorInvalidValue;
     const size_t smem = tc_layout().total;
+    const int grid = c.num_sms < kTcMaxCtas ? c.num_sms : kTcMaxCtas;   // tcpart blocks
     cudaError_t e;
     if (down) {
         if ((e = set_smem(prefill_tc_kernel<true>, smem)) != cudaSuccess)
             return e;
-        return launch_ex(prefill_tc_kernel<true>, dim3(c.num_sms), dim3(TC_THREADS), smem, c, 1, a, mp);
+        return launch_ex(prefill_tc_kernel<true>, dim3(grid), dim3(TC_THREADS), smem, c, 1, a, mp);
     }
     if ((e = set_smem(prefill_tc_kernel<false>, smem)) != cudaSuccess)
         return e;
-    return launch_ex(prefill_tc_kernel<false>, dim3(c.num_sms), dim3(TC_THREADS), smem, c, 1, a, mp);
+    return launch_ex(prefill_tc_kernel<false>, dim3(grid), dim3(TC_THREADS), smem, c, 1, a, mp);
 }
 
 }  // namespace qmoe
