@@ -104,6 +104,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_
     }
 }
 
+// Bounded wait until a ring stage has been armed for sequence `sq` (a word
+// the producer writes before each copy).  Returns false (and flags
+// QMOE_DEV_TIMEOUT) if it is not within kWaitLimitNs.
+__device__ __forceinline__ bool wait_armed(const volatile int *arm, int sq, int32_t *status)
+{
+    if (*arm == sq)
+        return true;
+    const unsigned long long t0 = global_timer_ns();
+    while (*arm != sq) {
+        __nanosleep(20);
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            flag_status(status, QMOE_DEV_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
 // ------------------------------------------------------ TMA bulk copies --
 // 1-D bulk copy global -> this CTA's shared memory, completing on `bar`
 // (transaction bytes).  Both addresses 16-byte aligned, bytes % 16 == 0.

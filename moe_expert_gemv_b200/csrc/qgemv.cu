@@ -56,6 +56,8 @@ namespace {
 
 constexpr int QG_CW = 16;                     // consumer warps
 constexpr int QG_CT = QG_CW * 32;             // consumer threads
+constexpr int QG_GW = 4;                      // warps per tile group
+constexpr int QG_NG = QG_CW / QG_GW;          // tile groups: tile k goes to group k % QG_NG
 constexpr int QG_THREADS = QG_CT + 32;        // + one producer warp
 constexpr int QG_MAX_STAGES = 8;
 
@@ -86,7 +88,7 @@ __host__ __device__ inline QgLayout qg_layout(int K, int bits, int ncol, int NS,
     L.red_off = off;
     off += 2 * QG_CW * 32 * 16;
     L.bar_off = off;
-    off += 2 * QG_MAX_STAGES * 8;
+    off += 2 * QG_MAX_STAGES * 8 + QG_MAX_STAGES * 4;   // full, empty, armed sequence
     off = (off + 1023) & ~(size_t)1023;
     L.stage_off = off;
     L.codes_bytes = (size_t)16 * L.S * 4;
@@ -112,6 +114,11 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
     float4 *red = reinterpret_cast<float4 *>(smem + L.red_off);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bar_off);
     uint64_t *empty = full + QG_MAX_STAGES;
+    // the tile sequence each stage has been armed for (written by the
+    // producer before the copy): a tile group waits for its own sequence
+    // there first, so running more than one use of a stage ahead of another
+    // group never lets it take an older phase of the full barrier for its own
+    volatile int *s_arm = reinterpret_cast<volatile int *>(empty + QG_MAX_STAGES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_items = (a.N + 15) / 16;
@@ -120,7 +127,8 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], QG_CW);
+            mbar_init(&empty[s], QG_GW);   // the warps of the consuming tile group
+            s_arm[s] = -1;
         }
         mbar_init_fence();
     }
@@ -141,6 +149,7 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                 const int st = k % NS, use = k / NS;
                 if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, a.status))
                     break;
+                s_arm[st] = k;
                 const int r0 = item * 16;
                 const int rows = min(16, a.N - r0);
                 const uint32_t row_bytes = (uint32_t)Kw * 4;
@@ -199,17 +208,21 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                       ctid, QG_CT);
     named_bar_sync(1, QG_CT);
 
-    // this warp's groups: a contiguous block, so that with G % 64 == 0 the
-    // scales and biases of a row come as one 8-byte load per 4 groups
-    const int gpw = (L.G + QG_CW - 1) / QG_CW;
-    const int g0 = min(L.G, warp * gpw), g1 = min(L.G, g0 + gpw);
+    // tiles go to groups of QG_GW warps (tile k to group k % QG_NG); a warp
+    // takes a contiguous quarter of the tile's groups, so that with G % 64 ==
+    // 0 the scales and biases of a row come as one 8-byte load per 4 groups,
+    // and the group's partial sums meet at a barrier of its own
+    const int grp = warp / QG_GW, wq = warp % QG_GW;
+    const int gpw = (L.G + QG_GW - 1) / QG_GW;
+    const int g0 = min(L.G, wq * gpw), g1 = min(L.G, g0 + gpw);
     const bool vec_sb = (L.G & 63) == 0;
     const int gid = lane >> 2, tig = lane & 3;
     bool failed = false;
-    int k = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++k) {
+    int kk = 0;   // tiles this group has done (alternates its partial-sum buffers)
+    for (int k = grp; blockIdx.x + k * gridDim.x < n_items; k += QG_NG, ++kk) {
+        const int item = blockIdx.x + k * gridDim.x;
         const int st = k % NS, use = k / NS;
-        if (!failed && !mbar_wait(&full[st], use & 1, a.status))
+        if (!failed && !(wait_armed(s_arm + st, k, a.status) && mbar_wait(&full[st], use & 1, a.status)))
             failed = true;
         // the lanes of a warp decide together: the mma below is warp-collective
         failed = __any_sync(0xffffffffu, failed);
@@ -355,12 +368,13 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&empty[st]);
-        red[((k & 1) * QG_CW + warp) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        named_bar_sync(1, QG_CT);
-        if (warp == k % QG_CW) {
+        float4 *gred = red + (size_t)((grp * 2 + (kk & 1)) * QG_GW) * 32;
+        gred[wq * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        named_bar_sync(2 + grp, QG_GW * 32);
+        if (wq == kk % QG_GW) {
             float v[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int w = 0; w < QG_CW; ++w) {
-                const float4 p = red[((k & 1) * QG_CW + w) * 32 + lane];
+            for (int w = 0; w < QG_GW; ++w) {
+                const float4 p = gred[w * 32 + lane];
                 v[0] += p.x;
                 v[1] += p.y;
                 v[2] += p.z;
