@@ -56,8 +56,9 @@ ROUTER_CALL_BYTES = ROUTER_BYTES + H * 2 + TOPK * 8
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source it was taken on (sha256 of csrc/decode.cu); otherwise reported null.
 NCU_TRAFFIC = {
-    # 6-layer capture (186,702,592 B) scaled to the 30 layers of one launch
-    "moe_decode_kernel": {"bytes": 933512960, "sha": "d09a383d19ca7a25"},
+    # 6-layer capture (183,117,312 B read + 3,729,408 B written) scaled to
+    # the 30 layers of one launch
+    "moe_decode_kernel": {"bytes": 934233600, "sha": "4cf7b9364af2122f"},
 }
 
 
