@@ -203,6 +203,16 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// the same product into a fresh accumulator: d = A B
+__device__ __forceinline__ void mma_16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                            uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
 
 __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic)
 {
@@ -427,6 +437,38 @@ __device__ __forceinline__ void mma_group_s4(float (&r)[4], uint2 wa, uint2 wb, 
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         r[i] = c[i] + d[i];
+}
+// One 64-input group in a single accumulator chain (the four products
+// added in the tensor core, the first into a fresh accumulator): fewer
+// instructions than two chains joined by fp32 adds, for callers with enough
+// independent groups in flight to hide the longer chain.
+__device__ __forceinline__ void mma_group_s4_1(float (&r)[4], uint2 wa, uint2 wb, uint4 x0, uint4 x1)
+{
+    uint32_t pa[8], pb[8];
+    dequant4s_word(wa.x, pa);
+    dequant4s_word(wa.y, pa + 4);
+    dequant4s_word(wb.x, pb);
+    dequant4s_word(wb.y, pb + 4);
+    mma_16816_z(r, pa[0], pb[0], pa[2], pb[2], x0.x, x0.y);
+    mma_16816(r, pa[1], pb[1], pa[3], pb[3], x1.x, x1.y);
+    mma_16816(r, pa[4], pb[4], pa[6], pb[6], x0.z, x0.w);
+    mma_16816(r, pa[5], pb[5], pa[7], pb[7], x1.z, x1.w);
+}
+__device__ __forceinline__ void mma_group_s8_1(float (&r)[4], uint4 wa, uint4 wb, uint4 x0, uint4 x1)
+{
+    uint32_t pa[8], pb[8];
+    dequant8s_word(wa.x, pa);
+    dequant8s_word(wb.x, pb);
+    dequant8s_word(wa.y, pa + 2);
+    dequant8s_word(wb.y, pb + 2);
+    dequant8s_word(wa.z, pa + 4);
+    dequant8s_word(wb.z, pb + 4);
+    dequant8s_word(wa.w, pa + 6);
+    dequant8s_word(wb.w, pb + 6);
+    mma_16816_z(r, pa[0], pb[0], pa[1], pb[1], x0.x, x0.y);
+    mma_16816(r, pa[2], pb[2], pa[3], pb[3], x0.z, x0.w);
+    mma_16816(r, pa[4], pb[4], pa[5], pb[5], x1.x, x1.y);
+    mma_16816(r, pa[6], pb[6], pa[7], pb[7], x1.z, x1.w);
 }
 __device__ __forceinline__ void mma_group_s8(float (&r)[4], uint4 wa, uint4 wb, uint4 x0, uint4 x1)
 {

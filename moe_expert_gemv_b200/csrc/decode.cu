@@ -834,7 +834,7 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                     const uint2 wb = *reinterpret_cast<const uint2 *>(rowB + 16 * ch);
                     const uint4 x0 = xq[g * xst], x1 = xq[g * xst + x1o];
                     float r[4];
-                    mma_group_s4(r, wa, wb, x0, x1);
+                    mma_group_s4_1(r, wa, wb, x0, x1);
                     const float X = xsum[g * 8];
                     const float2 pa = sb_word(sbA + 4 * g), pb = sb_word(sbB + 4 * g);
                     ag = fmaf(pa.x, r[0], ag);
@@ -891,7 +891,7 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                     const uint2 wb =
                         *reinterpret_cast<const uint2 *>(S + (size_t)(r0 + 8) * 32 + 8 * tig);
                     float r[4];
-                    mma_group_s4(r, wa, wb, x0, x1);
+                    mma_group_s4_1(r, wa, wb, x0, x1);
                     const float2 pa = sb_word(S + P.st_codes + 4 * (size_t)r0);
                     const float2 pb = sb_word(S + P.st_codes + 4 * (size_t)(r0 + 8));
                     const float va = fmaf(pa.x * kCode4, r[0] + r[1], pa.y * X);
@@ -983,7 +983,7 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                             rowb + 16 * swz_chunk(4 * g + tig, rb & 7));
                         const uint4 x0 = xq[g * xst], x1 = xq[g * xst + x1o];
                         float r[4];
-                        mma_group_s8(r, wa, wb, x0, x1);
+                        mma_group_s8_1(r, wa, wb, x0, x1);
                         const float X = xsum[g * 8];
                         const float2 pa = sb_word(sba + 4 * g), pb = sb_word(sbb + 4 * g);
                         acc_lo = fmaf(pa.x, r[0], acc_lo);

@@ -88,7 +88,7 @@ __host__ __device__ inline QgLayout qg_layout(int K, int bits, int ncol, int NS,
     L.red_off = off;
     off += 2 * QG_CW * 32 * 16;
     L.bar_off = off;
-    off += 2 * QG_MAX_STAGES * 8 + QG_MAX_STAGES * 4;   // full, empty, armed sequence
+    off += 2 * QG_MAX_STAGES * 8 + QG_MAX_STAGES * 4 + 16;   // full, empty, armed sequence, zeros
     off = (off + 1023) & ~(size_t)1023;
     L.stage_off = off;
     L.codes_bytes = (size_t)16 * L.S * 4;
@@ -119,6 +119,8 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
     // there first, so running more than one use of a stage ahead of another
     // group never lets it take an older phase of the full barrier for its own
     volatile int *s_arm = reinterpret_cast<volatile int *>(empty + QG_MAX_STAGES);
+    // 16 zero bytes: the x fragment of the MMA columns past the batch
+    uint4 *xzero = reinterpret_cast<uint4 *>(smem + L.bar_off + 2 * QG_MAX_STAGES * 8 + QG_MAX_STAGES * 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_items = (a.N + 15) / 16;
@@ -130,6 +132,7 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
             mbar_init(&empty[s], QG_GW);   // the warps of the consuming tile group
             s_arm[s] = -1;
         }
+        *xzero = make_uint4(0, 0, 0, 0);
         mbar_init_fence();
     }
     __syncthreads();
@@ -236,24 +239,26 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
             // factor is applied once at the end
             float aq[4] = {0.f, 0.f, 0.f, 0.f}, ab[4] = {0.f, 0.f, 0.f, 0.f};
             // one group from its fragment addresses (rows gid, gid+8)
+            // branch-free: the MMA columns past the batch read a zero block
+            const bool live = gid < a.B;
+            const uint4 *xq = live ? xs + gid * 4 + tig : xzero;
+            const uint4 *xql = live ? xs_lo + gid * 4 + tig : xzero;
+            const int xst = live ? 2 * a.B * 4 : 0, x1o = live ? a.B * 4 : 0;
             auto group = [&](int g, const void *fa, const void *fb, float s_lo, float s_hi,
                              float b_lo, float b_hi) {
-                uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0, l0 = x0, l1 = x0;
-                if (gid < a.B) {
-                    x0 = xs[((g * 2 + 0) * a.B + gid) * 4 + tig];
-                    x1 = xs[((g * 2 + 1) * a.B + gid) * 4 + tig];
-                    if (ROT) {
-                        l0 = xs_lo[((g * 2 + 0) * a.B + gid) * 4 + tig];
-                        l1 = xs_lo[((g * 2 + 1) * a.B + gid) * 4 + tig];
-                    }
+                const uint4 x0 = xq[g * xst], x1 = xq[g * xst + x1o];
+                uint4 l0 = make_uint4(0, 0, 0, 0), l1 = l0;
+                if (ROT) {
+                    l0 = xql[g * xst];
+                    l1 = xql[g * xst + x1o];
                 }
                 float r[4];
                 if (BITS == 4 && ROT)
                     mma_group_s4_hilo(r, *reinterpret_cast<const uint2 *>(fa),
                                       *reinterpret_cast<const uint2 *>(fb), x0, x1, l0, l1);
                 else if (BITS == 4)
-                    mma_group_s4(r, *reinterpret_cast<const uint2 *>(fa),
-                                 *reinterpret_cast<const uint2 *>(fb), x0, x1);
+                    mma_group_s4_1(r, *reinterpret_cast<const uint2 *>(fa),
+                                   *reinterpret_cast<const uint2 *>(fb), x0, x1);
                 else if (FMT == QG_SYM8) {
                     // two's-complement byte q -> q + 128 = byte ^ 0x80; the
                     // -128 s offset joins the folded bias
@@ -270,10 +275,10 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                     if (ROT)
                         mma_group_s8_hilo(r, wa, wb, x0, x1, l0, l1);
                     else
-                        mma_group_s8(r, wa, wb, x0, x1);
+                        mma_group_s8_1(r, wa, wb, x0, x1);
                 } else
-                    mma_group_s8(r, *reinterpret_cast<const uint4 *>(fa),
-                                 *reinterpret_cast<const uint4 *>(fb), x0, x1);
+                    mma_group_s8_1(r, *reinterpret_cast<const uint4 *>(fa),
+                                   *reinterpret_cast<const uint4 *>(fb), x0, x1);
                 const float2 X = *reinterpret_cast<const float2 *>(xsum + g * 8 + 2 * tig);
                 aq[0] = fmaf(s_lo, r[0], aq[0]);
                 aq[1] = fmaf(s_lo, r[1], aq[1]);
