@@ -117,7 +117,7 @@ typedef struct qmoe_moe_layer {
  * Errors: INVALID_ARG (NULL, batch outside 1..32, shape), ALIGNMENT,
  * UNSUPPORTED (group != 64, cols % 64, rows % 8, or rows too long for one
  * row of x plus one 16-row tile in shared memory: cols above 18624 at 4 bits,
- * 11008 at 8 bits; qgemv_affine_ws takes such rows from batch 9 on), CUDA.
+ * 10944 at 8 bits; qgemv_affine_ws takes such rows from batch 9 on), CUDA.
  * ------------------------------------------------------------------------- */
 qmoe_status qgemv_affine(const qmoe_qmatrix *W, const uint16_t *x, int32_t batch,
                          uint16_t *y, int32_t *status_dev, void *stream);

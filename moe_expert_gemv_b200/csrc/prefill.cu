@@ -528,7 +528,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const __half *gs = reinterpret_cast<const __half *>(stage + 2 * st.codes);
                 const __half *gb = gs + GU_ROWS * d.GH, *us = gb + GU_ROWS * d.GH,
                              *ub = us + GU_ROWS * d.GH;
-                const bool nvalid = gid < ut.nv;
+                // column gid of the MMA is tile token gid: tokens past ut.nv read
+                // whatever the tile row holds, which only reaches their own
+                // columns, and those are never stored
                 const uint4 *xr = xf + gid * d.xg_stride;
                 const float *xs0 = xsm + (2 * tig) * d.xs_stride;
                 const float *xs1 = xs0 + d.xs_stride;
@@ -565,14 +567,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int g = 4 * q4 + j;
-                        uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
-                        if (nvalid) {
-                            x0 = xr[(g * 2 + 0) * 4 + tig];
-                            x1 = xr[(g * 2 + 1) * 4 + tig];
-                        }
+                        const uint4 x0 = xr[(g * 2 + 0) * 4 + tig];
+                        const uint4 x1 = xr[(g * 2 + 1) * 4 + tig];
                         float r[4];
-                        mma_group_s4(r, *reinterpret_cast<const uint2 *>(gtc + off[j]),
-                                     *reinterpret_cast<const uint2 *>(utc + off[j]), x0, x1);
+                        mma_group_s4_1(r, *reinterpret_cast<const uint2 *>(gtc + off[j]),
+                                       *reinterpret_cast<const uint2 *>(utc + off[j]), x0, x1);
                         const float2 fsg = __half22float2(u32_as_h2(sgw[j >> 1]));
                         const float2 fbg = __half22float2(u32_as_h2(bgw[j >> 1]));
                         const float2 fsu = __half22float2(u32_as_h2(suw[j >> 1]));
@@ -727,7 +726,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const unsigned char *wt = smem + L.stage_off + (size_t)slot * st.bytes;
                 const __half *sc = reinterpret_cast<const __half *>(wt + st.codes);
                 const __half *bi = sc + DN_ROWS * d.GI;
-                const bool nvalid = gid < ut.nv;
+                // as in the gate/up kernel: columns of tokens past ut.nv are
+                // computed from whatever their tile rows hold and never stored
                 const uint4 *hr = hb + gid * d.hf_stride;
                 const float *hs0 = hsm + (2 * tig) * d.hs_stride;
                 const float *hs1 = hs0 + d.hs_stride;
@@ -741,13 +741,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 float aq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                 float ab[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                 for (int g = 0; g < d.GI; ++g) {
-                    uint4 h0 = make_uint4(0, 0, 0, 0), h1 = h0, l0 = h0, l1 = h0;
-                    if (nvalid) {
-                        h0 = hr[((g * 2 + 0) * 2 + 0) * 4 + tig];
-                        h1 = hr[((g * 2 + 1) * 2 + 0) * 4 + tig];
-                        l0 = hr[((g * 2 + 0) * 2 + 1) * 4 + tig];
-                        l1 = hr[((g * 2 + 1) * 2 + 1) * 4 + tig];
-                    }
+                    const uint4 h0 = hr[((g * 2 + 0) * 2 + 0) * 4 + tig];
+                    const uint4 h1 = hr[((g * 2 + 1) * 2 + 0) * 4 + tig];
+                    const uint4 l0 = hr[((g * 2 + 0) * 2 + 1) * 4 + tig];
+                    const uint4 l1 = hr[((g * 2 + 1) * 2 + 1) * 4 + tig];
                     const float2 S0 = *reinterpret_cast<const float2 *>(hs0 + g * 2);
                     const float2 S1 = *reinterpret_cast<const float2 *>(hs1 + g * 2);
                     const float X0 = S0.x + S0.y, X1 = S1.x + S1.y;

@@ -294,70 +294,60 @@ __global__ void __launch_bounds__(SM_THREADS, 1)
                 }
                 s_lo *= kCodeScale;
                 s_hi *= kCodeScale;
-                // one mma per accumulator first, then the dependent ones
-                float c[NT][4], d[NT][4];
+                // one chain per n-tile (the first product into a fresh
+                // accumulator), the n-tiles interleaved; columns past the
+                // batch repeat column B - 1 (never stored), so the x loads
+                // need no zero fill
+                float c[NT][4];
                 uint4 x0[NT], x1[NT];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    const int n = nt * 8 + gid;
-                    x0[nt] = make_uint4(0, 0, 0, 0);
-                    x1[nt] = x0[nt];
-                    if (n < a.B) {
-                        x0[nt] = xs[((g * 2 + 0) * a.B + n) * 4 + tig];
-                        x1[nt] = xs[((g * 2 + 1) * a.B + n) * 4 + tig];
-                    }
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        c[nt][i] = d[nt][i] = 0.f;
+                    const int n = min(nt * 8 + gid, a.B - 1);
+                    x0[nt] = xs[((g * 2 + 0) * a.B + n) * 4 + tig];
+                    x1[nt] = xs[((g * 2 + 1) * a.B + n) * 4 + tig];
                 }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     if (BITS == 4) {
-                        mma_16816(c[nt], pa[0], pb[0], pa[2], pb[2], x0[nt].x, x0[nt].y);
-                        mma_16816(d[nt], pa[1], pb[1], pa[3], pb[3], x1[nt].x, x1[nt].y);
+                        mma_16816_z(c[nt], pa[0], pb[0], pa[2], pb[2], x0[nt].x, x0[nt].y);
+                        mma_16816(c[nt], pa[1], pb[1], pa[3], pb[3], x1[nt].x, x1[nt].y);
                     } else {
-                        mma_16816(c[nt], pa[0], pb[0], pa[1], pb[1], x0[nt].x, x0[nt].y);
-                        mma_16816(d[nt], pa[2], pb[2], pa[3], pb[3], x0[nt].z, x0[nt].w);
+                        mma_16816_z(c[nt], pa[0], pb[0], pa[1], pb[1], x0[nt].x, x0[nt].y);
+                        mma_16816(c[nt], pa[2], pb[2], pa[3], pb[3], x0[nt].z, x0[nt].w);
                     }
                 }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     if (BITS == 4) {
                         mma_16816(c[nt], pa[4], pb[4], pa[6], pb[6], x0[nt].z, x0[nt].w);
-                        mma_16816(d[nt], pa[5], pb[5], pa[7], pb[7], x1[nt].z, x1[nt].w);
+                        mma_16816(c[nt], pa[5], pb[5], pa[7], pb[7], x1[nt].z, x1[nt].w);
                     } else {
                         mma_16816(c[nt], pa[4], pb[4], pa[5], pb[5], x1[nt].x, x1[nt].y);
-                        mma_16816(d[nt], pa[6], pb[6], pa[7], pb[7], x1[nt].z, x1[nt].w);
+                        mma_16816(c[nt], pa[6], pb[6], pa[7], pb[7], x1[nt].z, x1[nt].w);
                     }
                 }
                 if (ROT) {   // the lo part of the rotated x through the same codes
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        const int n = nt * 8 + gid;
-                        uint4 l0 = make_uint4(0, 0, 0, 0), l1 = l0;
-                        if (n < a.B) {
-                            l0 = xs_lo[((g * 2 + 0) * a.B + n) * 4 + tig];
-                            l1 = xs_lo[((g * 2 + 1) * a.B + n) * 4 + tig];
-                        }
+                        const int n = min(nt * 8 + gid, a.B - 1);
+                        const uint4 l0 = xs_lo[((g * 2 + 0) * a.B + n) * 4 + tig];
+                        const uint4 l1 = xs_lo[((g * 2 + 1) * a.B + n) * 4 + tig];
                         if (BITS == 4) {
                             mma_16816(c[nt], pa[0], pb[0], pa[2], pb[2], l0.x, l0.y);
-                            mma_16816(d[nt], pa[1], pb[1], pa[3], pb[3], l1.x, l1.y);
+                            mma_16816(c[nt], pa[1], pb[1], pa[3], pb[3], l1.x, l1.y);
                             mma_16816(c[nt], pa[4], pb[4], pa[6], pb[6], l0.z, l0.w);
-                            mma_16816(d[nt], pa[5], pb[5], pa[7], pb[7], l1.z, l1.w);
+                            mma_16816(c[nt], pa[5], pb[5], pa[7], pb[7], l1.z, l1.w);
                         } else {
                             mma_16816(c[nt], pa[0], pb[0], pa[1], pb[1], l0.x, l0.y);
-                            mma_16816(d[nt], pa[2], pb[2], pa[3], pb[3], l0.z, l0.w);
+                            mma_16816(c[nt], pa[2], pb[2], pa[3], pb[3], l0.z, l0.w);
                             mma_16816(c[nt], pa[4], pb[4], pa[5], pb[5], l1.x, l1.y);
-                            mma_16816(d[nt], pa[6], pb[6], pa[7], pb[7], l1.z, l1.w);
+                            mma_16816(c[nt], pa[6], pb[6], pa[7], pb[7], l1.z, l1.w);
                         }
                     }
                 }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    float r[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        r[i] = c[nt][i] + d[nt][i];
+                    const float *r = c[nt];
                     const float2 X = *reinterpret_cast<const float2 *>(xsum + g * 32 + nt * 8 + 2 * tig);
                     acc[nt][0] = fmaf(b_lo, X.x, fmaf(s_lo, r[0], acc[nt][0]));
                     acc[nt][1] = fmaf(b_lo, X.y, fmaf(s_lo, r[1], acc[nt][1]));

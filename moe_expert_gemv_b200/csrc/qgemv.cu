@@ -99,7 +99,9 @@ __host__ __device__ inline QgLayout qg_layout(int K, int bits, int ncol, int NS,
     return L;
 }
 
-template <int BITS, bool SWZ, int FMT, bool ROT>
+// ONE: a batch of one token (only MMA column 0 is kept, so the per-group
+// scale and bias steps of the other columns are left out)
+template <int BITS, bool SWZ, int FMT, bool ROT, bool ONE>
 __global__ void __launch_bounds__(QG_THREADS, 1)
     qgemv_kernel(QgemvArgs a, int NS, const __grid_constant__ CUtensorMap codes_map,
                  const __grid_constant__ CUtensorMap sb0_map,
@@ -279,15 +281,23 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                 } else
                     mma_group_s8_1(r, *reinterpret_cast<const uint4 *>(fa),
                                    *reinterpret_cast<const uint4 *>(fb), x0, x1);
-                const float2 X = *reinterpret_cast<const float2 *>(xsum + g * 8 + 2 * tig);
-                aq[0] = fmaf(s_lo, r[0], aq[0]);
-                aq[1] = fmaf(s_lo, r[1], aq[1]);
-                aq[2] = fmaf(s_hi, r[2], aq[2]);
-                aq[3] = fmaf(s_hi, r[3], aq[3]);
-                ab[0] = fmaf(b_lo, X.x, ab[0]);
-                ab[1] = fmaf(b_lo, X.y, ab[1]);
-                ab[2] = fmaf(b_hi, X.x, ab[2]);
-                ab[3] = fmaf(b_hi, X.y, ab[3]);
+                if (ONE) {
+                    const float X = xsum[g * 8];
+                    aq[0] = fmaf(s_lo, r[0], aq[0]);
+                    aq[2] = fmaf(s_hi, r[2], aq[2]);
+                    ab[0] = fmaf(b_lo, X, ab[0]);
+                    ab[2] = fmaf(b_hi, X, ab[2]);
+                } else {
+                    const float2 X = *reinterpret_cast<const float2 *>(xsum + g * 8 + 2 * tig);
+                    aq[0] = fmaf(s_lo, r[0], aq[0]);
+                    aq[1] = fmaf(s_lo, r[1], aq[1]);
+                    aq[2] = fmaf(s_hi, r[2], aq[2]);
+                    aq[3] = fmaf(s_hi, r[3], aq[3]);
+                    ab[0] = fmaf(b_lo, X.x, ab[0]);
+                    ab[1] = fmaf(b_lo, X.y, ab[1]);
+                    ab[2] = fmaf(b_hi, X.x, ab[2]);
+                    ab[3] = fmaf(b_hi, X.y, ab[3]);
+                }
             };
             // fragment address of row r, group g
             auto frag = [&](int r, int g) -> const void * {
@@ -438,7 +448,8 @@ cudaError_t launch_qgemv_t(const QgemvArgs &a, const LaunchCfg &c, const CUtenso
     const int n_items = (a.N + 15) / 16;
     const int grid = n_items < c.num_sms ? n_items : c.num_sms;
     cudaError_t e;
-    if ((e = set_smem(qgemv_kernel<BITS, SWZ, FMT, ROT>, L.total)) != cudaSuccess)
+    if ((e = set_smem(qgemv_kernel<BITS, SWZ, FMT, ROT, false>, L.total)) != cudaSuccess ||
+        (e = set_smem(qgemv_kernel<BITS, SWZ, FMT, ROT, true>, L.total)) != cudaSuccess)
         return e;
     // scales and biases (or the parameter words) transposed by tensor copies
     // where the rows take the swizzled tile path and G % 64 == 0
@@ -454,7 +465,10 @@ cudaError_t launch_qgemv_t(const QgemvArgs &a, const LaunchCfg &c, const CUtenso
         else
             sbT = encode_param_map_t(&m0, a.params, a.N, G, 4);
     }
-    return launch_ex(qgemv_kernel<BITS, SWZ, FMT, ROT>, dim3(grid), dim3(QG_THREADS), L.total, c, 1,
+    if (a.B == 1)
+        return launch_ex(qgemv_kernel<BITS, SWZ, FMT, ROT, true>, dim3(grid), dim3(QG_THREADS),
+                         L.total, c, 1, a, NS, m, m0, m1, sbT);
+    return launch_ex(qgemv_kernel<BITS, SWZ, FMT, ROT, false>, dim3(grid), dim3(QG_THREADS), L.total, c, 1,
                      a, NS, m, m0, m1, sbT);
 }
 

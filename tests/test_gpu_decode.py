@@ -55,6 +55,28 @@ def test_small_stacks(cuda_dev, E, H, I, k, n):
     check_layers(ms, E, H, I, k, x16, y, idx, wt, lg)
 
 
+def test_router_ties_lowest_index(cuda_dev):
+    """Exact ties inside the fused router: three identical router rows
+    (experts 5, 9 and 77, made the largest; their logits come from different
+    CTAs of a cluster) and an all-zero input (every logit 0) select the lower
+    index first, as the oracle's rule does."""
+    E, H, I, k = 128, 1024, 256, 8
+    ms = [synth.moe_layer(11, l, E=E, H=H, I=I) for l in range(2)]
+    P, S, B = (np.array(v, copy=True) for v in ms[0]["router"])
+    B[[5, 9, 77], :] = synth.to_f16_bits(np.full(H // 64, 10.0))
+    for r in (9, 77):
+        P[r], S[r], B[r] = P[5], S[5], B[5]
+    ms[0]["router"] = (P, S, B)
+    stack = qmoe.DecodeStack([qmoe.MoELayer.from_numpy(m, E, H, I) for m in ms], k)
+    xp = np.abs(synth.activations(12, 1, H, layer=0).view(np.float16)).astype(np.float64)
+    x16 = np.concatenate([synth.to_f16_bits(xp), np.zeros((1, H), np.uint16)])
+    y, idx, wt, lg = run(stack, x16, E, k)
+    assert lg[0, 5] == lg[0, 9] == lg[0, 77]
+    assert list(idx[0, :3]) == [5, 9, 77]
+    assert np.all(lg[1] == 0) and list(idx[1]) == list(range(k)) and np.all(wt[1] == 1.0 / k)
+    check_layers(ms, E, H, I, k, x16, y, idx, wt, lg)
+
+
 def test_moe_e128_three_layers_and_repeat(cuda_dev):
     E, H, I, k = synth.MOE_E, synth.MOE_H, synth.MOE_I, synth.MOE_TOPK
     ms, stack = make_stack(3, 3, E, H, I, k)

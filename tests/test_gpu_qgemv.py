@@ -239,10 +239,9 @@ def test_long_8bit_rows_take_fewer_rows_per_launch(cuda_dev, Bt):
 
 
 def test_rows_too_long_for_one_tile_unsupported(cuda_dev):
-    """A 16-row tile of 8-bit rows of 11072 columns plus one row of x does
-    not fit in shared memory (11008 is the longest that does): UNSUPPORTED,
-    and nothing is launched."""
-    N, K = 16, 11072
+    """A 16-row tile of 8-bit rows of 11008 columns plus one row of x does
+    not fit in shared memory: UNSUPPORTED, and nothing is launched."""
+    N, K = 16, 11008
     P, S, B = synth.qmatrix(synth.rng(N, K, 8, 42), N, K, 8)
     W = qmoe.QMatrix.from_numpy(P, S, B, N, K, 8)
     x = to_dev_f16(synth.activations(43, 1, K))
@@ -250,3 +249,16 @@ def test_rows_too_long_for_one_tile_unsupported(cuda_dev):
         qmoe.qgemv_affine(W, x)
     assert e.value.code == qmoe.ERR_UNSUPPORTED
     assert qmoe.qmoe_check_status() == 0
+
+
+@pytest.mark.parametrize("bits,K", [(8, 10944), (4, 18624)])
+def test_longest_rows_one_tile_takes(cuda_dev, bits, K):
+    """The longest rows the header documents for one row of x (10944 columns
+    at 8 bits, 18624 at 4 bits) run, with a ragged 24-row matrix, against the
+    oracle."""
+    N = 24
+    P, S, B = synth.qmatrix(synth.rng(N, K, bits, 44), N, K, bits)
+    x16 = synth.activations(45, 1, K)
+    y = run_qgemv(P, S, B, N, K, bits, x16)
+    y64, _ = oracle.qgemv(P, S, B, N, K, bits, x16)
+    assert_close_rows(y.view(np.float16), y64, what="%d-bit K=%d" % (bits, K))
