@@ -16,7 +16,7 @@ CPU oracle timed on a bounded sample (`cpu_baseline`).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload moe_decode|qgemv|qgemv_fmt|router|prefill|
                               expert_cache|expert_parallel]
-                  [--layers L] [--qgemv-batch 1,4,8,16,32]
+                  [--layers L] [--qgemv-batch 1,4,8,16,32] [--router-tokens 1,...,128]
 
 The other workloads print one JSON line of per-kernel numbers each: dense
 qGEMV at batch 1..32 (one pass over the weights from batch 9 on), the
@@ -56,9 +56,9 @@ ROUTER_CALL_BYTES = ROUTER_BYTES + H * 2 + TOPK * 8
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source it was taken on (sha256 of csrc/decode.cu); otherwise reported null.
 NCU_TRAFFIC = {
-    # 6-layer capture (183,117,312 B read + 3,729,408 B written) scaled to
+    # 6-layer capture (183,116,544 B read + 4,021,248 B written) scaled to
     # the 30 layers of one launch
-    "moe_decode_kernel": {"bytes": 934233600, "sha": "4cf7b9364af2122f"},
+    "moe_decode_kernel": {"bytes": 935688960, "sha": "9e3827855bf2d02c"},
 }
 
 
@@ -74,6 +74,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--qgemv-batch", default="1,4,8,16,32",
                     help="batch sizes of the qgemv workload (comma-separated)")
+    ap.add_argument("--router-tokens", default="1,2,4,8,16,32,64,128",
+                    help="token counts of the router workload (comma-separated)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="time budget of the CPU-oracle baseline sample")
@@ -604,7 +606,7 @@ def main_other(args):
     elif args.workload == "router":
         P, S, B = synth.router(args.seed)
         R = qmoe.QMatrix.from_numpy(P, S, B, E, H, 8, dev)
-        for T in (1, 2, 4, 8, 16, 32, 64, 128):
+        for T in [int(t) for t in args.router_tokens.split(",")]:
             x = torch.from_numpy(synth.activations(T, T, H).view(np.float16).copy()).to(dev)
             idx = torch.empty(T, TOPK, dtype=torch.int32, device=dev)
             wt = torch.empty(T, TOPK, dtype=torch.float32, device=dev)
