@@ -56,8 +56,6 @@ namespace {
 
 constexpr int QG_CW = 16;                     // consumer warps
 constexpr int QG_CT = QG_CW * 32;             // consumer threads
-constexpr int QG_GW = 4;                      // warps per tile group
-constexpr int QG_NG = QG_CW / QG_GW;          // tile groups: tile k goes to group k % QG_NG
 constexpr int QG_THREADS = QG_CT + 32;        // + one producer warp
 constexpr int QG_MAX_STAGES = 8;
 
@@ -100,8 +98,9 @@ __host__ __device__ inline QgLayout qg_layout(int K, int bits, int ncol, int NS,
 }
 
 // ONE: a batch of one token (only MMA column 0 is kept, so the per-group
-// scale and bias steps of the other columns are left out)
-template <int BITS, bool SWZ, int FMT, bool ROT, bool ONE>
+// scale and bias steps of the other columns are left out).  GW: consumer
+// warps per tile group (4; 8 for a full batch of 8, measured faster there)
+template <int BITS, bool SWZ, int FMT, bool ROT, bool ONE, int GW>
 __global__ void __launch_bounds__(QG_THREADS, 1)
     qgemv_kernel(QgemvArgs a, int NS, const __grid_constant__ CUtensorMap codes_map,
                  const __grid_constant__ CUtensorMap sb0_map,
@@ -131,7 +130,7 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], QG_GW);   // the warps of the consuming tile group
+            mbar_init(&empty[s], GW);   // the warps of the consuming tile group
             s_arm[s] = -1;
         }
         *xzero = make_uint4(0, 0, 0, 0);
@@ -213,18 +212,19 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
                       ctid, QG_CT);
     named_bar_sync(1, QG_CT);
 
-    // tiles go to groups of QG_GW warps (tile k to group k % QG_NG); a warp
+    // tiles go to groups of GW warps (tile k to group k % NG); a warp
     // takes a contiguous quarter of the tile's groups, so that with G % 64 ==
     // 0 the scales and biases of a row come as one 8-byte load per 4 groups,
     // and the group's partial sums meet at a barrier of its own
-    const int grp = warp / QG_GW, wq = warp % QG_GW;
-    const int gpw = (L.G + QG_GW - 1) / QG_GW;
+    constexpr int NG = QG_CW / GW;   // tile groups
+    const int grp = warp / GW, wq = warp % GW;
+    const int gpw = (L.G + GW - 1) / GW;
     const int g0 = min(L.G, wq * gpw), g1 = min(L.G, g0 + gpw);
     const bool vec_sb = (L.G & 63) == 0;
     const int gid = lane >> 2, tig = lane & 3;
     bool failed = false;
     int kk = 0;   // tiles this group has done (alternates its partial-sum buffers)
-    for (int k = grp; blockIdx.x + k * gridDim.x < n_items; k += QG_NG, ++kk) {
+    for (int k = grp; blockIdx.x + k * gridDim.x < n_items; k += NG, ++kk) {
         const int item = blockIdx.x + k * gridDim.x;
         const int st = k % NS, use = k / NS;
         if (!failed && !(wait_armed(s_arm + st, k, a.status) && mbar_wait(&full[st], use & 1, a.status)))
@@ -383,12 +383,12 @@ __global__ void __launch_bounds__(QG_THREADS, 1)
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&empty[st]);
-        float4 *gred = red + (size_t)((grp * 2 + (kk & 1)) * QG_GW) * 32;
+        float4 *gred = red + (size_t)((grp * 2 + (kk & 1)) * GW) * 32;
         gred[wq * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        named_bar_sync(2 + grp, QG_GW * 32);
-        if (wq == kk % QG_GW) {
+        named_bar_sync(2 + grp, GW * 32);
+        if (wq == kk % GW) {
             float v[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int w = 0; w < QG_GW; ++w) {
+            for (int w = 0; w < GW; ++w) {
                 const float4 p = gred[w * 32 + lane];
                 v[0] += p.x;
                 v[1] += p.y;
@@ -448,8 +448,9 @@ cudaError_t launch_qgemv_t(const QgemvArgs &a, const LaunchCfg &c, const CUtenso
     const int n_items = (a.N + 15) / 16;
     const int grid = n_items < c.num_sms ? n_items : c.num_sms;
     cudaError_t e;
-    if ((e = set_smem(qgemv_kernel<BITS, SWZ, FMT, ROT, false>, L.total)) != cudaSuccess ||
-        (e = set_smem(qgemv_kernel<BITS, SWZ, FMT, ROT, true>, L.total)) != cudaSuccess)
+    if ((e = set_smem(qgemv_kernel<BITS, SWZ, FMT, ROT, false, 4>, L.total)) != cudaSuccess ||
+        (e = set_smem(qgemv_kernel<BITS, SWZ, FMT, ROT, false, 8>, L.total)) != cudaSuccess ||
+        (e = set_smem(qgemv_kernel<BITS, SWZ, FMT, ROT, true, 4>, L.total)) != cudaSuccess)
         return e;
     // scales and biases (or the parameter words) transposed by tensor copies
     // where the rows take the swizzled tile path and G % 64 == 0
@@ -466,9 +467,12 @@ cudaError_t launch_qgemv_t(const QgemvArgs &a, const LaunchCfg &c, const CUtenso
             sbT = encode_param_map_t(&m0, a.params, a.N, G, 4);
     }
     if (a.B == 1)
-        return launch_ex(qgemv_kernel<BITS, SWZ, FMT, ROT, true>, dim3(grid), dim3(QG_THREADS),
+        return launch_ex(qgemv_kernel<BITS, SWZ, FMT, ROT, true, 4>, dim3(grid), dim3(QG_THREADS),
                          L.total, c, 1, a, NS, m, m0, m1, sbT);
-    return launch_ex(qgemv_kernel<BITS, SWZ, FMT, ROT, false>, dim3(grid), dim3(QG_THREADS), L.total, c, 1,
+    if (a.B == 8)
+        return launch_ex(qgemv_kernel<BITS, SWZ, FMT, ROT, false, 8>, dim3(grid), dim3(QG_THREADS),
+                         L.total, c, 1, a, NS, m, m0, m1, sbT);
+    return launch_ex(qgemv_kernel<BITS, SWZ, FMT, ROT, false, 4>, dim3(grid), dim3(QG_THREADS), L.total, c, 1,
                      a, NS, m, m0, m1, sbT);
 }
 
