@@ -474,7 +474,7 @@ def main_other(args):
     import torch
     from moe_expert_gemv_b200 import qmoe, synth
     dev = torch.device("cuda", 0)
-    hbm, _, peak_kind = peaks()
+    hbm, tflops, peak_kind = peaks()
     out = {"workload": args.workload, "peak_gbs": hbm, "peak_kind": peak_kind, "results": []}
     if args.workload == "qgemv":
         for N in (14336, 4096):
@@ -504,6 +504,43 @@ def main_other(args):
                 out["results"].append({"N": N, "K": K, "B": Bt, "us": round(ms * 1e3, 3),
                                        "GB/s": round(gbs, 1), "frac": round(gbs / hbm, 4),
                                        "rotated_copies": copies})
+        # the small case: N=512, K=1024, batch 1 (295 KB of weights, which fit
+        # L2): hot (the same matrix every call) and cold (L2 flushed by a
+        # 2 x L2 write before each call, the call alone timed)
+        N, K = 512, 1024
+        P, S, B = synth.dense(0, N, K)
+        W = qmoe.QMatrix.from_numpy(P, S, B, N, K, 4, dev)
+        x = torch.from_numpy(synth.activations(1, 1, K).view(np.float16).copy()).to(dev)
+        y = torch.empty(1, N, dtype=torch.float16, device=dev)
+        nbytes = N * K // 2 + 2 * N * (K // 64) * 2 + (K + N) * 2
+
+        def run_small():
+            for _ in range(20):
+                qmoe.qgemv_affine(W, x, y)
+        run_small()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run_small()
+        for _ in range(3):
+            g.replay()
+        reps = max(10, args.steps // 10)
+        hot_ms = timed_replays(g.replay, reps) / (reps * 20)
+        flush = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size,
+                            dtype=torch.uint8, device=dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        cold = []
+        for i in range(max(20, args.steps // 5)):
+            flush.fill_(i & 255)
+            e0.record()
+            qmoe.qgemv_affine(W, x, y)
+            e1.record()
+            e1.synchronize()
+            cold.append(e0.elapsed_time(e1))
+        cold_ms = float(np.median(cold))
+        out["results"].append({"N": N, "K": K, "B": 1, "us_hot": round(hot_ms * 1e3, 3),
+                               "us_cold": round(cold_ms * 1e3, 3),
+                               "GB/s_cold": round(nbytes / (cold_ms / 1e3) / 1e9, 1),
+                               "frac_cold": round(nbytes / (cold_ms / 1e3) / 1e9 / hbm, 4)})
     elif args.workload == "qgemv_fmt":
         # bf16-scale formats with the block-32 rotation of x, the K=4096 dense shapes
         for fmt, name in ((qmoe.FMT_ZP4_BF16, "zp4_bf16"), (qmoe.FMT_SYM8_BF16, "sym8_bf16")):
@@ -663,12 +700,18 @@ def main_other(args):
                     heavy = int((counts >= tmin).sum() + (T >= tmin)) if tmin else 0
                     nbytes = (touched + 1) * EXPERT_BYTES
                     gbs = nbytes / (ms / 1e3) / 1e9
+                    # the attainable time: the slower of streaming the touched
+                    # weights at the HBM peak and the useful flops at the
+                    # dense bf16 peak
+                    att_us = max(nbytes / (hbm * 1e9), flops / (tflops * 1e12)) * 1e6
                     out["results"].append({
                         "T": T, "routing": routing, "tensor_min_tokens": tmin,
                         "tensor_core_slots": heavy, "experts_touched": touched,
                         "us": round(ms * 1e3, 2), "tokens_per_s": round(T / (ms / 1e3), 1),
                         "weight_GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
-                        "useful_TFLOP/s": round(flops / (ms / 1e3) / 1e12, 2)})
+                        "useful_TFLOP/s": round(flops / (ms / 1e3) / 1e12, 2),
+                        "attainable_us": round(att_us, 2),
+                        "frac_attainable": round(att_us / (ms * 1e3), 4)})
         finally:
             qmoe.qmoe_set_prefill_tensor_min(old_min)
     else:
