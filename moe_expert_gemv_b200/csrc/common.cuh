@@ -421,27 +421,10 @@ __device__ __forceinline__ const void *swz128_frag(const unsigned char *tile, in
 // Subnormal-code group product of a 16-row tile (rows gid, gid+8 from wa, wb;
 // x fragments in the order of xperm(kPermS4, .) for 4-bit, xperm(8, .) for
 // 8-bit): returns sum_k q x per C element, scaled by 2^-18 (4-bit) or 2^-22
-// (8-bit).  Two accumulators (c, d) per call keep two mma chains in flight.
-__device__ __forceinline__ void mma_group_s4(float (&r)[4], uint2 wa, uint2 wb, uint4 x0, uint4 x1)
-{
-    uint32_t pa[8], pb[8];
-    dequant4s_word(wa.x, pa);
-    dequant4s_word(wa.y, pa + 4);
-    dequant4s_word(wb.x, pb);
-    dequant4s_word(wb.y, pb + 4);
-    float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
-    mma_16816(c, pa[0], pb[0], pa[2], pb[2], x0.x, x0.y);
-    mma_16816(d, pa[1], pb[1], pa[3], pb[3], x1.x, x1.y);
-    mma_16816(c, pa[4], pb[4], pa[6], pb[6], x0.z, x0.w);
-    mma_16816(d, pa[5], pb[5], pa[7], pb[7], x1.z, x1.w);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        r[i] = c[i] + d[i];
-}
-// One 64-input group in a single accumulator chain (the four products
-// added in the tensor core, the first into a fresh accumulator): fewer
-// instructions than two chains joined by fp32 adds, for callers with enough
-// independent groups in flight to hide the longer chain.
+// (8-bit).  The four products of the group are added in one accumulator
+// chain, the first into a fresh accumulator: fewer instructions than two
+// chains joined by fp32 adds (measured faster in every caller, which all keep
+// enough independent groups in flight to hide the longer chain).
 __device__ __forceinline__ void mma_group_s4_1(float (&r)[4], uint2 wa, uint2 wb, uint4 x0, uint4 x1)
 {
     uint32_t pa[8], pb[8];
@@ -470,33 +453,12 @@ __device__ __forceinline__ void mma_group_s8_1(float (&r)[4], uint4 wa, uint4 wb
     mma_16816(r, pa[4], pb[4], pa[5], pb[5], x1.x, x1.y);
     mma_16816(r, pa[6], pb[6], pa[7], pb[7], x1.z, x1.w);
 }
-__device__ __forceinline__ void mma_group_s8(float (&r)[4], uint4 wa, uint4 wb, uint4 x0, uint4 x1)
-{
-    uint32_t pa[8], pb[8];
-    dequant8s_word(wa.x, pa);
-    dequant8s_word(wb.x, pb);
-    dequant8s_word(wa.y, pa + 2);
-    dequant8s_word(wb.y, pb + 2);
-    dequant8s_word(wa.z, pa + 4);
-    dequant8s_word(wb.z, pb + 4);
-    dequant8s_word(wa.w, pa + 6);
-    dequant8s_word(wb.w, pb + 6);
-    float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
-    mma_16816(c, pa[0], pb[0], pa[1], pb[1], x0.x, x0.y);
-    mma_16816(d, pa[2], pb[2], pa[3], pb[3], x0.z, x0.w);
-    mma_16816(c, pa[4], pb[4], pa[5], pb[5], x1.x, x1.y);
-    mma_16816(d, pa[6], pb[6], pa[7], pb[7], x1.z, x1.w);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        r[i] = c[i] + d[i];
-}
-
 // The same products with an activation held as an fp16 (hi, lo) pair: the
-// codes are dequantised once and the result is that of mma_group_s4 /
-// mma_group_s8 applied to hi + lo.  The lo products (about 2^-11 of the hi
+// codes are dequantised once and the result is that of mma_group_s4_1 /
+// mma_group_s8_1 applied to hi + lo.  The lo products (about 2^-11 of the hi
 // ones) accumulate in their own registers and meet the hi sums only in an
-// fp32 add: chained into the hi accumulator, part of their bits were lost
-// inside the tensor-core addition.
+// fp32 add: a B200 probe of mma.sync measured twice the error (relative to
+// sum |a b|) when they were chained into the hi accumulator instead.
 __device__ __forceinline__ void mma_group_s4_hilo(float (&r)[4], uint2 wa, uint2 wb, uint4 h0,
                                                   uint4 h1, uint4 l0, uint4 l1)
 {

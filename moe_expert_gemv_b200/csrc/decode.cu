@@ -401,7 +401,7 @@ __device__ __forceinline__ float2 sb_word(const unsigned char *p)
 
 // The h of a unit (64 intermediate indices k, fp16 hi and lo columns) sits in
 // hfrag[unit] as the down projection's B fragments [hh][col][tig][8], in the x
-// order of mma_group_s4: index k = 16 tig + xperm_s4(8 hh + e) at slot
+// order of mma_group_s4_1: index k = 16 tig + xperm_s4(8 hh + e) at slot
 // ((hh * 2 + col) * 4 + tig) * 8 + e.
 
 // ------------------------------------------------------------------ kernel --
