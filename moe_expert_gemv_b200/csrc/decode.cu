@@ -245,15 +245,31 @@ __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v)
 {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
-__device__ __forceinline__ void st_cluster_v4f32(uint32_t addr, float4 v)
-{
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x),
-                 "f"(v.y), "f"(v.z), "f"(v.w)
-                 : "memory");
-}
 __device__ __forceinline__ void st_cluster_v2u32(uint32_t addr, uint32_t a, uint32_t b)
 {
     asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b)
+                 : "memory");
+}
+// stores into a CTA of the cluster that complete `bytes` of the transaction
+// count of an mbarrier in that CTA (the receiver's wait then sees the data):
+// no release fence and no separate remote arrive on the sender's side
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float4 v, uint32_t mbar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+                 "r"(__float_as_uint(v.x)), "r"(__float_as_uint(v.y)), "r"(__float_as_uint(v.z)),
+                 "r"(__float_as_uint(v.w)), "r"(mbar)
+                 : "memory");
+}
+__device__ __forceinline__ void st_async_b32(uint32_t addr, uint32_t v, uint32_t mbar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
+                 "r"(mbar)
+                 : "memory");
+}
+__device__ __forceinline__ void st_async_v2(uint32_t addr, uint32_t a, uint32_t b, uint32_t mbar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];" ::"r"(addr),
+                 "r"(a), "r"(b), "r"(mbar)
                  : "memory");
 }
 // fire-and-forget vector add (no value returned, so the thread does not wait)
@@ -268,14 +284,6 @@ __device__ __forceinline__ void red_add_v4(float4 *p, float4 v)
 __device__ __forceinline__ void red_release_add(unsigned *p, unsigned v)
 {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-// arrive on an mbarrier of a CTA of the cluster; orders this thread's
-// earlier shared::cluster stores before the arrival
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster_addr)
-{
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
-                     bar_cluster_addr)
-                 : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t *bar, uint32_t parity)
 {
@@ -458,10 +466,10 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
         mbar_init(rfull, 1);
         mbar_init(rempty, 1);
         mbar_init(topk_bar, 1);
-        mbar_init(logit_bar, DC_CLUSTER);
+        mbar_init(logit_bar, 1);   // the exchange warp's expect; the bytes by st.async
         mbar_init(red_bar, DC_CW);
         for (int s = 0; s < DC_MAX_UNITS; ++s) {
-            mbar_init(&hbar[s], DC_CLUSTER);
+            mbar_init(&hbar[s], 1);   // the local exchange warp; the others' bytes by st.async
             mbar_init(&gubar[s], DC_GW);
         }
         for (int j = 0; j < 16; ++j)
@@ -603,6 +611,10 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
         bool ok = true;
         for (int l = 0; l < a.L && ok; ++l) {
             if (xw == 0) {
+                // the other CTAs' logits of this layer (Rr from each) complete
+                // the phase; this CTA's own are written in place by this warp
+                if (lane == 0)
+                    mbar_arrive_expect_tx(logit_bar, (uint32_t)((DC_CLUSTER - 1) * Rr * 4));
                 ok = __all_sync(0xffffffffu, wait_bar(a, red_bar, l & 1));
                 if (!ok)
                     break;
@@ -620,17 +632,17 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                         s_logit[Rr * rank + lane] = v;
                 }
                 __syncwarp();
-                if (lane < DC_CLUSTER) {
+                if (lane < DC_CLUSTER && lane != (int)rank) {
                     const float *mine = s_logit + Rr * rank;
                     const uint32_t tb = mapa_rank(smem_u32(mine), lane);
+                    const uint32_t tbar = mapa_rank(smem_u32(logit_bar), lane);
                     if ((Rr & 3) == 0) {
                         for (int i = 0; i < Rr; i += 4)
-                            st_cluster_v4f32(tb + 4 * i, *reinterpret_cast<const float4 *>(mine + i));
+                            st_async_v4(tb + 4 * i, *reinterpret_cast<const float4 *>(mine + i), tbar);
                     } else {
                         for (int i = 0; i < Rr; ++i)
-                            st_cluster_f32(tb + 4 * i, mine[i]);
+                            st_async_b32(tb + 4 * i, __float_as_uint(mine[i]), tbar);
                     }
-                    mbar_arrive_remote(mapa_rank(smem_u32(logit_bar), lane));
                 }
             }
             // ---- top-k of this layer (exchange warp 0): each round's
@@ -758,20 +770,37 @@ __global__ void __cluster_dims__(DC_CLUSTER, 1, 1) __launch_bounds__(DC_THREADS,
                 }
                 if (lane < DC_CLUSTER) {
                     // the CTA's 8 indices k = 8 rank + j sit, per (hh, column),
-                    // in 4 consecutive fragment slots: j = hh + (0, 4, 2, 6)
+                    // in 4 consecutive fragment slots: j = hh + (0, 4, 2, 6);
+                    // the other CTAs' copies go by st.async (36 bytes each,
+                    // counted on their hbar), this CTA's own by plain stores
                     const uint32_t tb = mapa_rank(smem_u32(hfrag + (size_t)s * 128), lane);
+                    const uint32_t ts = mapa_rank(smem_u32(hsum + s * DC_CLUSTER + rank), lane);
+                    const uint32_t tbar = mapa_rank(smem_u32(&hbar[s]), lane);
+                    const bool self = lane == (int)rank;
 #pragma unroll
                     for (int hf = 0; hf < 2; ++hf) {
                         const int pos_hi = ((hf * 2 + 0) * 4 + (rank >> 1)) * 8 + 4 * (rank & 1);
                         const int pos_lo = ((hf * 2 + 1) * 4 + (rank >> 1)) * 8 + 4 * (rank & 1);
-                        st_cluster_v2u32(tb + 2 * pos_hi, vh[hf] | (vh[hf + 4] << 16),
-                                         vh[hf + 2] | (vh[hf + 6] << 16));
-                        st_cluster_v2u32(tb + 2 * pos_lo, vl[hf] | (vl[hf + 4] << 16),
-                                         vl[hf + 2] | (vl[hf + 6] << 16));
+                        const uint32_t h0 = vh[hf] | (vh[hf + 4] << 16), h1 = vh[hf + 2] | (vh[hf + 6] << 16);
+                        const uint32_t l0 = vl[hf] | (vl[hf + 4] << 16), l1 = vl[hf + 2] | (vl[hf + 6] << 16);
+                        if (self) {
+                            st_cluster_v2u32(tb + 2 * pos_hi, h0, h1);
+                            st_cluster_v2u32(tb + 2 * pos_lo, l0, l1);
+                        } else {
+                            st_async_v2(tb + 2 * pos_hi, h0, h1, tbar);
+                            st_async_v2(tb + 2 * pos_lo, l0, l1, tbar);
+                        }
                     }
-                    st_cluster_f32(mapa_rank(smem_u32(hsum + s * DC_CLUSTER + rank), lane), part);
-                    mbar_arrive_remote(mapa_rank(smem_u32(&hbar[s]), lane));
+                    if (self)
+                        st_cluster_f32(ts, part);
+                    else
+                        st_async_b32(ts, __float_as_uint(part), tbar);
                 }
+                // this CTA's own part is written: arrive, expecting the other
+                // CTAs' bytes of this unit
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive_expect_tx(&hbar[s], (uint32_t)((DC_CLUSTER - 1) * 36));
             }
         }
     } else {
