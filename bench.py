@@ -56,10 +56,9 @@ ROUTER_CALL_BYTES = ROUTER_BYTES + H * 2 + TOPK * 8
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source it was taken on (sha256 of csrc/decode.cu); otherwise reported null.
 NCU_TRAFFIC = {
-    # 6-layer capture (183,116,544 B read + 4,021,248 B written) scaled to
-    # the 30 layers of one launch; captured at decode.cu 9e3827855bf2d02c,
-    # which differs from the file recorded here by one comment only
-    "moe_decode_kernel": {"bytes": 935688960, "sha": "42e9af7f8bf83cf9"},
+    # 6-layer capture (183,117,312 B read + 3,406,848 B written) scaled to
+    # the 30 layers of one launch
+    "moe_decode_kernel": {"bytes": 932620800, "sha": "9c52866a00c89cf7"},
 }
 
 
