@@ -56,9 +56,10 @@ ROUTER_CALL_BYTES = ROUTER_BYTES + H * 2 + TOPK * 8
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source it was taken on (sha256 of csrc/decode.cu); otherwise reported null.
 NCU_TRAFFIC = {
-    # 6-layer capture (183,117,312 B read + 3,406,848 B written) scaled to
-    # the 30 layers of one launch
-    "moe_decode_kernel": {"bytes": 932620800, "sha": "9c52866a00c89cf7"},
+    # 6-layer capture (183,141,120 B read + 3,689,728 B written) scaled to
+    # the 30 layers of one launch; the hash covers decode.cu and common.cuh
+    # (the dequantisation the kernel inlines)
+    "moe_decode_kernel": {"bytes": 934154240, "sha": "71a522c459eccb88"},
 }
 
 
@@ -94,9 +95,13 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-def source_sha(name):
-    with open(os.path.join(ROOT, "moe_expert_gemv_b200", "csrc", name), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_sha(*names):
+    """sha256[:16] of the named csrc files, concatenated in order."""
+    h = hashlib.sha256()
+    for name in names:
+        with open(os.path.join(ROOT, "moe_expert_gemv_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 class ClockSampler:
@@ -391,7 +396,7 @@ def main_decode(args):
     gbs = step_bytes / (launch_ms / 1e3) / 1e9
     trf = NCU_TRAFFIC.get("moe_decode_kernel")
     # traffic grows in proportion to the layers a launch streams
-    traffic = (round(trf["bytes"] * nl / 30) if trf and trf["sha"] == source_sha("decode.cu")
+    traffic = (round(trf["bytes"] * nl / 30) if trf and trf["sha"] == source_sha("decode.cu", "common.cuh")
                else None)
     line = {
         "metric": "qGEMV/MoE-layer weight-stream GB/s vs HBM peak; MoE decode layers/s",

@@ -272,22 +272,23 @@ __device__ __forceinline__ void dequant8_word(uint32_t w, uint32_t *p)
 }
 
 // Cheaper dequantisation for the streaming kernels: the code itself becomes
-// the fp16 bit pattern (no exponent bits), i.e. an fp16 subnormal.  Every
-// code is placed in the top mantissa bits (a nibble in bits 6..9: 64q *
-// 2^-24 = q * 2^-18; a byte in bits 2..9: b * 2^-22).  Measured on B200
-// (mma.sync m16n8k16, f16 x f16 -> f32): with the codes in the top mantissa
-// bits the products are as accurate as with the codes as normal fp16
-// integers (~1e-7 of sum |a b|); a nibble left in bits 0..3 (q * 2^-24)
-// loses up to 2e-5 of sum |a b|.  A word costs four shifts and four ANDs.
-// Pairs (both halves of a register):
+// the fp16 bit pattern (no exponent bits), i.e. an fp16 subnormal, placed
+// high in the mantissa: a nibble in bits 4..7 (16q * 2^-24 = q * 2^-20), a
+// byte in bits 2..9 (b * 2^-22).  Measured on B200 (mma.sync m16n8k16, f16 x
+// f16 -> f32, error relative to sum |a b|): codes as normal fp16 integers
+// ~1e-7, a byte in bits 2..9 1.6e-7, a nibble in bits 6..9 1.0-1.5e-7, in
+// bits 4..7 2.9-4.6e-7, in bits 0..3 up to 1.6e-5 (the low subnormals lose
+// bits inside the tensor core).  Bits 4..7 cost one shift fewer than 6..9
+// (one nibble pair is already in place: 3 shifts + 4 ANDs per word) and stay
+// far inside the error budget.  Pairs (both halves of a register):
 //   p[0] = (c0, c4)   p[1] = (c1, c5)   p[2] = (c2, c6)   p[3] = (c3, c7)
-// all in units of 2^-18; callers scale results by kCode4 = 2^18.
+// all in units of 2^-20; callers scale results by kCode4 = 2^20.
 __device__ __forceinline__ void dequant4s_word(uint32_t w, uint32_t *p)
 {
-    p[0] = (w << 6) & 0x03C003C0u;
-    p[1] = (w << 2) & 0x03C003C0u;
-    p[2] = (w >> 2) & 0x03C003C0u;
-    p[3] = (w >> 6) & 0x03C003C0u;
+    p[0] = (w << 4) & 0x00F000F0u;
+    p[1] = w & 0x00F000F0u;
+    p[2] = (w >> 4) & 0x00F000F0u;
+    p[3] = (w >> 8) & 0x00F000F0u;
 }
 // 8-bit: bytes as subnormals b * 2^-22: p[0] = (c0, c2), p[1] = (c1, c3).
 __device__ __forceinline__ void dequant8s_word(uint32_t w, uint32_t *p)
@@ -295,7 +296,7 @@ __device__ __forceinline__ void dequant8s_word(uint32_t w, uint32_t *p)
     p[0] = (w << 2) & 0x03FC03FCu;
     p[1] = (w >> 6) & 0x03FC03FCu;
 }
-constexpr float kCode4 = 262144.f;    // 2^18: undoes dequant4s_word
+constexpr float kCode4 = 1048576.f;   // 2^20: undoes dequant4s_word
 constexpr float kCode8 = 4194304.f;   // 2^22: undoes dequant8s_word
 
 // x order matching dequant4s_word, k-blocks (c0,c4)(c2,c6) | (c8,c12)(c10,c14)

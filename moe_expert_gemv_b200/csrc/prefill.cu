@@ -549,7 +549,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         off[j] = gid * st.S * 4 + j * 32 + tig * 8;
                 }
                 // code products and folded biases accumulate apart; the
-                // subnormal factor 2^18 is applied once at the end
+                // subnormal factor kCode4 is applied once at the end
                 float aq[4] = {0.f, 0.f, 0.f, 0.f}, ab[4] = {0.f, 0.f, 0.f, 0.f};
                 const int nch = d.GH / 4;
                 for (int q4 = 0; q4 < nch; ++q4) {
