@@ -421,7 +421,7 @@ __device__ __forceinline__ const void *swz128_frag(const unsigned char *tile, in
 
 // Subnormal-code group product of a 16-row tile (rows gid, gid+8 from wa, wb;
 // x fragments in the order of xperm(kPermS4, .) for 4-bit, xperm(8, .) for
-// 8-bit): returns sum_k q x per C element, scaled by 2^-18 (4-bit) or 2^-22
+// 8-bit): returns sum_k q x per C element, scaled by 2^-20 (4-bit) or 2^-22
 // (8-bit).  The four products of the group are added in one accumulator
 // chain, the first into a fresh accumulator: fewer instructions than two
 // chains joined by fp32 adds (measured faster in every caller, which all keep
