@@ -497,9 +497,12 @@ uint64_t qmoe_set_decode_wait_limit_ns(uint64_t ns);
 
 /* Experts of a prefill chunk (and the shared expert) with at least
  * `min_tokens` tokens run on the tensor-core (tcgen05) kernels, the others on
- * the streaming kernels; 0 sends every expert to the streaming kernels.  The
- * default is 16.  Applies to later moe_prefill_qgemm calls in this process;
- * returns the previous setting. */
+ * the streaming kernels; 0 (the default) sends every expert to the streaming
+ * kernels, which are the faster choice on skewed (Zipf) routing; 16 is the
+ * threshold the tests use when they switch the tensor-core path on.  Shapes
+ * the tensor-core kernels do not take stay on the streaming kernels.
+ * Applies to later moe_prefill_qgemm calls in this process; returns the
+ * previous setting. */
 int32_t qmoe_set_prefill_tensor_min(int32_t min_tokens);
 
 /* Library version, major*10000 + minor*100 + patch. */

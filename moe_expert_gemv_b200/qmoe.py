@@ -680,7 +680,8 @@ def qmoe_set_decode_wait_limit_ns(ns):
     return int(lib().qmoe_set_decode_wait_limit_ns(int(ns)))
 
 
-# the library's threshold when the tensor-core prefill path is on
+# the threshold used when the tensor-core prefill path is switched on (the
+# library's own default is 0: off)
 TENSOR_MIN_DEFAULT = 16
 
 
