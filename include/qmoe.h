@@ -37,7 +37,10 @@
  *   - `stream` is a cudaStream_t (NULL: the legacy default stream).  Calls are
  *     asynchronous: they validate on the host, enqueue kernels and return.
  *     The library never allocates, frees or synchronises inside a compute
- *     call.  The current CUDA device must be the one that owns the pointers.
+ *     call, with one stated exception: moe_cache_layer synchronises its
+ *     stream once to read the router's choice on the host (its cache owns
+ *     device slots allocated by qmoe_cache_create).  The current CUDA device
+ *     must be the one that owns the pointers.
  *   - `status_dev` (optional, may be NULL) is a device int32 word that kernels
  *     OR device-detected problems into (QMOE_DEV_* flags).  With NULL the
  *     library's own per-device word is used.  qmoe_check_status() reads and
