@@ -16,15 +16,17 @@
 //   * Clusters of 8 CTAs (one CTA per SM).  Each CTA of a cluster holds E/8
 //     router rows in shared memory (loaded during the previous layer) and
 //     computes their logits; the logits meet in every CTA of the cluster
-//     through distributed shared memory, so each CTA takes the top-k itself
+//     through distributed shared memory (st.async stores that complete their
+//     bytes on the receiver's mbarrier), so each CTA takes the top-k itself
 //     without a grid-wide exchange.
 //   * Work is cut into units of (expert, 64 consecutive intermediate
 //     indices).  A unit belongs to ONE cluster: CTA r of the cluster computes
 //     the gate/up rows 8r..8r+7 of the unit and SwiGLU, sends its eight h
-//     values (as fp16 hi/lo pairs) to the 8 CTAs of the cluster and signals a
-//     remote mbarrier; each CTA then multiplies its own H/8 rows of the down
-//     projection by the unit's 64 h values.  The gate/up -> down dependency
-//     never leaves the cluster.
+//     values (as fp16 hi/lo pairs) to the other 7 CTAs of the cluster by
+//     st.async (their bytes complete the receiver's mbarrier of the unit);
+//     each CTA then multiplies its own H/8 rows of the down projection by the
+//     unit's 64 h values.  The gate/up -> down dependency never leaves the
+//     cluster.
 //   * Each CTA adds its weighted down rows of all its units in shared memory
 //     and then into an fp32 layer accumulator with one vector reduction per
 //     four rows; the thread that issued it then increments a grid-wide
@@ -37,17 +39,17 @@
 //     (every copy is one contiguous block of the packed layer) through a
 //     shared-memory ring, in the order the consumers use them: the shared
 //     expert's units need no routing and are fetched a layer ahead; the
-//     routed units are fetched as soon as the top-k is known.  The producer
-//     warp itself computes the top-k, since it is the one waiting for it.
+//     routed units are fetched expert by expert as the top-k rounds of the
+//     first exchange warp publish them.
 //   * 16 consumer warps in 4 groups; work item k of a layer goes to group
 //     k % 4 (gate/up items: the 4 warps split K; down items: the 4 warps
 //     split the rows).  Consumers hand partial sums over through shared
 //     memory and an mbarrier and move on: an exchange warp adds the router
 //     partials and sends the CTA's logits to the cluster, and adds each
 //     unit's gate/up partials, applies SwiGLU and sends the h values (four
-//     8-byte stores and one 4-byte store per destination CTA).  Remote
-//     stores wait on their acknowledgement; kept on one warp, that latency
-//     never holds a consumer group.
+//     8-byte st.async stores and one 4-byte one per destination CTA; no
+//     release fence or remote arrive is needed, the bytes themselves complete
+//     the receiver's barrier), so no consumer group waits on that traffic.
 //
 // The fp32 atomics make the last bits of a layer output depend on the order
 // in which clusters finish; routing, h and every per-CTA sum do not.

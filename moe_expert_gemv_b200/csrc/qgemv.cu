@@ -14,12 +14,14 @@
 // tracked by mbarriers: when the row length is a multiple of 128 bytes the
 // codes of a tile arrive in ONE 3-D TMA tensor copy with 128-byte swizzling
 // (a 32 KB tile at K = 4096, so the copy engine runs at full rate); otherwise
-// each row is a 1-D bulk copy into a padded row.  Sixteen consumer warps
-// split the tile's 64-wide groups (a contiguous block each), place the codes
-// in registers as exact fp16 values (the code bits as subnormals) and run
-// mma.sync m16n8k16 with the batch as the N=8 dimension; scale and bias are
-// applied per group in fp32; partial tiles are reduced through shared memory
-// and written as fp16.  x is staged once per CTA, one thread per (row, group).
+// each row is a 1-D bulk copy into a padded row.  Sixteen consumer warps form
+// tile groups of 4 (of 8 for a batch of 8); tile k goes to group k % groups,
+// and each warp of a group takes a contiguous block of the tile's 64-wide
+// groups, places the codes in registers as exact fp16 values (the code bits
+// as subnormals) and runs mma.sync m16n8k16 with the batch as the N=8
+// dimension; scale and bias are applied per group in fp32; the group's
+// partial sums meet at its own named barrier and are written as fp16.  x is
+// staged once per CTA, one thread per (row, group).
 #include <cuda.h>
 #include <string.h>
 
