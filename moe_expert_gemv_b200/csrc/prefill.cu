@@ -33,6 +33,8 @@
 // Every operand of the inner loops is in shared memory.  A light expert (at
 // most 8 tokens: most of them under skewed routing) is streamed from HBM
 // exactly once; a heavy one once per token tile, the repeats hitting L2.
+// Slots with at least qmoe_set_prefill_tensor_min tokens (0 by default: off)
+// skip steps 3 and 5 and run on the tcgen05 kernels of prefill_tc.cu.
 #include <cuda.h>
 #include <string.h>
 
